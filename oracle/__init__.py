@@ -1,0 +1,210 @@
+"""Float64 CPU oracle for depthwise 2-D convolution (forward and input gradient).
+
+TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and the CPU
+(reference / cpu_baseline) legs of ``bench.py`` may import this package; the
+product path never does.  The arithmetic lives in ``dw_oracle.c`` (plain C
+loops, float64); this module only compiles it with gcc and marshals numpy
+arrays through ctypes.  Nothing here is shared with the CUDA library.
+
+Source of every definition: page "LeanMlir Proofs/Architectures/Depthwise"
+(lean.brettkoonce.com), sections "Depthwise conv2d forward", "Closed-form
+input gradient ... direct formula", "Depthwise conv input-VJP", "Stride-2
+SAME depthwise conv" and "Stride-2 XLA-SAME depthwise conv".  Readings where
+the page leaves a step open (SAME at stride > 1, bias dtype, batch axis,
+layouts) are documented in ``dw_oracle.c``.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py
+(hand-derived golden values, dense grouped-conv library routine, adjoint
+identity, decimation identities, closed forms).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dw_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libdw_oracle.so")
+_lib = None
+
+LAYOUTS = {"nhwc": 0, "nchw": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile dw_oracle.c into oracle/libdw_oracle.so (gcc, -O2, OpenMP).
+
+    Floating-point contraction is disabled so every multiply and add rounds
+    to double exactly as written in the source.
+    """
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+           "-shared", "-fPIC", _SRC, "-o", tmp]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    i64, p_i64 = ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)
+    p_f64 = ctypes.POINTER(ctypes.c_double)
+    lib.dwo_out_extent.restype = i64
+    lib.dwo_out_extent.argtypes = [i64] * 6
+    lib.dwo_same_pads.restype = None
+    lib.dwo_same_pads.argtypes = [i64, i64, i64, i64, p_i64, p_i64]
+    lib.dwo_num_threads.restype = ctypes.c_int
+    lib.dwo_num_threads.argtypes = []
+    lib.dwo_fwd.restype = None
+    lib.dwo_fwd.argtypes = [p_i64, p_f64, p_f64, p_f64, p_f64]
+    lib.dwo_bwd_input.restype = None
+    lib.dwo_bwd_input.argtypes = [p_i64, p_f64, p_f64, p_f64]
+    lib.dwo_fwd_at.restype = None
+    lib.dwo_fwd_at.argtypes = [p_i64, p_f64, p_f64, p_f64, i64, p_i64, p_f64]
+    lib.dwo_bwd_input_at.restype = None
+    lib.dwo_bwd_input_at.argtypes = [p_i64, p_f64, p_f64, i64, p_i64, p_f64]
+    _lib = lib
+    return lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(_load().dwo_num_threads())
+
+
+def out_extent(n_in: int, k: int, s: int, d: int, lo: int, hi: int) -> int:
+    return int(_load().dwo_out_extent(n_in, k, s, d, lo, hi))
+
+
+def same_pads(n_in: int, k: int, s: int, d: int) -> tuple[int, int]:
+    lo, hi = ctypes.c_int64(), ctypes.c_int64()
+    _load().dwo_same_pads(n_in, k, s, d, ctypes.byref(lo), ctypes.byref(hi))
+    return int(lo.value), int(hi.value)
+
+
+def _pair(v):
+    return (int(v), int(v)) if np.isscalar(v) else (int(v[0]), int(v[1]))
+
+
+def resolve_pads(H, W, kH, kW, stride=1, dilation=1, padding="same"):
+    """(pt, pb, pl, pr) for padding "same" (XLA rule) or explicit.
+
+    Explicit padding is an int (all sides), a pair (vertical, horizontal) or a
+    4-tuple (top, bottom, left, right).
+    """
+    sh, sw = _pair(stride)
+    dh, dw = _pair(dilation)
+    if isinstance(padding, str):
+        if padding.lower() != "same":
+            raise ValueError(f"unknown padding mode {padding!r}")
+        pt, pb = same_pads(H, kH, sh, dh)
+        pl, pr = same_pads(W, kW, sw, dw)
+        return pt, pb, pl, pr
+    if np.isscalar(padding):
+        p = int(padding)
+        return p, p, p, p
+    padding = tuple(int(v) for v in padding)
+    if len(padding) == 2:
+        return padding[0], padding[0], padding[1], padding[1]
+    if len(padding) == 4:
+        return padding
+    raise ValueError(f"bad padding {padding!r}")
+
+
+def problem(shape, kH, kW, stride=1, dilation=1, padding="same", layout="nhwc"):
+    """int64[15] problem vector from an activation shape in `layout` order."""
+    layout = layout.lower()
+    if layout == "nhwc":
+        N, H, W, C = shape
+    elif layout == "nchw":
+        N, C, H, W = shape
+    else:
+        raise ValueError(layout)
+    sh, sw = _pair(stride)
+    dh, dw = _pair(dilation)
+    pt, pb, pl, pr = resolve_pads(H, W, kH, kW, stride, dilation, padding)
+    return np.array([N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr,
+                     LAYOUTS[layout]], dtype=np.int64)
+
+
+def out_shape(prob) -> tuple[int, ...]:
+    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, lay = (int(v) for v in prob)
+    Ho = out_extent(H, kH, sh, dh, pt, pb)
+    Wo = out_extent(W, kW, sw, dw, pl, pr)
+    return (N, Ho, Wo, C) if lay == 0 else (N, C, Ho, Wo)
+
+
+def in_shape(prob) -> tuple[int, ...]:
+    N, H, W, C = (int(v) for v in prob[:4])
+    return (N, H, W, C) if int(prob[14]) == 0 else (N, C, H, W)
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a, ty=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ty))
+
+
+def _weights(w, prob):
+    C, kH, kW = int(prob[3]), int(prob[4]), int(prob[5])
+    w = _f64(w).reshape(C, kH, kW)
+    return w
+
+
+def fwd(prob, x, w, b=None):
+    """y = depthwise forward (float64) for problem vector `prob`."""
+    prob = np.ascontiguousarray(prob, dtype=np.int64)
+    x = _f64(x).reshape(in_shape(prob))
+    w = _weights(w, prob)
+    bb = None if b is None else _f64(b).reshape(int(prob[3]))
+    y = np.empty(out_shape(prob), dtype=np.float64)
+    _load().dwo_fwd(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(w),
+                    None if bb is None else _ptr(bb), _ptr(y))
+    return y
+
+
+def bwd_input(prob, dy, w):
+    """dx = transpose of the forward's linear part applied to dy (float64)."""
+    prob = np.ascontiguousarray(prob, dtype=np.int64)
+    dy = _f64(dy).reshape(out_shape(prob))
+    w = _weights(w, prob)
+    dx = np.empty(in_shape(prob), dtype=np.float64)
+    _load().dwo_bwd_input(_ptr(prob, ctypes.c_int64), _ptr(dy), _ptr(w), _ptr(dx))
+    return dx
+
+
+def fwd_at(prob, x, w, b, flat_idx):
+    """Forward output at the given flat indices of y (layout order)."""
+    prob = np.ascontiguousarray(prob, dtype=np.int64)
+    x = _f64(x).reshape(in_shape(prob))
+    w = _weights(w, prob)
+    bb = None if b is None else _f64(b).reshape(int(prob[3]))
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    out = np.empty(idx.shape[0], dtype=np.float64)
+    _load().dwo_fwd_at(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(w),
+                       None if bb is None else _ptr(bb), idx.shape[0],
+                       _ptr(idx, ctypes.c_int64), _ptr(out))
+    return out
+
+
+def bwd_input_at(prob, dy, w, flat_idx):
+    """Input gradient at the given flat indices of dx, by the direct formula."""
+    prob = np.ascontiguousarray(prob, dtype=np.int64)
+    dy = _f64(dy).reshape(out_shape(prob))
+    w = _weights(w, prob)
+    idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
+    out = np.empty(idx.shape[0], dtype=np.float64)
+    _load().dwo_bwd_input_at(_ptr(prob, ctypes.c_int64), _ptr(dy), _ptr(w),
+                             idx.shape[0], _ptr(idx, ctypes.c_int64), _ptr(out))
+    return out
