@@ -1,0 +1,143 @@
+// Internal declarations shared by the CUDA translation units of libdwconv2d.
+// Nothing here is part of the public ABI (see include/dwconv2d.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dwconv2d.h"
+
+namespace dw {
+
+// A resolved problem: everything the kernels need, pads already resolved.
+// H, W, C, N are the extents of x (forward input) / dx (gradient output);
+// Ho, Wo the extents of y / dy.
+struct Problem {
+    int64_t N, H, W, C, Ho, Wo;
+    int kH, kW, sh, sw, dh, dw;
+    int pt, pb, pl, pr;
+    int layout;  // DW_NHWC / DW_NCHW
+    int wtype;   // DW_F32 / DW_F16
+};
+
+enum Op { OP_FWD = 0, OP_BWD_INPUT = 1 };
+
+// Launch entry points of each kernel family.  `dry_run` only answers whether
+// the family covers the problem (DW_OK / DW_ERR_UNSUPPORTED) without touching
+// the device.
+dw_status_t direct_launch(const Problem& p, Op op, const float* in, const void* w,
+                          const float* b, float* out, cudaStream_t stream);
+dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const float* in, const void* w,
+                              const float* b, float* out, cudaStream_t stream,
+                              int32_t* dev_err, bool dry_run);
+dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const void* w,
+                              const float* b, float* out, cudaStream_t stream,
+                              int32_t* dev_err, bool dry_run);
+
+// Host helpers (dw_host.cu).
+int current_device();
+int sm_count(int dev);
+// cuTensorMapEncodeTiled fetched through the runtime (no link-time libcuda
+// dependency, so the library also loads on machines without a driver).
+CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank,
+                           void* base, const cuuint64_t* dims, const cuuint64_t* strides,
+                           const cuuint32_t* box, const cuuint32_t* elem_strides);
+
+// Per (kernel instantiation, device) cache of the launch attributes.
+struct LaunchCache {
+    int occupancy[64];  // 0 = not queried yet
+};
+// Sets the dynamic shared memory limit once and returns resident CTAs per SM
+// (0 if the kernel cannot be resident at all).
+int prepare_kernel(const void* kernel, int threads, size_t smem_bytes, LaunchCache& cache,
+                   int dev);
+
+// ------------------------------------------------------------------ device --
+
+__device__ __forceinline__ float load_weight(const void* w, int wtype, int64_t idx) {
+    // float16 -> float32 widening is exact, so both weight types feed the
+    // same float32 FMA sequence.
+    return wtype == DW_F16 ? __half2float(static_cast<const __half*>(w)[idx])
+                           : static_cast<const float*>(w)[idx];
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Every wait on an asynchronous copy is bounded: after kWaitLimitNs without
+// completion it reports failure instead of spinning forever.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// 4-D tiled TMA load (no multicast) into this CTA's shared memory; completion
+// is signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fma4(float4& acc, const float4& v, const float4& w) {
+    acc.x = fmaf(v.x, w.x, acc.x);
+    acc.y = fmaf(v.y, w.y, acc.y);
+    acc.z = fmaf(v.z, w.z, acc.z);
+    acc.w = fmaf(v.w, w.w, acc.w);
+}
+
+__device__ __forceinline__ void store4(float* p, const float4& v) {
+    *reinterpret_cast<float4*>(p) = v;
+}
+
+}  // namespace dw

@@ -1,0 +1,318 @@
+// NCHW tiled kernels (stride 1): W innermost, TMA halo tiles, persistent CTAs.
+//
+// Each (n, c) plane is an independent image with its own filter (page
+// "LeanMlir Proofs/Architectures/Depthwise", comparison with regular conv2d:
+// no cross-channel mixing).  Lanes run along W: a thread owns 4 consecutive
+// outputs of a row (one float4) and THT rows, so a warp covers 128 columns
+// with 16-byte accesses on both the shared-memory reads and the global
+// stores.  For kH > 1 a CTA tile is TH x 128 outputs of one plane and its
+// input halo [TH + (kH-1)D][IWB] comes in one TMA load; for kH = 1 (the long
+// 1-D kernels) a tile is one row of 128 outputs in WY consecutive channels and
+// the TMA box spans those channels instead of rows.  TMA boxes must start on a
+// 16-byte boundary, so the box starts REM = (-pl) mod 4 columns left of the
+// first input column a tile needs; REM is a template parameter and every
+// thread's window is read as aligned float4s and indexed at compile time.
+// Taps sit in registers (per thread: the filter of its plane), streamed in
+// kh-major, kw-minor order per output.
+//
+// Modes: forward (y from x, pads pt/pl); reversed (input gradient at stride
+// 1: dx from dy with the reversed filter and the complementary pads
+// (kH-1)D - pt, (kW-1)D - pl; "Closed-form input gradient", reversed-kernel
+// form).
+#include <climits>
+#include <type_traits>
+
+#include "dw_common.cuh"
+
+namespace dw {
+namespace nchw {
+
+struct Args {
+    const void* w;
+    const float* b;
+    float* out;
+    int32_t* err;
+    int wtype;
+    int N, C, Hout, Wout;
+    int pt, pl;  // effective low pads of the correlation this kernel runs
+    int tiles_x, tiles_y, tiles_c;
+    int ntiles;
+};
+
+template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_>
+struct Cfg {
+    static constexpr int KH = KH_, KW = KW_, D = D_, REM = REM_;
+    static constexpr bool REV = REV_;
+    static constexpr bool ROWS = KH == 1;  // 1-D: thread rows are channels
+    static constexpr int THT = ROWS ? 1 : THT_, WX = WX_, WY = WY_, NS = NS_;
+    static constexpr int NT = WX * WY;
+    static constexpr int TW = 4 * WX;
+    static constexpr int TH = ROWS ? 1 : THT * WY;
+    static constexpr int IH = ROWS ? 1 : TH + (KH - 1) * D;
+    static constexpr int IWB = (REM + TW + (KW - 1) * D + 3) / 4 * 4;
+    static constexpr int BOXH = IH;
+    static constexpr int BOXC = ROWS ? WY : 1;
+    static constexpr int STAGE_FLOATS = IWB * IH * BOXC;
+    static constexpr int STAGE_BYTES = STAGE_FLOATS * 4;
+    static constexpr int RH = THT + (KH - 1) * D;           // window rows
+    static constexpr int NV = (REM + 3 + (KW - 1) * D) / 4 + 1;  // float4 per window row
+    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(NS) * 8;
+    static_assert(IWB <= 256 && IH <= 256 && BOXC <= 256, "TMA box dimension limit");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <int I, int N, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for<I + 1, N>(f);
+    }
+}
+
+// tile t -> (tx, ty or output row h, plane or channel group, n)
+template <class K>
+__device__ __forceinline__ void decode_tile(int t, const Args& a, int& tx, int& ty, int& c,
+                                            int& n) {
+    tx = t % a.tiles_x;
+    t /= a.tiles_x;
+    ty = t % a.tiles_y;  // ROWS: output row h
+    t /= a.tiles_y;
+    c = t % a.tiles_c;   // ROWS: channel group; else channel
+    n = t / a.tiles_c;
+}
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    float* stages = reinterpret_cast<float*>(smem);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+
+    const int tid = threadIdx.x;
+    const int xi = tid % K::WX;
+    const int yi = tid / K::WX;
+    // contiguous range of tiles for this CTA: neighbouring tiles share a
+    // plane (filter stays in registers) and their halos (L2 hits)
+    const int t_begin = int((int64_t(blockIdx.x) * a.ntiles) / gridDim.x);
+    const int t_end = int((int64_t(blockIdx.x + 1) * a.ntiles) / gridDim.x);
+
+    if (tid == 0) {
+        prefetch_tensor_map(&tmap);
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int s, int t) {
+        int tx, ty, c, n;
+        decode_tile<K>(t, a, tx, ty, c, n);
+        const int ix0 = tx * K::TW - a.pl - K::REM;
+        mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+        if constexpr (K::ROWS)
+            tma_load_4d(stages + size_t(s) * K::STAGE_FLOATS, &tmap, &full[s], ix0, ty - a.pt,
+                        c * K::WY, n);
+        else
+            tma_load_4d(stages + size_t(s) * K::STAGE_FLOATS, &tmap, &full[s], ix0,
+                        ty * K::TH - a.pt, c, n);
+    };
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s)
+            if (t_begin + s < t_end) issue(s, t_begin + s);
+    }
+
+    float wr[K::KH][K::KW];
+    float bias = 0.f;
+    int cur_key = -1;
+    bool live = false;
+
+    int k = 0;
+    for (int t = t_begin; t < t_end; ++t, ++k) {
+        const int s = k % K::NS;
+        const uint32_t parity = (k / K::NS) & 1;
+        int tx, ty, cg, n;
+        decode_tile<K>(t, a, tx, ty, cg, n);
+        const int c = K::ROWS ? cg * K::WY + yi : cg;
+        const int key = cg + n * a.tiles_c;
+        if (key != cur_key) {
+            cur_key = key;
+            live = c < a.C;
+            const int64_t base = int64_t(live ? c : 0) * (K::KH * K::KW);
+#pragma unroll
+            for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw) {
+                    const int src = K::REV ? (K::KH - 1 - kh) * K::KW + (K::KW - 1 - kw)
+                                           : kh * K::KW + kw;
+                    wr[kh][kw] = live ? load_weight(a.w, a.wtype, base + src) : 0.f;
+                }
+            bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
+        }
+
+        const bool ok = mbar_wait_bounded(&full[s], parity);
+
+        float acc[K::THT][4];
+#pragma unroll
+        for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+
+        const int row0 = K::ROWS ? yi : yi * K::THT;
+        const float4* win = reinterpret_cast<const float4*>(stages + size_t(s) * K::STAGE_FLOATS +
+                                                            size_t(row0) * K::IWB) + xi;
+        static_for<0, K::RH>([&](auto r_) {
+            constexpr int r = decltype(r_)::value;
+            float v[4 * K::NV];
+#pragma unroll
+            for (int u = 0; u < K::NV; ++u) {
+                const float4 f = win[r * (K::IWB / 4) + u];
+                v[4 * u] = f.x;
+                v[4 * u + 1] = f.y;
+                v[4 * u + 2] = f.z;
+                v[4 * u + 3] = f.w;
+            }
+            static_for<0, K::THT>([&](auto j_) {
+                constexpr int j = decltype(j_)::value;
+                constexpr int khn = r - j;
+                if constexpr (khn >= 0 && khn % K::D == 0 && khn / K::D < K::KH) {
+                    constexpr int kh = khn / K::D;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int kw = 0; kw < K::KW; ++kw)
+                            acc[j][i] = fmaf(v[K::REM + i + kw * K::D], wr[kh][kw], acc[j][i]);
+                }
+            });
+        });
+
+        if (live) {
+            const int wo0 = tx * K::TW + 4 * xi;
+#pragma unroll
+            for (int j = 0; j < K::THT; ++j) {
+                const int ho = K::ROWS ? ty : ty * K::TH + row0 + j;
+                if (ho >= a.Hout) continue;
+                float* dst = a.out + ((int64_t(n) * a.C + c) * a.Hout + ho) * a.Wout + wo0;
+                const float4 v = make_float4(acc[j][0] + bias, acc[j][1] + bias, acc[j][2] + bias,
+                                             acc[j][3] + bias);
+                if ((a.Wout & 3) == 0 && wo0 + 3 < a.Wout) {
+                    store4(dst, v);
+                } else {
+                    if (wo0 < a.Wout) dst[0] = v.x;
+                    if (wo0 + 1 < a.Wout) dst[1] = v.y;
+                    if (wo0 + 2 < a.Wout) dst[2] = v.z;
+                    if (wo0 + 3 < a.Wout) dst[3] = v.w;
+                }
+            }
+        }
+
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = 1; j < K::NS; ++j) {
+                    const int k2 = k + j;
+                    if (t + j < t_end) mbar_wait_bounded(&full[k2 % K::NS], (k2 / K::NS) & 1);
+                }
+            }
+            return;
+        }
+        if (tid == 0 && t + K::NS < t_end) issue(s, t + K::NS);
+    }
+}
+
+template <class K>
+dw_status_t launch(const Problem& p, const float* in, const void* w, const float* b, float* out,
+                   cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff, int pl_eff) {
+    const int64_t Hin = K::REV ? p.Ho : p.H, Win = K::REV ? p.Wo : p.W;
+    Args a;
+    a.w = w;
+    a.b = K::REV ? nullptr : b;
+    a.out = out;
+    a.err = err;
+    a.wtype = p.wtype;
+    a.N = static_cast<int>(p.N);
+    a.C = static_cast<int>(p.C);
+    a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
+    a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
+    a.pt = pt_eff;
+    a.pl = pl_eff;
+    const int64_t tx = (a.Wout + K::TW - 1) / K::TW;
+    const int64_t ty = K::ROWS ? a.Hout : (a.Hout + K::TH - 1) / K::TH;
+    const int64_t tc = K::ROWS ? (p.C + K::WY - 1) / K::WY : p.C;
+    const int64_t nt = tx * ty * tc * p.N;
+    if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.tiles_x = static_cast<int>(tx);
+    a.tiles_y = static_cast<int>(ty);
+    a.tiles_c = static_cast<int>(tc);
+    a.ntiles = static_cast<int>(nt);
+    if (dry_run) return DW_OK;
+
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&tiled_kernel<K>), K::NT,
+                                   K::SMEM, cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+
+    CUtensorMap map;
+    const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t strides[3] = {cuuint64_t(Win) * 4, cuuint64_t(Win * Hin) * 4,
+                                   cuuint64_t(Win * Hin * p.C) * 4};
+    const cuuint32_t box[4] = {K::IWB, K::BOXH, K::BOXC, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
+                          strides, box, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+    int64_t grid = int64_t(sm_count(dev)) * occ;
+    if (grid > a.ntiles) grid = a.ntiles;
+    tiled_kernel<K><<<static_cast<unsigned>(grid), K::NT, K::SMEM, stream>>>(map, a);
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS>
+dw_status_t launch_rem(const Problem& p, const float* in, const void* w, const float* b,
+                       float* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
+                       int pl_eff) {
+    const int rem = ((-pl_eff) % 4 + 4) % 4;
+    switch (rem) {
+        case 0: return launch<Cfg<KH, KW, 1, REV, 0, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 1: return launch<Cfg<KH, KW, 1, REV, 1, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 2: return launch<Cfg<KH, KW, 1, REV, 2, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        default: return launch<Cfg<KH, KW, 1, REV, 3, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+    }
+}
+
+template <int KH, int KW, int THT, int WX, int WY, int NS>
+dw_status_t launch_op(const Problem& p, Op op, const float* in, const void* w, const float* b,
+                      float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (op == OP_FWD)
+        return launch_rem<KH, KW, false, THT, WX, WY, NS>(p, in, w, b, out, stream, err, dry_run,
+                                                          p.pt, p.pl);
+    return launch_rem<KH, KW, true, THT, WX, WY, NS>(p, in, w, b, out, stream, err, dry_run,
+                                                     (KH - 1) - p.pt, (KW - 1) - p.pl);
+}
+
+}  // namespace nchw
+
+dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const void* w,
+                              const float* b, float* out, cudaStream_t stream, int32_t* err,
+                              bool dry_run) {
+    using namespace nchw;
+    if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
+    if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
+    const int64_t Win = op == OP_FWD ? p.W : p.Wo;
+    if (Win % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row stride: 16-byte multiple
+    if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return DW_ERR_UNSUPPORTED;
+    if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.C >= INT_MAX ||
+        p.Ho >= INT_MAX || p.Wo >= INT_MAX)
+        return DW_ERR_UNSUPPORTED;
+    //                                                   KH  KW THT WX  WY NS
+    if (p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 7 && p.kW == 7) return launch_op<7, 7, 4, 32, 4, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 1 && p.kW == 15) return launch_op<1, 15, 1, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 1 && p.kW == 31) return launch_op<1, 31, 1, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
+}  // namespace dw

@@ -1,0 +1,387 @@
+// NHWC tiled kernels: channels innermost, TMA halo tiles, persistent CTAs.
+//
+// Layout and mapping (page "cubek_convolution kernels::forward::depthwise",
+// module text: the channel axis is a batch axis, channels stay innermost and
+// consecutive lanes read consecutive channels of one pixel; the pass is
+// bandwidth-bound).  A CTA tile is TH x TW output pixels x 32 channels.  Each
+// lane owns 4 consecutive channels (one float4), 8 lanes cover the 32
+// channels of a pixel, so a quarter-warp reads or writes 128 contiguous
+// bytes.  The input halo tile [IH][IW][32] of every output tile is fetched by
+// one 4-D TMA load (zero fill outside the tensor == zero padding) into a ring
+// of NS shared-memory stages; a persistent CTA walks its tiles while the next
+// NS-1 loads are in flight.  Filter taps and bias of the CTA's 32 channels sit
+// in registers.  Each thread computes a THT x TWT block of outputs: it streams
+// the input cells of its block's window once from shared memory and feeds
+// every (output, tap) pair that reads that cell - a register sliding window
+// in both directions, resolved at compile time.
+//
+// Forward (LeanMlir Proofs/Architectures/Depthwise, "Depthwise conv2d
+// forward"): output (ho,wo) reads input (ho*S + kh*D - pt, wo*S + kw*D - pl);
+// stride and dilation are part of the index map (no decimation pass).
+// Transposed mode = input gradient ("Closed-form input gradient ... direct
+// formula" and the stride-2 input-VJP sections): dx tile rows start at
+// hi0 = ty*TH - (pt mod S) so that hi + pt is a multiple of S at the tile
+// origin; dx(hi) gathers W[kh] * dy((hi + pt - kh*D)/S) for the kh where the
+// division is exact - the zero-upsampled, reversed-kernel correlation without
+// the upsampled tensor.  At S = 1 this is the reversed kernel with the
+// complementary pad (kH-1)*D - pt.
+#include <climits>
+#include <type_traits>
+
+#include "dw_common.cuh"
+
+namespace dw {
+namespace nhwc {
+
+constexpr int CB = 32;      // channels per tile
+constexpr int CV = CB / 4;  // float4 lanes per pixel
+
+struct Args {
+    const void* w;
+    const float* b;
+    float* out;
+    int32_t* err;
+    int wtype;
+    int C;
+    int Hout, Wout;  // extents of the tensor written
+    int pt, pl;      // forward low pads
+    int org_y, org_x;
+    int tiles_x, tiles_y, tiles_c;
+    int ntiles;
+};
+
+template <int KH_, int KW_, int S_, int D_, bool TR_, int THT_, int TWT_, int WX_, int WY_, int NS_>
+struct Cfg {
+    static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
+    static constexpr bool TR = TR_;
+    static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
+    static constexpr int NT = CV * WX * WY;
+    static constexpr int TH = THT * WY, TW = TWT * WX;
+    static constexpr int AH = TR ? ((KH - 1) * D + S - 1) / S : 0;
+    static constexpr int AW = TR ? ((KW - 1) * D + S - 1) / S : 0;
+    static constexpr int IH = TR ? AH + TH / S : (TH - 1) * S + (KH - 1) * D + 1;
+    static constexpr int IW = TR ? AW + TW / S : (TW - 1) * S + (KW - 1) * D + 1;
+    // rows / columns of the input window one thread reads
+    static constexpr int RH = TR ? AH + (THT - 1) / S + 1 : (THT - 1) * S + (KH - 1) * D + 1;
+    static constexpr int RW = TR ? AW + (TWT - 1) / S + 1 : (TWT - 1) * S + (KW - 1) * D + 1;
+    static constexpr int STAGE_F4 = IH * IW * CV;
+    static constexpr int STAGE_BYTES = STAGE_F4 * 16;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(NS) * 8;
+    static_assert(IH <= 256 && IW <= 256, "TMA box dimension limit");
+    static_assert(!TR || (THT % S == 0 && TWT % S == 0), "transposed blocks are phase aligned");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <int I, int N, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for<I + 1, N>(f);
+    }
+}
+
+// Tap index that maps output offset j (within a thread block) to window
+// row r, or -1.  Forward: r = j*S + k*D.  Transposed: r - A = (j - k*D)/S
+// with exact division.
+template <class K, bool ROW>
+__host__ __device__ constexpr int tap_for(int r, int j) {
+    constexpr int Kn = ROW ? K::KH : K::KW;
+    constexpr int A = ROW ? K::AH : K::AW;
+    if constexpr (!K::TR) {
+        const int num = r - j * K::S;
+        if (num < 0 || num % K::D != 0 || num / K::D >= Kn) return -1;
+        return num / K::D;
+    } else {
+        for (int k = 0; k < Kn; ++k) {
+            const int num = j - k * K::D;  // must be (r - A) * S
+            if (num == (r - A) * K::S) return k;
+        }
+        return -1;
+    }
+}
+
+__device__ __forceinline__ void decode_tile(int t, const Args& a, int& cb, int& tx, int& ty,
+                                            int& n) {
+    cb = t % a.tiles_c;
+    t /= a.tiles_c;
+    tx = t % a.tiles_x;
+    t /= a.tiles_x;
+    ty = t % a.tiles_y;
+    n = t / a.tiles_y;
+}
+
+template <class K>
+__device__ __forceinline__ void tile_origin(const Args& a, int tx, int ty, int& oy0, int& ox0,
+                                            int& iy0, int& ix0) {
+    if constexpr (!K::TR) {
+        oy0 = ty * K::TH;
+        ox0 = tx * K::TW;
+        iy0 = oy0 * K::S - a.pt;
+        ix0 = ox0 * K::S - a.pl;
+    } else {
+        oy0 = ty * K::TH - a.org_y;
+        ox0 = tx * K::TW - a.org_x;
+        iy0 = (oy0 + a.pt) / K::S - K::AH;  // oy0 + pt >= 0 and divisible by S
+        ix0 = (ox0 + a.pl) / K::S - K::AW;
+    }
+}
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    float4* stages = reinterpret_cast<float4*>(smem);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+
+    const int tid = threadIdx.x;
+    const int cv = tid % CV;
+    const int xi = (tid / CV) % K::WX;
+    const int yi = tid / (CV * K::WX);
+    const int G = gridDim.x;
+
+    if (tid == 0) {
+        prefetch_tensor_map(&tmap);
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int s, int t) {
+        int cb, tx, ty, n, oy0, ox0, iy0, ix0;
+        decode_tile(t, a, cb, tx, ty, n);
+        tile_origin<K>(a, tx, ty, oy0, ox0, iy0, ix0);
+        mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+        tma_load_4d(stages + size_t(s) * K::STAGE_F4, &tmap, &full[s], cb * CB, ix0, iy0, n);
+    };
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) {
+            const int t = blockIdx.x + s * G;
+            if (t < a.ntiles) issue(s, t);
+        }
+    }
+
+    float4 wr[K::KH][K::KW];
+    float4 bias = make_float4(0.f, 0.f, 0.f, 0.f);
+    int cur_cb = -1;
+    // window origin of this thread inside a stage
+    const int r0 = K::TR ? yi * (K::THT / K::S) : yi * K::THT * K::S;
+    const int q0 = K::TR ? xi * (K::TWT / K::S) : xi * K::TWT * K::S;
+    const int j0 = yi * K::THT, i0 = xi * K::TWT;
+
+    int k = 0;
+    for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
+        const int s = k % K::NS;
+        const uint32_t parity = (k / K::NS) & 1;
+        int cb, tx, ty, n, oy0, ox0, iy0, ix0;
+        decode_tile(t, a, cb, tx, ty, n);
+        tile_origin<K>(a, tx, ty, oy0, ox0, iy0, ix0);
+        const int c = cb * CB + cv * 4;
+        if (cb != cur_cb) {
+            cur_cb = cb;
+            const bool live = c < a.C;
+#pragma unroll
+            for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw) {
+                    const int64_t o = int64_t(c) * (K::KH * K::KW) + kh * K::KW + kw;
+                    constexpr int step = K::KH * K::KW;
+                    wr[kh][kw] = live ? make_float4(load_weight(a.w, a.wtype, o),
+                                                    load_weight(a.w, a.wtype, o + step),
+                                                    load_weight(a.w, a.wtype, o + 2 * step),
+                                                    load_weight(a.w, a.wtype, o + 3 * step))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            if (!K::TR && a.b != nullptr && live)
+                bias = make_float4(__ldg(a.b + c), __ldg(a.b + c + 1), __ldg(a.b + c + 2),
+                                   __ldg(a.b + c + 3));
+        }
+
+        const bool ok = mbar_wait_bounded(&full[s], parity);
+
+        float4 acc[K::THT][K::TWT];
+#pragma unroll
+        for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+            for (int i = 0; i < K::TWT; ++i) acc[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+        const float4* win = stages + size_t(s) * K::STAGE_F4 + (r0 * K::IW + q0) * CV + cv;
+        static_for<0, K::RH>([&](auto r_) {
+            constexpr int r = decltype(r_)::value;
+            static_for<0, K::RW>([&](auto q_) {
+                constexpr int q = decltype(q_)::value;
+                // does any (output, tap) pair of this thread read cell (r,q)?
+                constexpr bool used = [] {
+                    for (int j = 0; j < K::THT; ++j)
+                        for (int i = 0; i < K::TWT; ++i)
+                            if (tap_for<K, true>(r, j) >= 0 && tap_for<K, false>(q, i) >= 0)
+                                return true;
+                    return false;
+                }();
+                if constexpr (used) {
+                    const float4 v = win[(r * K::IW + q) * CV];
+                    static_for<0, K::THT>([&](auto j_) {
+                        constexpr int j = decltype(j_)::value;
+                        constexpr int kh = tap_for<K, true>(r, j);
+                        if constexpr (kh >= 0) {
+                            static_for<0, K::TWT>([&](auto i_) {
+                                constexpr int i = decltype(i_)::value;
+                                constexpr int kw = tap_for<K, false>(q, i);
+                                if constexpr (kw >= 0) fma4(acc[j][i], v, wr[kh][kw]);
+                            });
+                        }
+                    });
+                }
+            });
+        });
+
+        if (c < a.C) {
+#pragma unroll
+            for (int j = 0; j < K::THT; ++j) {
+                const int ho = oy0 + j0 + j;
+                if (ho < 0 || ho >= a.Hout) continue;
+#pragma unroll
+                for (int i = 0; i < K::TWT; ++i) {
+                    const int wo = ox0 + i0 + i;
+                    if (wo < 0 || wo >= a.Wout) continue;
+                    float4 v = acc[j][i];
+                    if (!K::TR) {
+                        v.x += bias.x; v.y += bias.y; v.z += bias.z; v.w += bias.w;
+                    }
+                    store4(a.out + ((int64_t(n) * a.Hout + ho) * a.Wout + wo) * a.C + c, v);
+                }
+            }
+        }
+
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = 1; j < K::NS; ++j) {  // let issued copies land
+                    const int t2 = t + j * G, k2 = k + j;
+                    if (t2 < a.ntiles) mbar_wait_bounded(&full[k2 % K::NS], (k2 / K::NS) & 1);
+                }
+            }
+            return;
+        }
+        if (tid == 0) {
+            const int tn = t + K::NS * G;
+            if (tn < a.ntiles) issue(s, tn);
+        }
+    }
+}
+
+template <class K>
+dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, const float* b,
+                   float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    const bool tr = op == OP_BWD_INPUT;
+    if (tr != K::TR) return DW_ERR_UNSUPPORTED;
+    Args a;
+    a.w = w;
+    a.b = tr ? nullptr : b;
+    a.out = out;
+    a.err = err;
+    a.wtype = p.wtype;
+    a.C = static_cast<int>(p.C);
+    a.Hout = static_cast<int>(tr ? p.H : p.Ho);
+    a.Wout = static_cast<int>(tr ? p.W : p.Wo);
+    a.pt = p.pt;
+    a.pl = p.pl;
+    a.org_y = tr ? p.pt % K::S : 0;
+    a.org_x = tr ? p.pl % K::S : 0;
+    const int64_t ty = (a.Hout + a.org_y + K::TH - 1) / K::TH;
+    const int64_t tx = (a.Wout + a.org_x + K::TW - 1) / K::TW;
+    const int64_t tc = (p.C + CB - 1) / CB;
+    const int64_t nt = ty * tx * tc * p.N;
+    if (nt >= INT_MAX || ty >= INT_MAX || tx >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.tiles_y = static_cast<int>(ty);
+    a.tiles_x = static_cast<int>(tx);
+    a.tiles_c = static_cast<int>(tc);
+    a.ntiles = static_cast<int>(nt);
+    if (dry_run) return DW_OK;
+
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&tiled_kernel<K>), K::NT,
+                                   K::SMEM, cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+
+    const int64_t Hin = tr ? p.Ho : p.H, Win = tr ? p.Wo : p.W;
+    CUtensorMap map;
+    const cuuint64_t dims[4] = {cuuint64_t(p.C), cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.N)};
+    const cuuint64_t strides[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * Win) * 4,
+                                   cuuint64_t(p.C * Win * Hin) * 4};
+    const cuuint32_t box[4] = {CB, K::IW, K::IH, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
+                          strides, box, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+
+    int64_t grid = int64_t(sm_count(dev)) * occ;
+    // keep each CTA on one channel block (weights loaded once per CTA)
+    if (grid >= a.tiles_c) grid -= grid % a.tiles_c;
+    if (grid > a.ntiles) grid = a.ntiles;
+    if (grid < 1) grid = 1;
+    tiled_kernel<K><<<static_cast<unsigned>(grid), K::NT, K::SMEM, stream>>>(map, a);
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+// Instantiated configurations:   KH KW  S  D  TR   THT TWT WX WY NS
+using F33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4>;
+using F33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4>;
+using F33d2 = Cfg<3, 3, 1, 2, false, 2, 4, 8, 4, 3>;
+using F33d3 = Cfg<3, 3, 1, 3, false, 2, 4, 8, 4, 3>;
+using F55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 3>;
+using F1x3 = Cfg<1, 3, 1, 1, false, 1, 8, 16, 1, 4>;
+using F1x5 = Cfg<1, 5, 1, 1, false, 1, 8, 16, 1, 4>;
+using F1x7 = Cfg<1, 7, 1, 1, false, 1, 8, 16, 1, 4>;
+using F1x15 = Cfg<1, 15, 1, 1, false, 1, 8, 16, 1, 4>;
+using F1x31 = Cfg<1, 31, 1, 1, false, 1, 8, 16, 1, 4>;
+using B33s1 = Cfg<3, 3, 1, 1, true, 2, 4, 8, 4, 4>;
+using B33s2 = Cfg<3, 3, 2, 1, true, 4, 4, 8, 4, 4>;
+using B33d2 = Cfg<3, 3, 1, 2, true, 2, 4, 8, 4, 3>;
+using B33d3 = Cfg<3, 3, 1, 3, true, 2, 4, 8, 4, 3>;
+using B55s1 = Cfg<5, 5, 1, 1, true, 2, 4, 8, 4, 3>;
+using B1x3 = Cfg<1, 3, 1, 1, true, 1, 8, 16, 1, 4>;
+using B1x5 = Cfg<1, 5, 1, 1, true, 1, 8, 16, 1, 4>;
+using B1x7 = Cfg<1, 7, 1, 1, true, 1, 8, 16, 1, 4>;
+using B1x15 = Cfg<1, 15, 1, 1, true, 1, 8, 16, 1, 4>;
+using B1x31 = Cfg<1, 31, 1, 1, true, 1, 8, 16, 1, 4>;
+
+}  // namespace nhwc
+
+dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const float* in, const void* w,
+                              const float* b, float* out, cudaStream_t stream, int32_t* err,
+                              bool dry_run) {
+    using namespace nhwc;
+    if (p.layout != DW_NHWC) return DW_ERR_UNSUPPORTED;
+    // TMA needs 16-byte aligned base and row strides; float4 stores need an
+    // aligned output.
+    if (p.C % 4 != 0) return DW_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return DW_ERR_UNSUPPORTED;
+    if (p.sh != p.sw || p.dh != p.dw) return DW_ERR_UNSUPPORTED;
+    if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.C >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    const int S = p.sh, D = p.dh;
+    const bool f = op == OP_FWD;
+#define DW_TRY(KH_, KW_, S_, D_, FC, BC)                                               \
+    if (p.kH == KH_ && p.kW == KW_ && S == S_ && D == D_)                                \
+        return f ? launch<FC>(p, op, in, w, b, out, stream, err, dry_run)              \
+                 : launch<BC>(p, op, in, w, b, out, stream, err, dry_run);
+    DW_TRY(3, 3, 1, 1, F33s1, B33s1)
+    DW_TRY(3, 3, 1, 2, F33d2, B33d2)
+    DW_TRY(3, 3, 1, 3, F33d3, B33d3)
+    DW_TRY(5, 5, 1, 1, F55s1, B55s1)
+    DW_TRY(1, 3, 1, 1, F1x3, B1x3)
+    DW_TRY(1, 5, 1, 1, F1x5, B1x5)
+    DW_TRY(1, 7, 1, 1, F1x7, B1x7)
+    DW_TRY(1, 15, 1, 1, F1x15, B1x15)
+    DW_TRY(1, 31, 1, 1, F1x31, B1x31)
+#undef DW_TRY
+    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1)
+        return f ? launch<F33s2>(p, op, in, w, b, out, stream, err, dry_run)
+                 : launch<B33s2>(p, op, in, w, b, out, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
+}  // namespace dw

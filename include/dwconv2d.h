@@ -1,0 +1,175 @@
+/*
+ * dwconv2d.h - depthwise 2-D convolution on NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The operation (page "LeanMlir Proofs/Architectures/Depthwise",
+ * lean.brettkoonce.com, section "Depthwise conv2d forward"), generalised to a
+ * batch axis, stride s, dilation d and per-side padding:
+ *
+ *   y[n,ho,wo,c] = sum_{kh<kH, kw<kW} X(n, ho*sh + kh*dh - pt,
+ *                                         wo*sw + kw*dw - pl, c) * W[c,kh,kw]
+ *                  + b[c]
+ *
+ * where X is x inside [0,H) x [0,W) and 0 outside (zero padding).  It is a
+ * cross-correlation (the kernel is not flipped) and has no cross-channel
+ * mixing: channel c of y reads only channel c of x and filter c.  The input
+ * gradient (sections "Closed-form input gradient ... direct formula" and
+ * "Depthwise conv input-VJP") is the transpose of the linear part:
+ *
+ *   dx[n,hi,wi,c] = sum over (kh,kw) with hi + pt - kh*dh = ho*sh,
+ *                   wi + pl - kw*dw = wo*sw, 0 <= ho < Ho, 0 <= wo < Wo
+ *                   of W[c,kh,kw] * dy[n,ho,wo,c]
+ *
+ * which at stride 1 is the reversed-kernel correlation of dy with the
+ * complementary pads d(k-1) - p_lo, and at stride 2 is the zero-upsample of
+ * dy onto the forward's sampled positions followed by that correlation
+ * (sections "Stride-2 SAME depthwise input-VJP" and "Stride-2 XLA-SAME
+ * depthwise input-VJP"); both are computed without materialising anything.
+ *
+ * Conventions for every entry point:
+ *   - Activations (x, y, dy, dx) are float32, dense, in the layout of
+ *     desc->layout: DW_NHWC = [N][H][W][C] (C innermost), DW_NCHW =
+ *     [N][C][H][W] (W innermost).
+ *   - Weights are [C][kH][kW] row-major (the PyTorch [C,1,kH,kW] depthwise
+ *     weight, contiguous), float32 or float16 per desc->wtype.  float16 weights
+ *     are widened exactly to float32; accumulation is always float32, taps in
+ *     kh-major / kw-minor order, then the bias is added.  With weights that are
+ *     exactly representable in float16, the float16 and float32 weight paths
+ *     return bit-identical results.
+ *   - Bias is float32 [C] or NULL (NULL means zero).
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or retains them.  Unaligned pointers are accepted
+ *     (a slower kernel is chosen).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous: they enqueue kernels and return without synchronising.
+ *     They make no device allocation and may be captured in a CUDA graph once
+ *     the same descriptor shape has been run once outside capture on that
+ *     device.
+ *   - Errors: invalid descriptors (sizes <= 0, stride or dilation < 1,
+ *     negative pads, an empty output, unknown enum values, NULL required
+ *     pointers) return DW_ERR_INVALID_ARG and launch nothing; an output buffer
+ *     that overlaps an input returns DW_ERR_ALIAS and launches nothing;
+ *     DW_ALGO_TILED on a shape the tiled kernels do not cover returns
+ *     DW_ERR_UNSUPPORTED; a failed launch returns DW_ERR_CUDA.
+ */
+#ifndef DWCONV2D_H_
+#define DWCONV2D_H_
+
+#include <stdint.h>
+
+/* Exported entry points keep default visibility when the library is built
+ * with -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define DW_API __attribute__((visibility("default")))
+#else
+#define DW_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t dw_status_t;
+enum {
+    DW_OK = 0,
+    DW_ERR_INVALID_ARG = 1,
+    DW_ERR_UNSUPPORTED = 2,
+    DW_ERR_ALIAS = 3,
+    DW_ERR_CUDA = 4,
+    DW_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up waiting on a copy */
+};
+
+enum { DW_NHWC = 0, DW_NCHW = 1 };                 /* dw_desc_t.layout   */
+enum { DW_F32 = 0, DW_F16 = 1 };                   /* dw_desc_t.wtype    */
+enum { DW_PAD_EXPLICIT = 0, DW_PAD_SAME = 1 };     /* dw_desc_t.pad_mode */
+enum { DW_ALGO_AUTO = 0, DW_ALGO_DIRECT = 1, DW_ALGO_TILED = 2 }; /* .algo */
+
+/*
+ * Problem descriptor.  N,H,W,C are the INPUT (x / dx) extents.  pad_mode
+ * DW_PAD_SAME ignores the pad_* fields and uses the XLA rule per axis:
+ * Ho = ceil(H/sh), total = max((Ho-1)*sh + dh*(kH-1) + 1 - H, 0),
+ * pt = floor(total/2), pb = total - pt (the odd pad at the bottom/right, the
+ * page's "XLA-SAME" odd-position decimation at stride 2).  DW_PAD_EXPLICIT
+ * uses pad_top/bottom/left/right as given (>= 0); Ho = floor((H + pt + pb -
+ * dh*(kH-1) - 1)/sh) + 1, same for Wo.
+ * algo: DW_ALGO_AUTO picks the fastest kernel that covers the shape;
+ * DW_ALGO_DIRECT forces the one-thread-per-output kernel (any shape);
+ * DW_ALGO_TILED forces the TMA-tiled kernels (DW_ERR_UNSUPPORTED if they do
+ * not cover the shape).
+ */
+typedef struct dw_desc {
+    int64_t N, H, W, C;
+    int32_t kH, kW;
+    int32_t stride_h, stride_w;
+    int32_t dil_h, dil_w;
+    int32_t pad_mode;
+    int32_t pad_top, pad_bottom, pad_left, pad_right;
+    int32_t layout;
+    int32_t wtype;
+    int32_t algo;
+} dw_desc_t;
+
+/* Output extents Ho, Wo of the forward for `desc` (host only, no CUDA call).
+ * Returns DW_ERR_INVALID_ARG for an invalid descriptor. */
+DW_API dw_status_t dwconv2d_out_shape(const dw_desc_t* desc, int64_t* Ho, int64_t* Wo);
+
+/* Resolved pads {top, bottom, left, right} for `desc` (host only). */
+DW_API dw_status_t dwconv2d_resolved_pads(const dw_desc_t* desc, int32_t pads[4]);
+
+/*
+ * Forward: y = depthwise(x; w) + b.
+ *   x: [N,H,W,C] or [N,C,H,W] float32, read only.
+ *   w: [C,kH,kW] float32 or float16 (desc->wtype), read only.
+ *   b: [C] float32 or NULL, read only.
+ *   y: [N,Ho,Wo,C] or [N,C,Ho,Wo] float32, every element written.
+ * y must not overlap x, w or b (DW_ERR_ALIAS).
+ * Page: LeanMlir Depthwise, "Depthwise conv2d forward"; strided forms
+ * "Stride-2 SAME" / "Stride-2 XLA-SAME depthwise conv" (computed directly at
+ * the sampled positions, never as a decimated stride-1 pass).
+ */
+DW_API dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const float* x, const void* w,
+                         const float* b, float* y, void* stream);
+
+/*
+ * Input gradient: dx = J^T dy for the forward of `desc` (bias plays no part).
+ *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] float32, read only.
+ *   w:  [C,kH,kW] float32 or float16, read only.
+ *   dx: [N,H,W,C] or [N,C,H,W] float32, every element written (positions no
+ *       output reads get 0; nothing is accumulated into previous contents).
+ * dx must not overlap dy or w (DW_ERR_ALIAS).
+ * Page: LeanMlir Depthwise, "Closed-form input gradient ... direct formula",
+ * its reversed-kernel form, and the stride-2 / XLA-SAME input-VJP sections
+ * (the forward's actual low pad is used, never a symmetric one).
+ */
+DW_API dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy,
+                               const void* w, float* dx, void* stream);
+
+/*
+ * Which kernel family a call with these arguments would run (host only, no
+ * launch): returns DW_ALGO_DIRECT or DW_ALGO_TILED, or -DW_ERR_* when the call
+ * would fail.  op: 0 = forward (in = x, out = y), 1 = input gradient
+ * (in = dy, out = dx).  Pointers are only inspected for alignment.
+ */
+DW_API int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void* in,
+                            const void* w, const void* out);
+
+/*
+ * Reads and clears the library's device error word on the current device
+ * (synchronous: waits for all prior work on the device).  *code receives 0 if
+ * no kernel has reported a problem since the last call, else DW_ERR_*.
+ * Kernels that wait on asynchronous copies bound every wait; a wait that runs
+ * out sets this word and the kernel returns early (its output is then
+ * undefined).
+ */
+DW_API dw_status_t dwconv2d_take_device_error(int32_t* code);
+
+/* Human-readable name of a status code (static string). */
+DW_API const char* dwconv2d_status_string(dw_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+DW_API int32_t dwconv2d_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DWCONV2D_H_ */

@@ -1,0 +1,158 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, resolves pads and output extents exactly as the oracle's
+(separately written) rules do, and rejects invalid or aliasing calls before
+touching CUDA.  No call here reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import depthwise_convolution_fwd_b200 as dw
+from depthwise_convolution_fwd_b200 import build as dwbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dwbuild.build()
+    return dw.lib()
+
+
+def header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(dwconv2d_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = header_functions()
+    assert "dwconv2d_fwd" in declared and "dwconv2d_bwd_input" in declared
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert sorted(dw.EXPORTS) == declared
+
+
+def test_version_and_status_strings(lib):
+    assert dw.dwconv2d_version() >= 10000
+    for st in range(6):
+        assert dw.status_string(st).startswith("DW_")
+
+
+def random_desc(rng):
+    N, H, W, C = (int(v) for v in rng.integers(1, 40, size=4))
+    kH, kW = (int(v) for v in rng.integers(1, 8, size=2))
+    s = tuple(int(v) for v in rng.integers(1, 4, size=2))
+    d = tuple(int(v) for v in rng.integers(1, 4, size=2))
+    pad = "same" if rng.random() < 0.5 else tuple(int(v) for v in rng.integers(0, 5, size=4))
+    layout = "nhwc" if rng.random() < 0.5 else "nchw"
+    return (N, H, W, C, kH, kW, s, d, pad, layout)
+
+
+def test_out_shape_and_pads_match_oracle(lib):
+    rng = np.random.default_rng(7)
+    checked = 0
+    for _ in range(3000):
+        N, H, W, C, kH, kW, s, d, pad, layout = random_desc(rng)
+        shape = (N, H, W, C) if layout == "nhwc" else (N, C, H, W)
+        p = oracle.problem(shape, kH, kW, s, d, pad, layout)
+        desc = dw.make_desc(N, H, W, C, kH, kW, stride=s, dilation=d, padding=pad, layout=layout)
+        o = oracle.out_shape(p)
+        Ho, Wo = (o[1], o[2]) if layout == "nhwc" else (o[2], o[3])
+        if Ho < 1 or Wo < 1:
+            with pytest.raises(dw.DwError) as e:
+                dw.dwconv2d_out_shape(desc)
+            assert e.value.status == dw.DW_ERR_INVALID_ARG
+            continue
+        assert dw.dwconv2d_out_shape(desc) == (Ho, Wo)
+        assert dw.dwconv2d_resolved_pads(desc) == tuple(int(v) for v in p[10:14])
+        checked += 1
+    assert checked > 1500
+
+
+BAD = [
+    dict(N=0), dict(H=0), dict(W=-1), dict(C=0), dict(kH=0), dict(kW=-2),
+    dict(stride_h=0), dict(stride_w=-1), dict(dil_h=0), dict(dil_w=0),
+    dict(pad_mode=2), dict(pad_mode=0, pad_top=-1), dict(pad_mode=0, pad_right=-3),
+    dict(layout=2), dict(wtype=5), dict(algo=3), dict(algo=-1),
+    dict(kH=9, pad_mode=0),  # no output row left: Ho = 0
+]
+
+
+@pytest.mark.parametrize("bad", BAD)
+def test_invalid_descriptors_rejected_before_launch(lib, bad):
+    desc = dw.make_desc(1, 8, 8, 4, 3, 3)
+    for k, v in bad.items():
+        setattr(desc, k, v)
+    fake = 1 << 40  # never dereferenced: validation fails first
+    assert dw.fwd_raw(desc, fake, fake + (1 << 20), None, fake + (2 << 20), 0) == dw.DW_ERR_INVALID_ARG
+    assert dw.bwd_input_raw(desc, fake, fake + (1 << 20), fake + (2 << 20), 0) == dw.DW_ERR_INVALID_ARG
+    assert dw.dwconv2d_query_algo(desc, 0, fake, fake + (1 << 20), fake + (2 << 20)) == -dw.DW_ERR_INVALID_ARG
+
+
+def test_null_pointers_rejected(lib):
+    desc = dw.make_desc(1, 8, 8, 4, 3, 3)
+    fake = 1 << 40
+    assert dw.fwd_raw(desc, 0, fake, None, fake + 4096, 0) == dw.DW_ERR_INVALID_ARG
+    assert dw.fwd_raw(desc, fake, 0, None, fake + 4096, 0) == dw.DW_ERR_INVALID_ARG
+    assert dw.fwd_raw(desc, fake, fake + 4096, None, 0, 0) == dw.DW_ERR_INVALID_ARG
+    assert lib.dwconv2d_fwd(None, fake, fake, None, fake, None) == dw.DW_ERR_INVALID_ARG
+
+
+def test_aliasing_rejected_before_launch(lib):
+    # 1x8x8x4 NHWC, 3x3 SAME: x and y are 1 KiB each
+    desc = dw.make_desc(1, 8, 8, 4, 3, 3)
+    base = 1 << 40
+    w = base + (1 << 20)
+    assert dw.fwd_raw(desc, base, w, None, base, 0) == dw.DW_ERR_ALIAS            # in place
+    assert dw.fwd_raw(desc, base, w, None, base + 1020, 0) == dw.DW_ERR_ALIAS     # partial overlap
+    assert dw.fwd_raw(desc, base + 1020, w, None, base, 0) == dw.DW_ERR_ALIAS
+    assert dw.fwd_raw(desc, base, w, None, w - 100, 0) == dw.DW_ERR_ALIAS         # y over w
+    assert dw.fwd_raw(desc, base, w, w + 4096, w + 4096 - 8, 0) == dw.DW_ERR_ALIAS  # y over b
+    assert dw.bwd_input_raw(desc, base, w, base + 512, 0) == dw.DW_ERR_ALIAS
+    # adjacent but disjoint buffers are fine (query does not launch)
+    assert dw.dwconv2d_query_algo(desc, 0, base, w, base + 1024) > 0
+
+
+def q(desc, op=0, align=0):
+    base = (1 << 40) + align
+    return dw.dwconv2d_query_algo(desc, op, base, base + (1 << 30), base + (2 << 30))
+
+
+def test_query_algo_selects_tiled_for_covered_shapes(lib):
+    T, D = dw.DW_ALGO_TILED, dw.DW_ALGO_DIRECT
+    # NHWC, C % 4 == 0, aligned: tiled for the instantiated kernel shapes
+    assert q(dw.make_desc(1, 512, 512, 256, 3, 3)) == T
+    assert q(dw.make_desc(1, 512, 512, 256, 3, 3), op=1) == T
+    assert q(dw.make_desc(32, 56, 56, 144, 3, 3, stride=2, padding=1)) == T
+    assert q(dw.make_desc(32, 56, 56, 144, 3, 3, stride=2, padding=1), op=1) == T
+    assert q(dw.make_desc(16, 1, 512, 512, 1, 31)) == T
+    assert q(dw.make_desc(1, 56, 56, 128, 5, 5)) == T
+    # NCHW stride 1 with W % 4 == 0
+    assert q(dw.make_desc(1, 512, 512, 256, 3, 3, layout="nchw")) == T
+    assert q(dw.make_desc(16, 1, 512, 512, 1, 31, layout="nchw"), op=1) == T
+    # not covered -> direct
+    assert q(dw.make_desc(1, 13, 17, 7, 3, 3)) == D                      # C % 4 != 0
+    assert q(dw.make_desc(1, 30, 19, 128, 7, 7, layout="nchw")) == D     # W % 4 != 0
+    assert q(dw.make_desc(1, 16, 16, 8, 3, 3), align=4) == D             # unaligned pointers
+    assert q(dw.make_desc(1, 16, 16, 8, 2, 2)) == D                      # no 2x2 instance
+    assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2)) == D
+    # forcing
+    assert q(dw.make_desc(1, 13, 17, 7, 3, 3, algo="direct")) == D
+    assert q(dw.make_desc(1, 512, 512, 256, 3, 3, algo="direct")) == D
+    assert q(dw.make_desc(1, 13, 17, 7, 3, 3, algo="tiled")) == -dw.DW_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 8, 8, 4)
+    w = torch.zeros(4, 3, 3)
+    with pytest.raises(TypeError):
+        dw.dwconv2d_fwd(x, w)

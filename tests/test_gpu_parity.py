@@ -1,0 +1,256 @@
+"""GPU parity: the CUDA kernels (through the C ABI) against the float64 oracle.
+
+Every configuration of the workload set runs forward and input gradient,
+elementwise against the oracle under the rule of tests/gpu_util.py
+(|gpu - ref| <= 1e-5 * sum|terms|, exact where there are no terms), on both
+kernel families where they apply; the full-size large case is checked on a
+structured sample of outputs.  float16 weights must give bit-identical
+results to float32 weights holding the same (float16-exact) values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import depthwise_convolution_fwd_b200 as dw
+from depthwise_convolution_fwd_b200 import build as dwbuild
+from depthwise_convolution_fwd_b200 import workloads as wl
+from depthwise_convolution_fwd_b200.workloads import Case
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dwbuild.build()
+    dw.lib()
+    yield
+    torch.cuda.synchronize()
+    assert dw.dwconv2d_take_device_error() == 0
+
+
+def check_case(case: Case, algos=("auto", "direct")):
+    inp = gu.inputs(case)
+    ref_y, sc_y = gu.reference_fwd(case, inp)
+    ref_dx, sc_dx = gu.reference_bwd(case, inp)
+    for algo in algos:
+        y = gu.gpu_fwd(case, inp, algo=algo)
+        dx = gu.gpu_bwd(case, inp, algo=algo)
+        torch.cuda.synchronize()
+        gu.assert_close(y.cpu().numpy(), ref_y, sc_y, f"{case.name} fwd [{algo}]")
+        gu.assert_close(dx.cpu().numpy(), ref_dx, sc_dx, f"{case.name} bwd_input [{algo}]")
+    return inp
+
+
+SMALL = wl.tiny() + wl.mobilenet() + [c for c in wl.conformer() if c.W == 24] + \
+    [c for c in wl.large() if c.H == 30]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
+def test_config_cases_match_oracle(case):
+    check_case(case)
+
+
+@pytest.mark.parametrize("case", [c for c in wl.conformer() if c.W == 512], ids=lambda c: c.name)
+def test_conformer_long_matches_oracle(case):
+    check_case(case, algos=("auto",))
+
+
+@pytest.mark.parametrize("case", wl.edge(), ids=lambda c: c.name)
+def test_edge_cases_match_oracle(case):
+    inp = check_case(case)
+    if case.wtype == "f16":
+        # float16 weights == float32 weights holding the same values, bit for bit
+        for algo in ("auto", "direct"):
+            y16 = gu.gpu_fwd(case, inp, algo=algo, w_key="w")
+            y32 = gu.gpu_fwd(case, inp, algo=algo, w_key="w32")
+            d16 = gu.gpu_bwd(case, inp, algo=algo, w_key="w")
+            d32 = gu.gpu_bwd(case, inp, algo=algo, w_key="w32")
+            assert torch.equal(y16, y32), f"{case.name}: f16/f32 forward differ [{algo}]"
+            assert torch.equal(d16, d32), f"{case.name}: f16/f32 input gradient differ [{algo}]"
+
+
+# Tiled-kernel instances, each forced and compared, with f16 twins.
+TILED = [
+    Case("t_nhwc_3x3_s1", 2, 37, 45, 72, 3, 3, seed=1),
+    Case("t_nhwc_3x3_s1_pad", 1, 23, 70, 36, 3, 3, padding=(0, 2, 2, 1), seed=2),
+    Case("t_nhwc_3x3_s2", 3, 29, 41, 44, 3, 3, stride=2, padding=1, seed=3),
+    Case("t_nhwc_3x3_s2_same", 2, 30, 34, 40, 3, 3, stride=2, seed=4),
+    Case("t_nhwc_3x3_s2_asym", 2, 19, 23, 8, 3, 3, stride=2, padding=(2, 0, 1, 2), seed=5),
+    Case("t_nhwc_3x3_d2", 2, 21, 40, 36, 3, 3, dilation=2, seed=6),
+    Case("t_nhwc_3x3_d3", 1, 25, 30, 64, 3, 3, dilation=3, seed=7),
+    Case("t_nhwc_5x5", 2, 17, 39, 68, 5, 5, seed=8),
+    Case("t_nhwc_5x5_pad", 1, 17, 20, 32, 5, 5, padding=(4, 0, 1, 3), seed=9),
+    Case("t_nhwc_1x3", 3, 2, 150, 36, 1, 3, seed=10),
+    Case("t_nhwc_1x5", 2, 3, 130, 20, 1, 5, seed=11),
+    Case("t_nhwc_1x7", 2, 1, 260, 40, 1, 7, padding=(0, 0, 5, 2), seed=12),
+    Case("t_nhwc_1x15", 2, 2, 300, 44, 1, 15, act="normal", seed=13),
+    Case("t_nhwc_1x31", 3, 1, 290, 68, 1, 31, act="normal", seed=14),
+    Case("t_nhwc_1x31_pad", 1, 1, 100, 32, 1, 31, padding=(1, 2, 31, 0), act="normal", seed=15),
+    Case("t_nchw_3x3", 2, 45, 140, 5, 3, 3, layout="nchw", seed=16),
+    Case("t_nchw_3x3_pad0", 1, 40, 132, 3, 3, 3, padding=0, layout="nchw", seed=17),
+    Case("t_nchw_3x3_pad2", 1, 40, 132, 3, 3, 3, padding=(2, 1, 2, 3), layout="nchw", seed=18),
+    Case("t_nchw_3x3_pad3", 1, 33, 260, 2, 3, 3, padding=(1, 1, 3, 0), layout="nchw", seed=19),
+    Case("t_nchw_5x5", 2, 36, 136, 3, 5, 5, layout="nchw", seed=20),
+    Case("t_nchw_7x7", 1, 37, 140, 4, 7, 7, layout="nchw", seed=21),
+    Case("t_nchw_1x15", 2, 3, 300, 19, 1, 15, layout="nchw", act="normal", seed=22),
+    Case("t_nchw_1x31", 2, 2, 264, 21, 1, 31, layout="nchw", act="normal", seed=23),
+    Case("t_nchw_1x31_pad", 1, 1, 132, 9, 1, 31, padding=(2, 0, 4, 9), layout="nchw",
+         act="normal", seed=24),
+]
+
+
+@pytest.mark.parametrize("case", TILED, ids=lambda c: c.name)
+def test_tiled_kernels_match_oracle(case):
+    inp = gu.inputs(case)
+    x = inp["x"].cuda()
+    w = inp["w"].cuda()
+    y = torch.empty(case.out_shape(*gu.out_hw(case)), device="cuda")
+    assert gu.chosen_algo(case, 0, x, w, y) == dw.DW_ALGO_TILED, "expected the tiled path"
+    assert gu.chosen_algo(case, 1, y, w, x) == dw.DW_ALGO_TILED, "expected the tiled path"
+    check_case(case, algos=("tiled", "direct"))
+    case16 = case.with_(wtype="f16", name=case.name + "_f16")
+    inp16 = gu.inputs(case16)
+    for fn in (gu.gpu_fwd, gu.gpu_bwd):
+        a = fn(case16, inp16, algo="tiled", w_key="w")
+        b = fn(case16, inp16, algo="tiled", w_key="w32")
+        assert torch.equal(a, b), f"{case.name}: f16 weights not bit-identical"
+
+
+def test_random_sweep_matches_oracle():
+    rng = np.random.default_rng(2024)
+    count = 0
+    while count < 120:
+        layout = "nhwc" if rng.random() < 0.5 else "nchw"
+        k = int(rng.choice([1, 2, 3, 4, 5, 7, 15, 31]))
+        kH, kW = (1, k) if rng.random() < 0.3 else (k, int(rng.choice([1, 3, 5, k])))
+        C = int(rng.choice([1, 3, 4, 7, 8, 36, 131, 132]))
+        s = int(rng.integers(1, 4))
+        d = int(rng.integers(1, 4))
+        pad = "same" if rng.random() < 0.5 else tuple(int(v) for v in rng.integers(0, 4, size=4))
+        case = Case(f"sweep{count}", int(rng.integers(1, 4)), int(rng.integers(1, 38)),
+                    int(rng.integers(1, 38)), C, kH, kW, stride=s, dilation=d, padding=pad,
+                    layout=layout, wtype="f16" if rng.random() < 0.3 else "f32",
+                    bias=bool(rng.random() < 0.8), seed=5000 + count)
+        try:
+            ho, wo = gu.out_hw(case)
+        except Exception:
+            continue
+        if ho < 1 or wo < 1:
+            continue
+        check_case(case)
+        count += 1
+
+
+# ----------------------------------------------------------- full size ---
+
+@pytest.mark.parametrize("case", [c for c in wl.large() if c.H == 512], ids=lambda c: c.name)
+def test_large_full_size_sampled(case):
+    """1x512x512x256 3x3 SAME, the launch configuration the benchmark times,
+    checked on border rows/columns plus 20k random outputs."""
+    inp = gu.inputs(case)
+    rng = np.random.default_rng(77)
+    x = inp["x"].cuda()
+    w = inp["w"].cuda()
+    b = inp["b"].cuda()
+    y = dw.dwconv2d_fwd(x, w, b, padding="same", layout=case.layout)
+    assert gu.chosen_algo(case, 0, x, w, y) == dw.DW_ALGO_TILED
+    dx = gu.gpu_bwd(case, inp)
+    torch.cuda.synchronize()
+    iy = gu.structured_sample(tuple(y.shape), case.layout, rng)
+    ref, sc = gu.reference_fwd_at(case, inp, iy)
+    gu.assert_close(y.reshape(-1).cpu().numpy()[iy], ref, sc, case.name + " fwd")
+    ix = gu.structured_sample(tuple(dx.shape), case.layout, rng)
+    ref, sc = gu.reference_bwd_at(case, inp, ix)
+    gu.assert_close(dx.reshape(-1).cpu().numpy()[ix], ref, sc, case.name + " bwd_input")
+
+
+# --------------------------------------------------------- memory hygiene --
+
+GUARD = 4096
+
+
+@pytest.mark.parametrize("case", [
+    Case("g_nhwc", 2, 19, 37, 40, 3, 3, seed=31),
+    Case("g_nhwc_s2", 2, 19, 37, 44, 3, 3, stride=2, padding=1, seed=32),
+    Case("g_nchw", 2, 19, 36, 5, 3, 3, layout="nchw", seed=33),
+    Case("g_nhwc_1x31", 2, 1, 70, 36, 1, 31, seed=34),
+    Case("g_odd", 2, 9, 11, 7, 5, 5, stride=2, seed=35),
+], ids=lambda c: c.name)
+@pytest.mark.parametrize("shift", [0, 1])
+def test_outputs_stay_inside_their_buffer(case, shift):
+    """Canary floats around the output: no kernel writes outside it.  shift=1
+    offsets every pointer by one float (unaligned -> direct kernel)."""
+    inp = gu.inputs(case)
+    canary = float("nan")
+
+    def padded(t):
+        buf = torch.full((t.numel() + 2 * GUARD + shift,), 7.0, device="cuda")
+        view = buf[GUARD + shift: GUARD + shift + t.numel()].view(t.shape)
+        view.copy_(t)
+        return buf, view
+
+    _, x = padded(inp["x"])
+    _, dy = padded(inp["dy"])
+    w = inp["w"].cuda()
+    b = inp["b"].cuda()
+    ho, wo = gu.out_hw(case)
+    for op in ("fwd", "bwd"):
+        shape = case.out_shape(ho, wo) if op == "fwd" else case.in_shape()
+        n = int(np.prod(shape))
+        obuf = torch.full((n + 2 * GUARD + shift,), canary, device="cuda")
+        out = obuf[GUARD + shift: GUARD + shift + n].view(shape)
+        if op == "fwd":
+            dw.dwconv2d_fwd(x, w, b, stride=case.stride, padding=case.padding,
+                            layout=case.layout, out=out)
+            ref, sc = gu.reference_fwd(case, inp)
+        else:
+            dw.dwconv2d_bwd_input(dy, w, (case.H, case.W), stride=case.stride,
+                                  padding=case.padding, layout=case.layout, out=out)
+            ref, sc = gu.reference_bwd(case, inp)
+        torch.cuda.synchronize()
+        host = obuf.cpu()
+        assert torch.isnan(host[:GUARD + shift]).all(), f"{case.name} {op}: write before buffer"
+        assert torch.isnan(host[GUARD + shift + n:]).all(), f"{case.name} {op}: write after buffer"
+        gu.assert_close(out.cpu().numpy(), ref, sc, f"{case.name} {op} shift={shift}")
+
+
+def test_input_gradient_overwrites_stale_output():
+    case = Case("stale", 2, 16, 20, 8, 3, 3, stride=2, padding=1, seed=41)
+    inp = gu.inputs(case)
+    ref, sc = gu.reference_bwd(case, inp)
+    for algo in ("auto", "direct"):
+        out = torch.full(case.in_shape(), 123.0, device="cuda")
+        gu.gpu_bwd(case, inp, algo=algo, out=out)
+        torch.cuda.synchronize()
+        gu.assert_close(out.cpu().numpy(), ref, sc, f"stale [{algo}]")
+
+
+def test_side_stream_and_repeatability():
+    case = wl.mobilenet()[2]
+    inp = gu.inputs(case)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y1 = gu.gpu_fwd(case, inp)
+        d1 = gu.gpu_bwd(case, inp)
+    s.synchronize()
+    y2 = gu.gpu_fwd(case, inp)
+    d2 = gu.gpu_bwd(case, inp)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(d1, d2)
+    ref, sc = gu.reference_fwd(case, inp)
+    gu.assert_close(y1.cpu().numpy(), ref, sc, "side stream fwd")
+
+
+def test_no_bias_and_aliasing_errors_on_device():
+    case = Case("nob", 1, 12, 12, 16, 3, 3, bias=False, seed=42)
+    inp = gu.inputs(case)
+    ref, sc = gu.reference_fwd(case, inp)
+    y = gu.gpu_fwd(case, inp)
+    torch.cuda.synchronize()
+    gu.assert_close(y.cpu().numpy(), ref, sc, "no bias")
+    x = inp["x"].cuda()
+    with pytest.raises(dw.DwError) as e:
+        dw.dwconv2d_fwd(x, inp["w"].cuda(), out=x)
+    assert e.value.status == dw.DW_ERR_ALIAS
