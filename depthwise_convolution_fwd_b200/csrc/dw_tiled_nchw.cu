@@ -52,12 +52,16 @@ struct Cfg {
     static constexpr int IWB = (REM + TW + (KW - 1) * D + 3) / 4 * 4;
     static constexpr int BOXH = IH;
     static constexpr int BOXC = ROWS ? WY : 1;
-    static constexpr int STAGE_FLOATS = IWB * IH * BOXC;
-    static constexpr int STAGE_BYTES = STAGE_FLOATS * 4;
+    // bytes one TMA box delivers, and the stage pitch: every stage must start
+    // on a 128-byte boundary (shared-memory destination rule of tensor copies)
+    static constexpr int STAGE_BYTES = IWB * IH * BOXC * 4;
+    static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
+    static constexpr int STAGE_FLOATS = STAGE_PITCH / 4;
     static constexpr int RH = THT + (KH - 1) * D;           // window rows
     static constexpr int NV = (REM + 3 + (KW - 1) * D) / 4 + 1;  // float4 per window row
-    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(NS) * 8;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(NS) * 8;
     static_assert(IWB <= 256 && IH <= 256 && BOXC <= 256, "TMA box dimension limit");
+    static_assert(STAGE_PITCH % 128 == 0 && (IWB * 4) % 16 == 0, "TMA alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -86,7 +90,7 @@ __global__ void __launch_bounds__(K::NT, 1)
     tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
     extern __shared__ __align__(128) unsigned char smem[];
     float* stages = reinterpret_cast<float*>(smem);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH);
 
     const int tid = threadIdx.x;
     const int xi = tid % K::WX;

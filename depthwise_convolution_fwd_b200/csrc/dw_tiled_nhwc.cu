@@ -68,6 +68,8 @@ struct Cfg {
     static constexpr int STAGE_BYTES = STAGE_F4 * 16;
     static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(NS) * 8;
     static_assert(IH <= 256 && IW <= 256, "TMA box dimension limit");
+    // every stage starts on a 128-byte boundary (tensor-copy destination rule)
+    static_assert(STAGE_BYTES % 128 == 0, "TMA shared-memory alignment");
     static_assert(!TR || (THT % S == 0 && TWT % S == 0), "transposed blocks are phase aligned");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };

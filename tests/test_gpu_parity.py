@@ -71,7 +71,10 @@ def test_edge_cases_match_oracle(case):
             assert torch.equal(d16, d32), f"{case.name}: f16/f32 input gradient differ [{algo}]"
 
 
-# Tiled-kernel instances, each forced and compared, with f16 twins.
+# Tiled-kernel instances, each forced and compared, with f16 twins.  The NCHW
+# cases keep W and Wo multiples of 4 (the TMA row-stride rule applies to the
+# input of both directions) and cover every box alignment REM = (-pl) mod 4 of
+# the forward and (pl - kW + 1) mod 4 of the input gradient.
 TILED = [
     Case("t_nhwc_3x3_s1", 2, 37, 45, 72, 3, 3, seed=1),
     Case("t_nhwc_3x3_s1_pad", 1, 23, 70, 36, 3, 3, padding=(0, 2, 2, 1), seed=2),
@@ -89,14 +92,14 @@ TILED = [
     Case("t_nhwc_1x31", 3, 1, 290, 68, 1, 31, act="normal", seed=14),
     Case("t_nhwc_1x31_pad", 1, 1, 100, 32, 1, 31, padding=(1, 2, 31, 0), act="normal", seed=15),
     Case("t_nchw_3x3", 2, 45, 140, 5, 3, 3, layout="nchw", seed=16),
-    Case("t_nchw_3x3_pad0", 1, 40, 132, 3, 3, 3, padding=0, layout="nchw", seed=17),
-    Case("t_nchw_3x3_pad2", 1, 40, 132, 3, 3, 3, padding=(2, 1, 2, 3), layout="nchw", seed=18),
-    Case("t_nchw_3x3_pad3", 1, 33, 260, 2, 3, 3, padding=(1, 1, 3, 0), layout="nchw", seed=19),
+    Case("t_nchw_3x3_pad0", 1, 40, 132, 3, 3, 3, padding=(0, 0, 0, 2), layout="nchw", seed=17),
+    Case("t_nchw_3x3_pad2", 1, 40, 132, 3, 3, 3, padding=(2, 1, 2, 0), layout="nchw", seed=18),
+    Case("t_nchw_3x3_pad3", 1, 33, 260, 2, 3, 3, padding=(1, 1, 3, 3), layout="nchw", seed=19),
     Case("t_nchw_5x5", 2, 36, 136, 3, 5, 5, layout="nchw", seed=20),
     Case("t_nchw_7x7", 1, 37, 140, 4, 7, 7, layout="nchw", seed=21),
     Case("t_nchw_1x15", 2, 3, 300, 19, 1, 15, layout="nchw", act="normal", seed=22),
     Case("t_nchw_1x31", 2, 2, 264, 21, 1, 31, layout="nchw", act="normal", seed=23),
-    Case("t_nchw_1x31_pad", 1, 1, 132, 9, 1, 31, padding=(2, 0, 4, 9), layout="nchw",
+    Case("t_nchw_1x31_pad", 1, 1, 132, 9, 1, 31, padding=(2, 0, 4, 10), layout="nchw",
          act="normal", seed=24),
 ]
 
@@ -116,6 +119,31 @@ def test_tiled_kernels_match_oracle(case):
         a = fn(case16, inp16, algo="tiled", w_key="w")
         b = fn(case16, inp16, algo="tiled", w_key="w32")
         assert torch.equal(a, b), f"{case.name}: f16 weights not bit-identical"
+
+
+# Enough tiles that every persistent CTA walks its TMA stage ring several
+# times (stage pitch, phase parity and re-issue paths), ragged at every edge.
+RING = [
+    Case("r_nhwc_3x3_s1", 4, 125, 250, 60, 3, 3, seed=51),
+    Case("r_nhwc_3x3_s2", 16, 63, 126, 68, 3, 3, stride=2, padding=1, seed=52),
+    Case("r_nhwc_5x5", 16, 61, 125, 64, 5, 5, seed=53),
+    Case("r_nhwc_1x31", 16, 15, 250, 124, 1, 31, act="normal", seed=54),
+    Case("r_nchw_3x3", 2, 125, 508, 64, 3, 3, layout="nchw", seed=55),
+    Case("r_nchw_5x5", 2, 93, 252, 32, 5, 5, layout="nchw", seed=56),
+    Case("r_nchw_7x7", 2, 61, 252, 48, 7, 7, layout="nchw", seed=57),
+    Case("r_nchw_1x31", 8, 15, 252, 124, 1, 31, layout="nchw", act="normal", seed=58),
+]
+
+
+@pytest.mark.parametrize("case", RING, ids=lambda c: c.name)
+def test_tiled_ring_wraps(case):
+    inp = gu.inputs(case)
+    x = inp["x"].cuda()
+    w = inp["w"].cuda()
+    y = torch.empty(case.out_shape(*gu.out_hw(case)), device="cuda")
+    assert gu.chosen_algo(case, 0, x, w, y) == dw.DW_ALGO_TILED
+    assert gu.chosen_algo(case, 1, y, w, x) == dw.DW_ALGO_TILED
+    check_case(case, algos=("tiled",))
 
 
 def test_random_sweep_matches_oracle():
