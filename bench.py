@@ -403,6 +403,34 @@ def run_e2e(args, torch, dw, shapes, device, stream, world):
             "api": "depthwise_convolution_fwd_b200.dwconv2d_fwd / dwconv2d_bwd_input"}
 
 
+def run_profile(args, local_rank):
+    """Launch one kernel of the workload `--steps` times (no timing, no other
+    kernels), so a profiler capture sees only that kernel."""
+    import torch
+
+    import depthwise_convolution_fwd_b200 as dw
+    from depthwise_convolution_fwd_b200 import build as dwbuild
+    dwbuild.build()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    name, op = args.profile.split(":")
+    cases, _ = workload_cases(args.workload)
+    match = [c for c in cases if c.name == name]
+    if not match or op not in ("fwd", "bwd"):
+        raise SystemExit(f"unknown kernel {args.profile!r}; shapes: {[c.name for c in cases]}")
+    sh = Shape(match[0], dw, torch, device, 1)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            sh.call(dw, op, 0, stream.cuda_stream)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "launches": args.steps,
+                      "algo": dw.dwconv2d_query_algo(sh.desc, 0 if op == "fwd" else 1,
+                                                     sh.sets[0]["x"].data_ptr(), sh.w.data_ptr(),
+                                                     sh.sets[0]["y"].data_ptr())}), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------- CPU arms --
 
 def oracle_step(cases, fraction, oracle, np, torch):
@@ -509,6 +537,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=8.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", metavar="SHAPE:OP", default=None,
+                    help="launch only this kernel (e.g. mobilenet_32x56x56x144_3x3_s2:fwd) "
+                         "--steps times on one buffer set, untimed; for ncu captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -516,6 +547,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.profile:
+        return run_profile(args, local_rank)
 
     if args.impl == "reference":
         if rank != 0:

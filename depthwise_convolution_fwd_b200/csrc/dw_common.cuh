@@ -94,6 +94,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -111,6 +115,42 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
         if (global_timer_ns() - t0 > kWaitLimitNs) return false;
     }
     return true;
+}
+
+// Bounded wait that also gives up as soon as another warp of the CTA has
+// raised `abort` (a shared-memory flag), so one failed wait ends every warp.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
+                                                   const volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// Division by a run-time constant d as a multiply and shift, exact for every
+// 0 <= n < 2^31: with s = ceil(log2 d) and m = floor(2^(31+s) / d) + 1,
+// floor(n*m / 2^(31+s)) = floor(n/d) because n*(m - 2^(31+s)/d) < 2^(31+s)/d.
+struct FastDiv {
+    uint64_t m;
+    uint32_t shift;  // 31 + s
+    int d;
+};
+
+inline FastDiv make_fastdiv(int d) {
+    uint32_t s = 0;
+    while ((int64_t(1) << s) < d) ++s;
+    FastDiv f;
+    f.m = ((uint64_t(1) << (31 + s)) / uint64_t(d)) + 1;
+    f.shift = 31 + s;
+    f.d = d;
+    return f;
+}
+
+__device__ __forceinline__ int fast_div(int n, const FastDiv& f) {
+    return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * f.m) >> f.shift);
 }
 
 // 4-D tiled TMA load (no multicast) into this CTA's shared memory; completion

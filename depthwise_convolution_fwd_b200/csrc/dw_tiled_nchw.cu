@@ -35,7 +35,7 @@ struct Args {
     int wtype;
     int N, C, Hout, Wout;
     int pt, pl;  // effective low pads of the correlation this kernel runs
-    int tiles_x, tiles_y, tiles_c;
+    FastDiv tiles_x, tiles_y, tiles_c;
     int ntiles;
 };
 
@@ -45,7 +45,8 @@ struct Cfg {
     static constexpr bool REV = REV_;
     static constexpr bool ROWS = KH == 1;  // 1-D: thread rows are channels
     static constexpr int THT = ROWS ? 1 : THT_, WX = WX_, WY = WY_, NS = NS_;
-    static constexpr int NT = WX * WY;
+    static constexpr int NCW = WX * WY / 32;  // consumer warps
+    static constexpr int NT = WX * WY + 32;   // + one producer warp
     static constexpr int TW = 4 * WX;
     static constexpr int TH = ROWS ? 1 : THT * WY;
     static constexpr int IH = ROWS ? 1 : TH + (KH - 1) * D;
@@ -59,7 +60,8 @@ struct Cfg {
     static constexpr int STAGE_FLOATS = STAGE_PITCH / 4;
     static constexpr int RH = THT + (KH - 1) * D;           // window rows
     static constexpr int NV = (REM + 3 + (KW - 1) * D) / 4 + 1;  // float4 per window row
-    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(NS) * 8;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NS) * 8 + 16;
+    static_assert((WX * WY) % 32 == 0, "whole consumer warps");
     static_assert(IWB <= 256 && IH <= 256 && BOXC <= 256, "TMA box dimension limit");
     static_assert(STAGE_PITCH % 128 == 0 && (IWB * 4) % 16 == 0, "TMA alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -77,12 +79,12 @@ __device__ __forceinline__ void static_for(F&& f) {
 template <class K>
 __device__ __forceinline__ void decode_tile(int t, const Args& a, int& tx, int& ty, int& c,
                                             int& n) {
-    tx = t % a.tiles_x;
-    t /= a.tiles_x;
-    ty = t % a.tiles_y;  // ROWS: output row h
-    t /= a.tiles_y;
-    c = t % a.tiles_c;   // ROWS: channel group; else channel
-    n = t / a.tiles_c;
+    int q = fast_div(t, a.tiles_x);
+    tx = t - q * a.tiles_x.d;
+    int r = fast_div(q, a.tiles_y);
+    ty = q - r * a.tiles_y.d;  // ROWS: output row h
+    n = fast_div(r, a.tiles_c);
+    c = r - n * a.tiles_c.d;   // ROWS: channel group; else channel
 }
 
 template <class K>
@@ -91,41 +93,62 @@ __global__ void __launch_bounds__(K::NT, 1)
     extern __shared__ __align__(128) unsigned char smem[];
     float* stages = reinterpret_cast<float*>(smem);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
 
     const int tid = threadIdx.x;
-    const int xi = tid % K::WX;
-    const int yi = tid / K::WX;
+    const int warp = tid >> 5, lane = tid & 31;
     // contiguous range of tiles for this CTA: neighbouring tiles share a
     // plane (filter stays in registers) and their halos (L2 hits)
     const int t_begin = int((int64_t(blockIdx.x) * a.ntiles) / gridDim.x);
     const int t_end = int((int64_t(blockIdx.x + 1) * a.ntiles) / gridDim.x);
 
     if (tid == 0) {
-        prefetch_tensor_map(&tmap);
 #pragma unroll
-        for (int s = 0; s < K::NS; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
+        }
+        *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
-    auto issue = [&](int s, int t) {
-        int tx, ty, c, n;
-        decode_tile<K>(t, a, tx, ty, c, n);
-        const int ix0 = tx * K::TW - a.pl - K::REM;
-        mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
-        if constexpr (K::ROWS)
-            tma_load_4d(stages + size_t(s) * K::STAGE_FLOATS, &tmap, &full[s], ix0, ty - a.pt,
-                        c * K::WY, n);
-        else
-            tma_load_4d(stages + size_t(s) * K::STAGE_FLOATS, &tmap, &full[s], ix0,
-                        ty * K::TH - a.pt, c, n);
-    };
-    if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < K::NS; ++s)
-            if (t_begin + s < t_end) issue(s, t_begin + s);
+    if (warp == K::NCW) {
+        // ---------------- producer warp: one lane issues every TMA load ----
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap);
+            int k = 0;
+            bool ok = true;
+            for (int t = t_begin; t < t_end; ++t, ++k) {
+                const int s = k % K::NS;
+                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                int tx, ty, c, n;
+                decode_tile<K>(t, a, tx, ty, c, n);
+                const int ix0 = tx * K::TW - a.pl - K::REM;
+                float* dst = stages + size_t(s) * K::STAGE_FLOATS;
+                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+                if constexpr (K::ROWS)
+                    tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
+                else
+                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH - a.pt, c, n);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
+        }
+        return;
     }
 
+    // -------------------------- consumer warps --------------------------------
+    const int xi = tid % K::WX;
+    const int yi = tid / K::WX;
     float wr[K::KH][K::KW];
     float bias = 0.f;
     int cur_key = -1;
@@ -134,11 +157,10 @@ __global__ void __launch_bounds__(K::NT, 1)
     int k = 0;
     for (int t = t_begin; t < t_end; ++t, ++k) {
         const int s = k % K::NS;
-        const uint32_t parity = (k / K::NS) & 1;
         int tx, ty, cg, n;
         decode_tile<K>(t, a, tx, ty, cg, n);
         const int c = K::ROWS ? cg * K::WY + yi : cg;
-        const int key = cg + n * a.tiles_c;
+        const int key = cg + n * a.tiles_c.d;
         if (key != cur_key) {
             cur_key = key;
             live = c < a.C;
@@ -154,7 +176,13 @@ __global__ void __launch_bounds__(K::NT, 1)
             bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
         }
 
-        const bool ok = mbar_wait_bounded(&full[s], parity);
+        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+            }
+            break;
+        }
 
         float acc[K::THT][4];
 #pragma unroll
@@ -190,6 +218,9 @@ __global__ void __launch_bounds__(K::NT, 1)
             });
         });
 
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
         if (live) {
             const int wo0 = tx * K::TW + 4 * xi;
 #pragma unroll
@@ -209,18 +240,6 @@ __global__ void __launch_bounds__(K::NT, 1)
                 }
             }
         }
-
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
-                for (int j = 1; j < K::NS; ++j) {
-                    const int k2 = k + j;
-                    if (t + j < t_end) mbar_wait_bounded(&full[k2 % K::NS], (k2 / K::NS) & 1);
-                }
-            }
-            return;
-        }
-        if (tid == 0 && t + K::NS < t_end) issue(s, t + K::NS);
     }
 }
 
@@ -245,9 +264,9 @@ dw_status_t launch(const Problem& p, const float* in, const void* w, const float
     const int64_t tc = K::ROWS ? (p.C + K::WY - 1) / K::WY : p.C;
     const int64_t nt = tx * ty * tc * p.N;
     if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
-    a.tiles_x = static_cast<int>(tx);
-    a.tiles_y = static_cast<int>(ty);
-    a.tiles_c = static_cast<int>(tc);
+    a.tiles_x = make_fastdiv(static_cast<int>(tx));
+    a.tiles_y = make_fastdiv(static_cast<int>(ty));
+    a.tiles_c = make_fastdiv(static_cast<int>(tc));
     a.ntiles = static_cast<int>(nt);
     if (dry_run) return DW_OK;
 

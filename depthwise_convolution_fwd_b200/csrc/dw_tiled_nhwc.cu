@@ -8,12 +8,14 @@
 // channels of a pixel, so a quarter-warp reads or writes 128 contiguous
 // bytes.  The input halo tile [IH][IW][32] of every output tile is fetched by
 // one 4-D TMA load (zero fill outside the tensor == zero padding) into a ring
-// of NS shared-memory stages; a persistent CTA walks its tiles while the next
-// NS-1 loads are in flight.  Filter taps and bias of the CTA's 32 channels sit
-// in registers.  Each thread computes a THT x TWT block of outputs: it streams
-// the input cells of its block's window once from shared memory and feeds
-// every (output, tap) pair that reads that cell - a register sliding window
-// in both directions, resolved at compile time.
+// of NS shared-memory stages.  One producer warp issues the loads; the
+// consumer warps wait on a per-stage "full" mbarrier, compute, and release the
+// stage on a per-stage "empty" mbarrier, so no block-wide barrier sits in the
+// tile loop and NS-1 loads stay in flight.  Filter taps and bias of the CTA's
+// 32 channels sit in registers.  Each consumer thread computes a THT x TWT
+// block of outputs: it streams the input cells of its block's window once
+// from shared memory and feeds every (output, tap) pair that reads that cell,
+// a register sliding window in both directions resolved at compile time.
 //
 // Forward (LeanMlir Proofs/Architectures/Depthwise, "Depthwise conv2d
 // forward"): output (ho,wo) reads input (ho*S + kh*D - pt, wo*S + kw*D - pl);
@@ -46,7 +48,7 @@ struct Args {
     int Hout, Wout;  // extents of the tensor written
     int pt, pl;      // forward low pads
     int org_y, org_x;
-    int tiles_x, tiles_y, tiles_c;
+    FastDiv tiles_c, tiles_x, tiles_y;
     int ntiles;
 };
 
@@ -55,7 +57,8 @@ struct Cfg {
     static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
     static constexpr bool TR = TR_;
     static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
-    static constexpr int NT = CV * WX * WY;
+    static constexpr int NCW = WX * WY * CV / 32;  // consumer warps
+    static constexpr int NT = NCW * 32 + 32;       // + one producer warp
     static constexpr int TH = THT * WY, TW = TWT * WX;
     static constexpr int AH = TR ? ((KH - 1) * D + S - 1) / S : 0;
     static constexpr int AW = TR ? ((KW - 1) * D + S - 1) / S : 0;
@@ -66,7 +69,8 @@ struct Cfg {
     static constexpr int RW = TR ? AW + (TWT - 1) / S + 1 : (TWT - 1) * S + (KW - 1) * D + 1;
     static constexpr int STAGE_F4 = IH * IW * CV;
     static constexpr int STAGE_BYTES = STAGE_F4 * 16;
-    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(NS) * 8;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(2 * NS) * 8 + 16;
+    static_assert((WX * WY * CV) % 32 == 0, "whole consumer warps");
     static_assert(IH <= 256 && IW <= 256, "TMA box dimension limit");
     // every stage starts on a 128-byte boundary (tensor-copy destination rule)
     static_assert(STAGE_BYTES % 128 == 0, "TMA shared-memory alignment");
@@ -102,30 +106,31 @@ __host__ __device__ constexpr int tap_for(int r, int j) {
     }
 }
 
-__device__ __forceinline__ void decode_tile(int t, const Args& a, int& cb, int& tx, int& ty,
-                                            int& n) {
-    cb = t % a.tiles_c;
-    t /= a.tiles_c;
-    tx = t % a.tiles_x;
-    t /= a.tiles_x;
-    ty = t % a.tiles_y;
-    n = t / a.tiles_y;
-}
+struct Tile {
+    int cb, n, oy0, ox0, iy0, ix0;
+};
 
 template <class K>
-__device__ __forceinline__ void tile_origin(const Args& a, int tx, int ty, int& oy0, int& ox0,
-                                            int& iy0, int& ix0) {
+__device__ __forceinline__ Tile decode_tile(int t, const Args& a) {
+    Tile T;
+    int q = fast_div(t, a.tiles_c);
+    T.cb = t - q * a.tiles_c.d;
+    const int r = fast_div(q, a.tiles_x);
+    const int tx = q - r * a.tiles_x.d;
+    T.n = fast_div(r, a.tiles_y);
+    const int ty = r - T.n * a.tiles_y.d;
     if constexpr (!K::TR) {
-        oy0 = ty * K::TH;
-        ox0 = tx * K::TW;
-        iy0 = oy0 * K::S - a.pt;
-        ix0 = ox0 * K::S - a.pl;
+        T.oy0 = ty * K::TH;
+        T.ox0 = tx * K::TW;
+        T.iy0 = T.oy0 * K::S - a.pt;
+        T.ix0 = T.ox0 * K::S - a.pl;
     } else {
-        oy0 = ty * K::TH - a.org_y;
-        ox0 = tx * K::TW - a.org_x;
-        iy0 = (oy0 + a.pt) / K::S - K::AH;  // oy0 + pt >= 0 and divisible by S
-        ix0 = (ox0 + a.pl) / K::S - K::AW;
+        T.oy0 = ty * K::TH - a.org_y;
+        T.ox0 = tx * K::TW - a.org_x;
+        T.iy0 = (T.oy0 + a.pt) / K::S - K::AH;  // oy0 + pt >= 0 and divisible by S
+        T.ix0 = (T.ox0 + a.pl) / K::S - K::AW;
     }
+    return T;
 }
 
 template <class K>
@@ -134,54 +139,72 @@ __global__ void __launch_bounds__(K::NT, 1)
     extern __shared__ __align__(128) unsigned char smem[];
     float4* stages = reinterpret_cast<float4*>(smem);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
 
     const int tid = threadIdx.x;
-    const int cv = tid % CV;
-    const int xi = (tid / CV) % K::WX;
-    const int yi = tid / (CV * K::WX);
+    const int warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
 
     if (tid == 0) {
-        prefetch_tensor_map(&tmap);
 #pragma unroll
-        for (int s = 0; s < K::NS; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
+        }
+        *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
-    auto issue = [&](int s, int t) {
-        int cb, tx, ty, n, oy0, ox0, iy0, ix0;
-        decode_tile(t, a, cb, tx, ty, n);
-        tile_origin<K>(a, tx, ty, oy0, ox0, iy0, ix0);
-        mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
-        tma_load_4d(stages + size_t(s) * K::STAGE_F4, &tmap, &full[s], cb * CB, ix0, iy0, n);
-    };
-    if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < K::NS; ++s) {
-            const int t = blockIdx.x + s * G;
-            if (t < a.ntiles) issue(s, t);
+    if (warp == K::NCW) {
+        // ---------------- producer warp: one lane issues every TMA load ----
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap);
+            int k = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
+                const int s = k % K::NS;
+                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const Tile T = decode_tile<K>(t, a);
+                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+                tma_load_4d(stages + size_t(s) * K::STAGE_F4, &tmap, &full[s], T.cb * CB, T.ix0,
+                            T.iy0, T.n);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                // let the loads already issued land before the CTA can exit
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
         }
+        return;
     }
+
+    // -------------------------- consumer warps --------------------------------
+    const int cv = tid % CV;
+    const int xi = (tid / CV) % K::WX;
+    const int yi = tid / (CV * K::WX);
+    const int r0 = K::TR ? yi * (K::THT / K::S) : yi * K::THT * K::S;
+    const int q0 = K::TR ? xi * (K::TWT / K::S) : xi * K::TWT * K::S;
+    const int j0 = yi * K::THT, i0 = xi * K::TWT;
+    const int64_t row_pitch = int64_t(a.Wout) * a.C;
 
     float4 wr[K::KH][K::KW];
     float4 bias = make_float4(0.f, 0.f, 0.f, 0.f);
     int cur_cb = -1;
-    // window origin of this thread inside a stage
-    const int r0 = K::TR ? yi * (K::THT / K::S) : yi * K::THT * K::S;
-    const int q0 = K::TR ? xi * (K::TWT / K::S) : xi * K::TWT * K::S;
-    const int j0 = yi * K::THT, i0 = xi * K::TWT;
 
     int k = 0;
     for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
         const int s = k % K::NS;
-        const uint32_t parity = (k / K::NS) & 1;
-        int cb, tx, ty, n, oy0, ox0, iy0, ix0;
-        decode_tile(t, a, cb, tx, ty, n);
-        tile_origin<K>(a, tx, ty, oy0, ox0, iy0, ix0);
-        const int c = cb * CB + cv * 4;
-        if (cb != cur_cb) {
-            cur_cb = cb;
+        const Tile T = decode_tile<K>(t, a);
+        const int c = T.cb * CB + cv * 4;
+        if (T.cb != cur_cb) {
+            cur_cb = T.cb;
             const bool live = c < a.C;
 #pragma unroll
             for (int kh = 0; kh < K::KH; ++kh)
@@ -200,7 +223,13 @@ __global__ void __launch_bounds__(K::NT, 1)
                                    __ldg(a.b + c + 3));
         }
 
-        const bool ok = mbar_wait_bounded(&full[s], parity);
+        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+            }
+            break;
+        }
 
         float4 acc[K::THT][K::TWT];
 #pragma unroll
@@ -238,41 +267,33 @@ __global__ void __launch_bounds__(K::NT, 1)
             });
         });
 
+        // every lane of this warp is done with stage s
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
         if (c < a.C) {
+            const int ho0 = T.oy0 + j0, wo0 = T.ox0 + i0;
+            float* base = a.out + (int64_t(T.n) * a.Hout + ho0) * row_pitch + int64_t(wo0) * a.C + c;
 #pragma unroll
             for (int j = 0; j < K::THT; ++j) {
-                const int ho = oy0 + j0 + j;
+                const int ho = ho0 + j;
                 if (ho < 0 || ho >= a.Hout) continue;
 #pragma unroll
                 for (int i = 0; i < K::TWT; ++i) {
-                    const int wo = ox0 + i0 + i;
+                    const int wo = wo0 + i;
                     if (wo < 0 || wo >= a.Wout) continue;
                     float4 v = acc[j][i];
                     if (!K::TR) {
                         v.x += bias.x; v.y += bias.y; v.z += bias.z; v.w += bias.w;
                     }
-                    store4(a.out + ((int64_t(n) * a.Hout + ho) * a.Wout + wo) * a.C + c, v);
+                    store4(base + j * row_pitch + int64_t(i) * a.C, v);
                 }
             }
-        }
-
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
-                for (int j = 1; j < K::NS; ++j) {  // let issued copies land
-                    const int t2 = t + j * G, k2 = k + j;
-                    if (t2 < a.ntiles) mbar_wait_bounded(&full[k2 % K::NS], (k2 / K::NS) & 1);
-                }
-            }
-            return;
-        }
-        if (tid == 0) {
-            const int tn = t + K::NS * G;
-            if (tn < a.ntiles) issue(s, tn);
         }
     }
 }
 
+// Launch attributes and the tensor map; `grid_cap` caps resident CTAs.
 template <class K>
 dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, const float* b,
                    float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
@@ -296,9 +317,9 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     const int64_t tc = (p.C + CB - 1) / CB;
     const int64_t nt = ty * tx * tc * p.N;
     if (nt >= INT_MAX || ty >= INT_MAX || tx >= INT_MAX) return DW_ERR_UNSUPPORTED;
-    a.tiles_y = static_cast<int>(ty);
-    a.tiles_x = static_cast<int>(tx);
-    a.tiles_c = static_cast<int>(tc);
+    a.tiles_y = make_fastdiv(static_cast<int>(ty));
+    a.tiles_x = make_fastdiv(static_cast<int>(tx));
+    a.tiles_c = make_fastdiv(static_cast<int>(tc));
     a.ntiles = static_cast<int>(nt);
     if (dry_run) return DW_OK;
 
@@ -321,29 +342,56 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
 
     int64_t grid = int64_t(sm_count(dev)) * occ;
     // keep each CTA on one channel block (weights loaded once per CTA)
-    if (grid >= a.tiles_c) grid -= grid % a.tiles_c;
-    if (grid > a.ntiles) grid = a.ntiles;
+    if (grid >= tc) grid -= grid % tc;
+    if (grid > nt) grid = nt;
     if (grid < 1) grid = 1;
     tiled_kernel<K><<<static_cast<unsigned>(grid), K::NT, K::SMEM, stream>>>(map, a);
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
+// Tiles a configuration would cut the problem into (host side).
+template <class K>
+int64_t tile_count(const Problem& p, Op op) {
+    const bool tr = op == OP_BWD_INPUT;
+    const int64_t Hout = tr ? p.H : p.Ho, Wout = tr ? p.W : p.Wo;
+    const int64_t oy = tr ? p.pt % K::S : 0, ox = tr ? p.pl % K::S : 0;
+    return ((Hout + oy + K::TH - 1) / K::TH) * ((Wout + ox + K::TW - 1) / K::TW) *
+           ((p.C + CB - 1) / CB) * p.N;
+}
+
+// Big tiles for large problems; small tiles when the big ones would leave
+// most SMs idle.
+template <class Big, class Small>
+dw_status_t launch_pick(const Problem& p, Op op, const float* in, const void* w, const float* b,
+                        float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    const int sms = dry_run ? 148 : sm_count(current_device());
+    if (tile_count<Big>(p, op) >= 2 * int64_t(sms))
+        return launch<Big>(p, op, in, w, b, out, stream, err, dry_run);
+    return launch<Small>(p, op, in, w, b, out, stream, err, dry_run);
+}
+
 // Instantiated configurations:   KH KW  S  D  TR   THT TWT WX WY NS
 using F33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4>;
-using F33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4>;
+using F33s1s = Cfg<3, 3, 1, 1, false, 1, 2, 8, 4, 4>;
+using F33s2 = Cfg<3, 3, 2, 1, false, 2, 2, 8, 4, 3>;
+using F33s2s = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4>;
 using F33d2 = Cfg<3, 3, 1, 2, false, 2, 4, 8, 4, 3>;
 using F33d3 = Cfg<3, 3, 1, 3, false, 2, 4, 8, 4, 3>;
 using F55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 3>;
+using F55s1s = Cfg<5, 5, 1, 1, false, 1, 2, 8, 4, 4>;
 using F1x3 = Cfg<1, 3, 1, 1, false, 1, 8, 16, 1, 4>;
 using F1x5 = Cfg<1, 5, 1, 1, false, 1, 8, 16, 1, 4>;
 using F1x7 = Cfg<1, 7, 1, 1, false, 1, 8, 16, 1, 4>;
 using F1x15 = Cfg<1, 15, 1, 1, false, 1, 8, 16, 1, 4>;
 using F1x31 = Cfg<1, 31, 1, 1, false, 1, 8, 16, 1, 4>;
 using B33s1 = Cfg<3, 3, 1, 1, true, 2, 4, 8, 4, 4>;
+using B33s1s = Cfg<3, 3, 1, 1, true, 1, 2, 8, 4, 4>;
 using B33s2 = Cfg<3, 3, 2, 1, true, 4, 4, 8, 4, 4>;
+using B33s2s = Cfg<3, 3, 2, 1, true, 2, 2, 8, 4, 4>;
 using B33d2 = Cfg<3, 3, 1, 2, true, 2, 4, 8, 4, 3>;
 using B33d3 = Cfg<3, 3, 1, 3, true, 2, 4, 8, 4, 3>;
 using B55s1 = Cfg<5, 5, 1, 1, true, 2, 4, 8, 4, 3>;
+using B55s1s = Cfg<5, 5, 1, 1, true, 1, 2, 8, 4, 4>;
 using B1x3 = Cfg<1, 3, 1, 1, true, 1, 8, 16, 1, 4>;
 using B1x5 = Cfg<1, 5, 1, 1, true, 1, 8, 16, 1, 4>;
 using B1x7 = Cfg<1, 7, 1, 1, true, 1, 8, 16, 1, 4>;
@@ -366,23 +414,26 @@ dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const float* in, const vo
     if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.C >= INT_MAX) return DW_ERR_UNSUPPORTED;
     const int S = p.sh, D = p.dh;
     const bool f = op == OP_FWD;
-#define DW_TRY(KH_, KW_, S_, D_, FC, BC)                                               \
-    if (p.kH == KH_ && p.kW == KW_ && S == S_ && D == D_)                                \
-        return f ? launch<FC>(p, op, in, w, b, out, stream, err, dry_run)              \
-                 : launch<BC>(p, op, in, w, b, out, stream, err, dry_run);
-    DW_TRY(3, 3, 1, 1, F33s1, B33s1)
-    DW_TRY(3, 3, 1, 2, F33d2, B33d2)
-    DW_TRY(3, 3, 1, 3, F33d3, B33d3)
-    DW_TRY(5, 5, 1, 1, F55s1, B55s1)
-    DW_TRY(1, 3, 1, 1, F1x3, B1x3)
-    DW_TRY(1, 5, 1, 1, F1x5, B1x5)
-    DW_TRY(1, 7, 1, 1, F1x7, B1x7)
-    DW_TRY(1, 15, 1, 1, F1x15, B1x15)
-    DW_TRY(1, 31, 1, 1, F1x31, B1x31)
-#undef DW_TRY
-    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1)
-        return f ? launch<F33s2>(p, op, in, w, b, out, stream, err, dry_run)
-                 : launch<B33s2>(p, op, in, w, b, out, stream, err, dry_run);
+#define DW_ONE(FC, BC)                                                  \
+    return f ? launch<FC>(p, op, in, w, b, out, stream, err, dry_run) \
+             : launch<BC>(p, op, in, w, b, out, stream, err, dry_run);
+#define DW_TWO(FC, FCS, BC, BCS)                                                      \
+    return f ? launch_pick<FC, FCS>(p, op, in, w, b, out, stream, err, dry_run)     \
+             : launch_pick<BC, BCS>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 1) DW_TWO(F33s1, F33s1s, B33s1, B33s1s)
+    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1) DW_TWO(F33s2, F33s2s, B33s2, B33s2s)
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 2) DW_ONE(F33d2, B33d2)
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 3) DW_ONE(F33d3, B33d3)
+    if (p.kH == 5 && p.kW == 5 && S == 1 && D == 1) DW_TWO(F55s1, F55s1s, B55s1, B55s1s)
+    if (p.kH == 1 && S == 1 && D == 1) {
+        if (p.kW == 3) DW_ONE(F1x3, B1x3)
+        if (p.kW == 5) DW_ONE(F1x5, B1x5)
+        if (p.kW == 7) DW_ONE(F1x7, B1x7)
+        if (p.kW == 15) DW_ONE(F1x15, B1x15)
+        if (p.kW == 31) DW_ONE(F1x31, B1x31)
+    }
+#undef DW_ONE
+#undef DW_TWO
     return DW_ERR_UNSUPPORTED;
 }
 
