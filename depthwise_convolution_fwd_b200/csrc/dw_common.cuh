@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "dwconv2d.h"
 
 namespace dw {
@@ -44,6 +46,23 @@ int sm_count(int dev);
 CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank,
                            void* base, const cuuint64_t* dims, const cuuint64_t* strides,
                            const cuuint32_t* box, const cuuint32_t* elem_strides);
+
+// Launch with programmatic stream serialization (see grid_dependency_wait).
+template <class... KArgs, class... Actual>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Actual&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Actual>(args)...);
+}
 
 // Per (kernel instantiation, device) cache of the launch attributes.
 struct LaunchCache {
@@ -167,6 +186,20 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
 
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialization, so it may be scheduled while the
+// previous kernel on the stream is still draining.  grid_dependency_wait()
+// blocks until every prerequisite grid has completed and its memory is
+// visible; each kernel calls it before its first global-memory access (read
+// or write), which keeps plain stream-order semantics for the caller.
+// allow_dependents() lets the next kernel on the stream start its prologue.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void fma4(float4& acc, const float4& v, const float4& w) {

@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(256) direct_fwd_kernel(const float* __restrict
                                                          const void* __restrict__ w,
                                                          const float* __restrict__ b,
                                                          float* __restrict__ y, DirectArgs a) {
+    grid_dependency_wait();
+    allow_dependents();
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.total; i += stride) {
         int64_t n, c, ho, wo;
@@ -71,6 +73,8 @@ template <int LAYOUT>
 __global__ void __launch_bounds__(256) direct_bwd_kernel(const float* __restrict__ dy,
                                                          const void* __restrict__ w,
                                                          float* __restrict__ dx, DirectArgs a) {
+    grid_dependency_wait();
+    allow_dependents();
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.total; i += stride) {
         int64_t n, c, hi, wi;
@@ -111,17 +115,18 @@ dw_status_t direct_launch(const Problem& p, Op op, const float* in, const void* 
     if (blocks > max_blocks) blocks = max_blocks;
     if (blocks < 1) blocks = 1;
     const dim3 grid(static_cast<unsigned>(blocks));
+    cudaError_t e;
+    const dim3 block(threads);
     if (op == OP_FWD) {
-        if (p.layout == DW_NHWC)
-            direct_fwd_kernel<DW_NHWC><<<grid, threads, 0, stream>>>(in, w, b, out, a);
-        else
-            direct_fwd_kernel<DW_NCHW><<<grid, threads, 0, stream>>>(in, w, b, out, a);
+        e = p.layout == DW_NHWC
+                ? launch_pdl(direct_fwd_kernel<DW_NHWC>, grid, block, 0, stream, in, w, b, out, a)
+                : launch_pdl(direct_fwd_kernel<DW_NCHW>, grid, block, 0, stream, in, w, b, out, a);
     } else {
-        if (p.layout == DW_NHWC)
-            direct_bwd_kernel<DW_NHWC><<<grid, threads, 0, stream>>>(in, w, out, a);
-        else
-            direct_bwd_kernel<DW_NCHW><<<grid, threads, 0, stream>>>(in, w, out, a);
+        e = p.layout == DW_NHWC
+                ? launch_pdl(direct_bwd_kernel<DW_NHWC>, grid, block, 0, stream, in, w, out, a)
+                : launch_pdl(direct_bwd_kernel<DW_NCHW>, grid, block, 0, stream, in, w, out, a);
     }
+    if (e != cudaSuccess) return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 

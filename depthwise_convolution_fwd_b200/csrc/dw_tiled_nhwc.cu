@@ -156,6 +156,8 @@ __global__ void __launch_bounds__(K::NT, 1)
         fence_mbar_init();
     }
     __syncthreads();
+    grid_dependency_wait();
+    allow_dependents();
 
     if (warp == K::NCW) {
         // ---------------- producer warp: one lane issues every TMA load ----
@@ -345,7 +347,9 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     if (grid >= tc) grid -= grid % tc;
     if (grid > nt) grid = nt;
     if (grid < 1) grid = 1;
-    tiled_kernel<K><<<static_cast<unsigned>(grid), K::NT, K::SMEM, stream>>>(map, a);
+    if (launch_pdl(tiled_kernel<K>, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM,
+                   stream, map, a) != cudaSuccess)
+        return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 

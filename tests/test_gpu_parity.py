@@ -282,3 +282,63 @@ def test_no_bias_and_aliasing_errors_on_device():
     with pytest.raises(dw.DwError) as e:
         dw.dwconv2d_fwd(x, inp["w"].cuda(), out=x)
     assert e.value.status == dw.DW_ERR_ALIAS
+
+
+# ------------------------------------------------- stream-order semantics --
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+@pytest.mark.parametrize("graph", [False, True])
+def test_dependent_calls_keep_stream_order(layout, graph):
+    """Kernels start early (programmatic dependent launch) but must not touch
+    memory before their predecessor on the stream has finished: a chain of
+    calls, each reading the previous call's output (tiled and direct kernels
+    alternating), must equal the oracle's composition."""
+    import oracle
+    N, H, W, C = 2, 40, 132, 64
+    shape = (N, H, W, C) if layout == "nhwc" else (N, C, H, W)
+    g = torch.Generator().manual_seed(99)
+    x = torch.rand(shape, generator=g) * 2 - 1
+    w3 = torch.randn(C, 3, 3, generator=g) / 3
+    w5 = torch.randn(C, 5, 5, generator=g) / 5
+    b = torch.rand(C, generator=g) * 0.2 - 0.1
+    xd, w3d, w5d, bd = x.cuda(), w3.cuda(), w5.cuda(), b.cuda()
+    stages = [("fwd", w3d, "tiled"), ("bwd", w5d, "direct"), ("fwd", w5d, "auto"),
+              ("bwd", w3d, "tiled"), ("fwd", w3d, "direct"), ("bwd", w3d, "auto")]
+
+    def chain(src):
+        t = src
+        for op, w, algo in stages:
+            if op == "fwd":
+                t = dw.dwconv2d_fwd(t, w, bd, layout=layout, algo=algo)
+            else:
+                t = dw.dwconv2d_bwd_input(t, w, (H, W), layout=layout, algo=algo)
+        return t
+
+    if graph:
+        chain(xd)  # warm-up outside capture
+        torch.cuda.synchronize()
+        static_in = xd.clone()
+        gr = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        with torch.cuda.graph(gr, stream=s):
+            out = chain(static_in)
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        got = out
+    else:
+        for _ in range(3):
+            got = chain(xd)
+        torch.cuda.synchronize()
+
+    p3 = oracle.problem(shape, 3, 3, 1, 1, "same", layout)
+    p5 = oracle.problem(shape, 5, 5, 1, 1, "same", layout)
+    ref = x.double().numpy()
+    wmap = {id(w3d): (p3, w3.double().numpy()), id(w5d): (p5, w5.double().numpy())}
+    for op, w, _ in stages:
+        p, wn = wmap[id(w)]
+        ref = oracle.fwd(p, ref, wn, b.double().numpy()) if op == "fwd" else \
+            oracle.bwd_input(p, ref, wn)
+    err = np.abs(got.cpu().double().numpy() - ref)
+    # six chained float32 passes: compare relative to the reference's scale
+    assert err.max() <= 1e-4 * np.abs(ref).max(), err.max()
