@@ -16,6 +16,11 @@
 // block of outputs: it streams the input cells of its block's window once
 // from shared memory and feeds every (output, tap) pair that reads that cell,
 // a register sliding window in both directions resolved at compile time.
+// Lane width VEC: 4 (a lane owns 4 channels as one float4; 8 lanes per pixel,
+// the memory-bound small kernels) or 1 (a lane owns one channel, a warp covers
+// the 32 channels of a pixel with 4-byte shared loads and 128-byte coalesced
+// stores; a thread then holds only kH*kW taps, so long and large kernels keep
+// many warps resident).
 //
 // Forward (LeanMlir Proofs/Architectures/Depthwise, "Depthwise conv2d
 // forward"): output (ho,wo) reads input (ho*S + kh*D - pt, wo*S + kw*D - pl);
@@ -35,8 +40,44 @@
 namespace dw {
 namespace nhwc {
 
-constexpr int CB = 32;      // channels per tile
-constexpr int CV = CB / 4;  // float4 lanes per pixel
+
+template <int VEC>
+struct VecOps;
+
+template <>
+struct VecOps<4> {
+    using T = float4;
+    static __device__ __forceinline__ T zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+    static __device__ __forceinline__ void fma(T& acc, const T& v, const T& w) { fma4(acc, v, w); }
+    static __device__ __forceinline__ T add(const T& a, const T& b) {
+        return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+    }
+    static __device__ __forceinline__ void store(float* p, const T& v) { store4(p, v); }
+    template <class WT>
+    static __device__ __forceinline__ T load_w(const WT* w, int64_t o, int step) {
+        return make_float4(float(w[o]), float(w[o + step]), float(w[o + 2 * step]),
+                           float(w[o + 3 * step]));
+    }
+    static __device__ __forceinline__ T load_b(const float* b, int c) {
+        return make_float4(__ldg(b + c), __ldg(b + c + 1), __ldg(b + c + 2), __ldg(b + c + 3));
+    }
+};
+
+template <>
+struct VecOps<1> {
+    using T = float;
+    static __device__ __forceinline__ T zero() { return 0.f; }
+    static __device__ __forceinline__ void fma(T& acc, const T& v, const T& w) {
+        acc = fmaf(v, w, acc);
+    }
+    static __device__ __forceinline__ T add(const T& a, const T& b) { return a + b; }
+    static __device__ __forceinline__ void store(float* p, const T& v) { *p = v; }
+    template <class WT>
+    static __device__ __forceinline__ T load_w(const WT* w, int64_t o, int) {
+        return float(w[o]);
+    }
+    static __device__ __forceinline__ T load_b(const float* b, int c) { return __ldg(b + c); }
+};
 
 struct Args {
     const void* w;
@@ -52,12 +93,24 @@ struct Args {
     int ntiles;
 };
 
-template <int KH_, int KW_, int S_, int D_, bool TR_, int THT_, int TWT_, int WX_, int WY_, int NS_>
+// NO: output staging buffers for the TMA-store epilogue (0 = results are
+// stored straight from registers).  MINB: CTAs per SM the register budget is
+// sized for.
+template <int KH_, int KW_, int S_, int D_, bool TR_, int THT_, int TWT_, int WX_, int WY_, int NS_,
+          int VEC_ = 4, int NO_ = 2, int MINB_ = 1, int CB_ = 32>
 struct Cfg {
+    static constexpr int CB = CB_;  // channels per tile
     static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
     static constexpr bool TR = TR_;
     static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
+    static constexpr int VEC = VEC_;
+    // transposed tiles with S > 1 may start at a negative row/column, where a
+    // TMA store must not start: those keep register stores
+    static constexpr int NO = (TR && S > 1) ? 0 : NO_;
+    static constexpr int MINB = MINB_;
+    static constexpr int CV = CB / VEC;  // lanes per pixel
     static constexpr int NCW = WX * WY * CV / 32;  // consumer warps
+    static constexpr int NCT = NCW * 32;           // consumer threads
     static constexpr int NT = NCW * 32 + 32;       // + one producer warp
     static constexpr int TH = THT * WY, TW = TWT * WX;
     static constexpr int AH = TR ? ((KH - 1) * D + S - 1) / S : 0;
@@ -67,9 +120,12 @@ struct Cfg {
     // rows / columns of the input window one thread reads
     static constexpr int RH = TR ? AH + (THT - 1) / S + 1 : (THT - 1) * S + (KH - 1) * D + 1;
     static constexpr int RW = TR ? AW + (TWT - 1) / S + 1 : (TWT - 1) * S + (KW - 1) * D + 1;
-    static constexpr int STAGE_F4 = IH * IW * CV;
-    static constexpr int STAGE_BYTES = STAGE_F4 * 16;
-    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(2 * NS) * 8 + 16;
+    static constexpr int STAGE_V = IH * IW * CV;  // stage size in lane vectors
+    static constexpr int STAGE_BYTES = IH * IW * CB * 4;
+    static constexpr int OUT_V = TH * TW * CV;  // output staging buffer in lane vectors
+    static constexpr int OUT_BYTES = TH * TW * CB * 4;
+    static constexpr size_t SMEM =
+        size_t(NS) * STAGE_BYTES + size_t(NO) * OUT_BYTES + size_t(2 * NS) * 8 + 16;
     static_assert((WX * WY * CV) % 32 == 0, "whole consumer warps");
     static_assert(IH <= 256 && IW <= 256, "TMA box dimension limit");
     // every stage starts on a 128-byte boundary (tensor-copy destination rule)
@@ -134,11 +190,17 @@ __device__ __forceinline__ Tile decode_tile(int t, const Args& a) {
 }
 
 template <class K>
-__global__ void __launch_bounds__(K::NT, 1)
-    tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
+__global__ void __launch_bounds__(K::NT, K::MINB)
+    tiled_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
+                 const Args a) {
+    using VO = VecOps<K::VEC>;
+    using V = typename VO::T;
+    constexpr int CV = K::CV;
     extern __shared__ __align__(128) unsigned char smem[];
-    float4* stages = reinterpret_cast<float4*>(smem);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+    V* stages = reinterpret_cast<V*>(smem);
+    V* outbuf = reinterpret_cast<V*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES +
+                                                 size_t(K::NO) * K::OUT_BYTES);
     uint64_t* empty = full + K::NS;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
 
@@ -163,6 +225,7 @@ __global__ void __launch_bounds__(K::NT, 1)
         // ---------------- producer warp: one lane issues every TMA load ----
         if (lane == 0) {
             prefetch_tensor_map(&tmap);
+            if constexpr (K::NO > 0) prefetch_tensor_map(&omap);
             int k = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
@@ -173,7 +236,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                 }
                 const Tile T = decode_tile<K>(t, a);
                 mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
-                tma_load_4d(stages + size_t(s) * K::STAGE_F4, &tmap, &full[s], T.cb * CB, T.ix0,
+                tma_load_4d(stages + size_t(s) * K::STAGE_V, &tmap, &full[s], T.cb * K::CB, T.ix0,
                             T.iy0, T.n);
             }
             if (!ok) {
@@ -196,50 +259,66 @@ __global__ void __launch_bounds__(K::NT, 1)
     const int j0 = yi * K::THT, i0 = xi * K::TWT;
     const int64_t row_pitch = int64_t(a.Wout) * a.C;
 
-    float4 wr[K::KH][K::KW];
-    float4 bias = make_float4(0.f, 0.f, 0.f, 0.f);
+    V wr[K::KH][K::KW];
+    V bias = VO::zero();
     int cur_cb = -1;
 
     int k = 0;
     for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
         const int s = k % K::NS;
         const Tile T = decode_tile<K>(t, a);
-        const int c = T.cb * CB + cv * 4;
+        const int c = T.cb * K::CB + cv * K::VEC;
         if (T.cb != cur_cb) {
             cur_cb = T.cb;
             const bool live = c < a.C;
+            constexpr int step = K::KH * K::KW;
+            const int64_t o = int64_t(live ? c : 0) * step;
+            // one branch on the weight type, then straight loads
+            if (a.wtype == DW_F16) {
+                const __half* wp = static_cast<const __half*>(a.w);
 #pragma unroll
-            for (int kh = 0; kh < K::KH; ++kh)
+                for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
-                for (int kw = 0; kw < K::KW; ++kw) {
-                    const int64_t o = int64_t(c) * (K::KH * K::KW) + kh * K::KW + kw;
-                    constexpr int step = K::KH * K::KW;
-                    wr[kh][kw] = live ? make_float4(load_weight(a.w, a.wtype, o),
-                                                    load_weight(a.w, a.wtype, o + step),
-                                                    load_weight(a.w, a.wtype, o + 2 * step),
-                                                    load_weight(a.w, a.wtype, o + 3 * step))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            if (!K::TR && a.b != nullptr && live)
-                bias = make_float4(__ldg(a.b + c), __ldg(a.b + c + 1), __ldg(a.b + c + 2),
-                                   __ldg(a.b + c + 3));
-        }
-
-        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
-            if (lane == 0) {
-                *abort_flag = 1;
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                    for (int kw = 0; kw < K::KW; ++kw)
+                        wr[kh][kw] = VO::load_w(wp, o + kh * K::KW + kw, step);
+            } else {
+                const float* wp = static_cast<const float*>(a.w);
+#pragma unroll
+                for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                    for (int kw = 0; kw < K::KW; ++kw)
+                        wr[kh][kw] = VO::load_w(wp, o + kh * K::KW + kw, step);
             }
-            break;
+            if (!live) {
+#pragma unroll
+                for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                    for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] = VO::zero();
+            }
+            if (!K::TR && a.b != nullptr && live) bias = VO::load_b(a.b, c);
         }
 
-        float4 acc[K::THT][K::TWT];
+        const bool ok = mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag);
+        if constexpr (K::NO == 0) {
+            if (!ok) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                }
+                break;
+            }
+        }
+        // (with the TMA-store epilogue a failed wait is acted on at the
+        // consumer barrier below, so every consumer leaves together; the
+        // shared-memory reads in between stay inside the stage)
+
+        V acc[K::THT][K::TWT];
 #pragma unroll
         for (int j = 0; j < K::THT; ++j)
 #pragma unroll
-            for (int i = 0; i < K::TWT; ++i) acc[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < K::TWT; ++i) acc[j][i] = VO::zero();
 
-        const float4* win = stages + size_t(s) * K::STAGE_F4 + (r0 * K::IW + q0) * CV + cv;
+        const V* win = stages + size_t(s) * K::STAGE_V + (r0 * K::IW + q0) * CV + cv;
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             static_for<0, K::RW>([&](auto q_) {
@@ -253,7 +332,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                     return false;
                 }();
                 if constexpr (used) {
-                    const float4 v = win[(r * K::IW + q) * CV];
+                    const V v = win[(r * K::IW + q) * CV];
                     static_for<0, K::THT>([&](auto j_) {
                         constexpr int j = decltype(j_)::value;
                         constexpr int kh = tap_for<K, true>(r, j);
@@ -261,7 +340,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                             static_for<0, K::TWT>([&](auto i_) {
                                 constexpr int i = decltype(i_)::value;
                                 constexpr int kw = tap_for<K, false>(q, i);
-                                if constexpr (kw >= 0) fma4(acc[j][i], v, wr[kh][kw]);
+                                if constexpr (kw >= 0) VO::fma(acc[j][i], v, wr[kh][kw]);
                             });
                         }
                     });
@@ -273,7 +352,33 @@ __global__ void __launch_bounds__(K::NT, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
-        if (c < a.C) {
+        if constexpr (K::NO > 0) {
+            // ------- epilogue: registers -> staging buffer -> TMA store ----
+            const int ob = k % K::NO;
+            if (k >= K::NO) {
+                // the store issued NO tiles ago must be done reading buffer ob
+                if (tid == 0) bulk_wait_group_read<K::NO - 1>();
+                named_barrier_sync(1, K::NCT);
+            }
+            V* o = outbuf + size_t(ob) * K::OUT_V + (j0 * K::TW + i0) * CV + cv;
+#pragma unroll
+            for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+                for (int i = 0; i < K::TWT; ++i)
+                    o[(j * K::TW + i) * CV] = K::TR ? acc[j][i] : VO::add(acc[j][i], bias);
+            fence_proxy_async_smem();
+            if (named_barrier_or(1, K::NCT, !ok)) {
+                if (tid == 0) {
+                    *abort_flag = 1;
+                    atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                }
+                break;
+            }
+            if (tid == 0) {
+                tma_store_4d(&omap, outbuf + size_t(ob) * K::OUT_V, T.cb * K::CB, T.ox0, T.oy0, T.n);
+                bulk_commit_group();
+            }
+        } else if (c < a.C) {
             const int ho0 = T.oy0 + j0, wo0 = T.ox0 + i0;
             float* base = a.out + (int64_t(T.n) * a.Hout + ho0) * row_pitch + int64_t(wo0) * a.C + c;
 #pragma unroll
@@ -284,14 +389,15 @@ __global__ void __launch_bounds__(K::NT, 1)
                 for (int i = 0; i < K::TWT; ++i) {
                     const int wo = wo0 + i;
                     if (wo < 0 || wo >= a.Wout) continue;
-                    float4 v = acc[j][i];
-                    if (!K::TR) {
-                        v.x += bias.x; v.y += bias.y; v.z += bias.z; v.w += bias.w;
-                    }
-                    store4(base + j * row_pitch + int64_t(i) * a.C, v);
+                    const V v = K::TR ? acc[j][i] : VO::add(acc[j][i], bias);
+                    VO::store(base + j * row_pitch + int64_t(i) * a.C, v);
                 }
             }
         }
+    }
+    // stores issued by this CTA complete before it exits
+    if constexpr (K::NO > 0) {
+        if (tid == 0) bulk_wait_group<0>();
     }
 }
 
@@ -316,7 +422,7 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     a.org_x = tr ? p.pl % K::S : 0;
     const int64_t ty = (a.Hout + a.org_y + K::TH - 1) / K::TH;
     const int64_t tx = (a.Wout + a.org_x + K::TW - 1) / K::TW;
-    const int64_t tc = (p.C + CB - 1) / CB;
+    const int64_t tc = (p.C + K::CB - 1) / K::CB;
     const int64_t nt = ty * tx * tc * p.N;
     if (nt >= INT_MAX || ty >= INT_MAX || tx >= INT_MAX) return DW_ERR_UNSUPPORTED;
     a.tiles_y = make_fastdiv(static_cast<int>(ty));
@@ -336,11 +442,23 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     const cuuint64_t dims[4] = {cuuint64_t(p.C), cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.N)};
     const cuuint64_t strides[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * Win) * 4,
                                    cuuint64_t(p.C * Win * Hin) * 4};
-    const cuuint32_t box[4] = {CB, K::IW, K::IH, 1};
+    const cuuint32_t box[4] = {K::CB, K::IW, K::IH, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
                           strides, box, estr) != CUDA_SUCCESS)
         return DW_ERR_CUDA;
+    // output map: the staging buffer is a [TH][TW][32] box of the output
+    CUtensorMap omap = map;
+    if constexpr (K::NO > 0) {
+        const cuuint64_t odims[4] = {cuuint64_t(p.C), cuuint64_t(a.Wout), cuuint64_t(a.Hout),
+                                     cuuint64_t(p.N)};
+        const cuuint64_t ostrides[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C) * a.Wout * 4,
+                                        cuuint64_t(p.C) * a.Wout * a.Hout * 4};
+        const cuuint32_t obox[4] = {K::CB, K::TW, K::TH, 1};
+        if (encode_tensor_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out, odims, ostrides,
+                              obox, estr) != CUDA_SUCCESS)
+            return DW_ERR_CUDA;
+    }
 
     int64_t grid = int64_t(sm_count(dev)) * occ;
     // keep each CTA on one channel block (weights loaded once per CTA)
@@ -348,7 +466,7 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     if (grid > nt) grid = nt;
     if (grid < 1) grid = 1;
     if (launch_pdl(tiled_kernel<K>, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM,
-                   stream, map, a) != cudaSuccess)
+                   stream, map, omap, a) != cudaSuccess)
         return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
@@ -360,7 +478,7 @@ int64_t tile_count(const Problem& p, Op op) {
     const int64_t Hout = tr ? p.H : p.Ho, Wout = tr ? p.W : p.Wo;
     const int64_t oy = tr ? p.pt % K::S : 0, ox = tr ? p.pl % K::S : 0;
     return ((Hout + oy + K::TH - 1) / K::TH) * ((Wout + ox + K::TW - 1) / K::TW) *
-           ((p.C + CB - 1) / CB) * p.N;
+           ((p.C + K::CB - 1) / K::CB) * p.N;
 }
 
 // Big tiles for large problems; small tiles when the big ones would leave
@@ -374,33 +492,35 @@ dw_status_t launch_pick(const Problem& p, Op op, const float* in, const void* w,
     return launch<Small>(p, op, in, w, b, out, stream, err, dry_run);
 }
 
-// Instantiated configurations:   KH KW  S  D  TR   THT TWT WX WY NS
-using F33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4>;
-using F33s1s = Cfg<3, 3, 1, 1, false, 1, 2, 8, 4, 4>;
-using F33s2 = Cfg<3, 3, 2, 1, false, 2, 2, 8, 4, 3>;
-using F33s2s = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4>;
-using F33d2 = Cfg<3, 3, 1, 2, false, 2, 4, 8, 4, 3>;
-using F33d3 = Cfg<3, 3, 1, 3, false, 2, 4, 8, 4, 3>;
-using F55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 3>;
-using F55s1s = Cfg<5, 5, 1, 1, false, 1, 2, 8, 4, 4>;
+// Instantiated configurations (KH KW S D TR | THT TWT WX WY NS [VEC NO MINB CB]);
+// shared memory = NS input stages + NO output staging buffers <= 227 KB.
+using F33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4, 4, 0, 2>;
+using F33s1s = Cfg<3, 3, 1, 1, false, 2, 4, 4, 2, 4, 1, 2, 2>;
+using F33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4, 4, 0, 2>;
+using F33d2 = Cfg<3, 3, 1, 2, false, 2, 4, 8, 4, 2>;
+using F33d3 = Cfg<3, 3, 1, 3, false, 2, 4, 8, 4, 2>;
+using F55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 2>;
+using F55s1s = Cfg<5, 5, 1, 1, false, 2, 4, 4, 2, 4, 1, 2, 2>;
 using F1x3 = Cfg<1, 3, 1, 1, false, 1, 8, 16, 1, 4>;
 using F1x5 = Cfg<1, 5, 1, 1, false, 1, 8, 16, 1, 4>;
 using F1x7 = Cfg<1, 7, 1, 1, false, 1, 8, 16, 1, 4>;
-using F1x15 = Cfg<1, 15, 1, 1, false, 1, 8, 16, 1, 4>;
-using F1x31 = Cfg<1, 31, 1, 1, false, 1, 8, 16, 1, 4>;
-using B33s1 = Cfg<3, 3, 1, 1, true, 2, 4, 8, 4, 4>;
-using B33s1s = Cfg<3, 3, 1, 1, true, 1, 2, 8, 4, 4>;
+using F1x15 = Cfg<1, 15, 1, 1, false, 1, 16, 8, 1, 4, 1>;
+using F1x31 = Cfg<1, 31, 1, 1, false, 1, 16, 2, 1, 4, 1, 2, 1, 128>;
+using F77s1 = Cfg<7, 7, 1, 1, false, 2, 4, 4, 2, 3, 1>;
+using B33s1 = Cfg<3, 3, 1, 1, true, 2, 4, 8, 4, 4, 4, 0, 2>;
+using B33s1s = Cfg<3, 3, 1, 1, true, 2, 4, 4, 2, 4, 1, 2, 2>;
 using B33s2 = Cfg<3, 3, 2, 1, true, 4, 4, 8, 4, 4>;
 using B33s2s = Cfg<3, 3, 2, 1, true, 2, 2, 8, 4, 4>;
-using B33d2 = Cfg<3, 3, 1, 2, true, 2, 4, 8, 4, 3>;
-using B33d3 = Cfg<3, 3, 1, 3, true, 2, 4, 8, 4, 3>;
-using B55s1 = Cfg<5, 5, 1, 1, true, 2, 4, 8, 4, 3>;
-using B55s1s = Cfg<5, 5, 1, 1, true, 1, 2, 8, 4, 4>;
+using B33d2 = Cfg<3, 3, 1, 2, true, 2, 4, 8, 4, 2>;
+using B33d3 = Cfg<3, 3, 1, 3, true, 2, 4, 8, 4, 2>;
+using B55s1 = Cfg<5, 5, 1, 1, true, 2, 4, 8, 4, 2>;
+using B55s1s = Cfg<5, 5, 1, 1, true, 2, 4, 4, 2, 4, 1, 2, 2>;
 using B1x3 = Cfg<1, 3, 1, 1, true, 1, 8, 16, 1, 4>;
 using B1x5 = Cfg<1, 5, 1, 1, true, 1, 8, 16, 1, 4>;
 using B1x7 = Cfg<1, 7, 1, 1, true, 1, 8, 16, 1, 4>;
-using B1x15 = Cfg<1, 15, 1, 1, true, 1, 8, 16, 1, 4>;
-using B1x31 = Cfg<1, 31, 1, 1, true, 1, 8, 16, 1, 4>;
+using B1x15 = Cfg<1, 15, 1, 1, true, 1, 16, 8, 1, 4, 1>;
+using B1x31 = Cfg<1, 31, 1, 1, true, 1, 16, 2, 1, 4, 1, 2, 1, 128>;
+using B77s1 = Cfg<7, 7, 1, 1, true, 2, 4, 4, 2, 3, 1>;
 
 }  // namespace nhwc
 
@@ -425,10 +545,13 @@ dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const float* in, const vo
     return f ? launch_pick<FC, FCS>(p, op, in, w, b, out, stream, err, dry_run)     \
              : launch_pick<BC, BCS>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 3 && p.kW == 3 && S == 1 && D == 1) DW_TWO(F33s1, F33s1s, B33s1, B33s1s)
-    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1) DW_TWO(F33s2, F33s2s, B33s2, B33s2s)
+    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1)
+        return f ? launch<F33s2>(p, op, in, w, b, out, stream, err, dry_run)
+                 : launch_pick<B33s2, B33s2s>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 3 && p.kW == 3 && S == 1 && D == 2) DW_ONE(F33d2, B33d2)
     if (p.kH == 3 && p.kW == 3 && S == 1 && D == 3) DW_ONE(F33d3, B33d3)
     if (p.kH == 5 && p.kW == 5 && S == 1 && D == 1) DW_TWO(F55s1, F55s1s, B55s1, B55s1s)
+    if (p.kH == 7 && p.kW == 7 && S == 1 && D == 1) DW_ONE(F77s1, B77s1)
     if (p.kH == 1 && S == 1 && D == 1) {
         if (p.kW == 3) DW_ONE(F1x3, B1x3)
         if (p.kW == 5) DW_ONE(F1x5, B1x5)
