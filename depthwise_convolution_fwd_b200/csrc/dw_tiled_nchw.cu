@@ -295,6 +295,285 @@ dw_status_t launch(const Problem& p, const float* in, const void* w, const float
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Channel-lane kernel for 1 x kW filters (the long 1-D kernels): one TMA box
+// is 32 channel rows x the W halo of one output row; lane = channel row,
+// warp = W strip, each thread computes TWT consecutive outputs of its own
+// channel with its kW taps in registers, streaming its window from shared
+// memory once.  The stage row pitch IWB is chosen with IWB/4 odd, so the
+// 32 lanes' 16-byte reads (32 different rows, same column) fall in distinct
+// bank groups and never conflict.  Results leave through a per-warp TMA
+// store: each warp stages its 32-row x TWT-column block in its own
+// double-buffered slot and one lane issues the bulk store (the tensor engine
+// does the 32-row scatter); when the output row pitch is not a multiple of
+// 16 bytes they are stored from registers instead.
+template <int KW_, bool REV_, int REM_, int TWT_, int NCW_, int NS_>
+struct ClCfg {
+    static constexpr int KW = KW_, REM = REM_, TWT = TWT_, NCW = NCW_, NS = NS_;
+    static constexpr bool REV = REV_;
+    static constexpr int CH = 32;  // channel rows per tile (lanes)
+    static constexpr int NT = NCW * 32 + 32;
+    static constexpr int TW = TWT * NCW;
+    static constexpr int IWB0 = (REM + TW + (KW - 1) + 3) / 4 * 4;
+    static constexpr int IWB = (IWB0 / 4) % 2 == 1 ? IWB0 : IWB0 + 4;
+    static constexpr int STAGE_BYTES = IWB * CH * 4;
+    static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
+    static constexpr int STAGE_FLOATS = STAGE_PITCH / 4;
+    static constexpr int NV = (REM + TWT + KW - 1 + 3) / 4;  // float4 per thread window
+    static constexpr int OUT_FLOATS = CH * TWT;  // one warp's staging slot
+    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NCW) * OUT_FLOATS * 4 +
+                                   size_t(2 * NS) * 8 + 16;
+    static_assert(TWT % 4 == 0, "thread strips are whole float4s");
+    static_assert((OUT_FLOATS * 4) % 128 == 0, "staging slots on 128-byte boundaries");
+    static_assert(IWB <= 256, "TMA box dimension limit");
+    static_assert((IWB / 4) % 2 == 1, "conflict-free row pitch");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    chl_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
+               const Args a, const int tma_store) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    float* stages = reinterpret_cast<float*>(smem);
+    float* outbuf = reinterpret_cast<float*>(smem + size_t(K::NS) * K::STAGE_PITCH);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH +
+                                                 size_t(2 * K::NCW) * K::OUT_FLOATS * 4);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int t_begin = int((int64_t(blockIdx.x) * a.ntiles) / gridDim.x);
+    const int t_end = int((int64_t(blockIdx.x + 1) * a.ntiles) / gridDim.x);
+
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    allow_dependents();
+
+    if (warp == K::NCW) {
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap);
+            int k = 0;
+            bool ok = true;
+            for (int t = t_begin; t < t_end; ++t, ++k) {
+                const int s = k % K::NS;
+                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                int tx, h, cg, n;
+                decode_tile<K>(t, a, tx, h, cg, n);
+                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+                tma_load_4d(stages + size_t(s) * K::STAGE_FLOATS, &tmap, &full[s],
+                            tx * K::TW - a.pl - K::REM, h - a.pt, cg * K::CH, n);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
+        }
+        return;
+    }
+
+    float wr[K::KW];
+    float bias = 0.f;
+    int cur_key = -1;
+    bool live = false;
+    int k = 0;
+    for (int t = t_begin; t < t_end; ++t, ++k) {
+        const int s = k % K::NS;
+        int tx, h, cg, n;
+        decode_tile<K>(t, a, tx, h, cg, n);
+        const int c = cg * K::CH + lane;
+        const int key = cg + n * a.tiles_c.d;
+        if (key != cur_key) {
+            cur_key = key;
+            live = c < a.C;
+            const int64_t base = int64_t(live ? c : 0) * K::KW;
+            if (a.wtype == DW_F16) {
+                const __half* wp = static_cast<const __half*>(a.w) + base;
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw)
+                    wr[kw] = __half2float(wp[K::REV ? K::KW - 1 - kw : kw]);
+            } else {
+                const float* wp = static_cast<const float*>(a.w) + base;
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw) wr[kw] = __ldg(wp + (K::REV ? K::KW - 1 - kw : kw));
+            }
+            bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
+        }
+
+        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+            }
+            break;
+        }
+
+        float acc[K::TWT];
+#pragma unroll
+        for (int i = 0; i < K::TWT; ++i) acc[i] = 0.f;
+        const float4* win = reinterpret_cast<const float4*>(stages + size_t(s) * K::STAGE_FLOATS) +
+                            lane * (K::IWB / 4) + warp * (K::TWT / 4);
+        static_for<0, K::NV>([&](auto u_) {
+            constexpr int u = decltype(u_)::value;
+            const float4 f = win[u];
+            const float e[4] = {f.x, f.y, f.z, f.w};
+            static_for<0, 4>([&](auto m_) {
+                constexpr int q = 4 * u + decltype(m_)::value - K::REM;  // window column
+                static_for<0, K::TWT>([&](auto i_) {
+                    constexpr int i = decltype(i_)::value;
+                    constexpr int kw = q - i;
+                    if constexpr (kw >= 0 && kw < K::KW)
+                        acc[i] = fmaf(e[decltype(m_)::value], wr[kw], acc[i]);
+                });
+            });
+        });
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
+        if (tma_store) {
+            // warp-private staging slot ob: the store issued two tiles ago
+            // by this warp must have finished reading it
+            const int ob = k & 1;
+            if (k >= 2 && lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            float4* o = reinterpret_cast<float4*>(outbuf + size_t(2 * warp + ob) * K::OUT_FLOATS) +
+                        lane * (K::TWT / 4);
+#pragma unroll
+            for (int u = 0; u < K::TWT / 4; ++u)
+                o[u] = make_float4(acc[4 * u] + bias, acc[4 * u + 1] + bias, acc[4 * u + 2] + bias,
+                                   acc[4 * u + 3] + bias);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_4d(&omap, outbuf + size_t(2 * warp + ob) * K::OUT_FLOATS,
+                             tx * K::TW + warp * K::TWT, h, cg * K::CH, n);
+                bulk_commit_group();
+            }
+        } else if (live && h < a.Hout) {
+            const int wo0 = tx * K::TW + warp * K::TWT;
+            float* dst = a.out + ((int64_t(n) * a.C + c) * a.Hout + h) * a.Wout + wo0;
+            const bool vec = (a.Wout & 3) == 0;
+#pragma unroll
+            for (int u = 0; u < K::TWT / 4; ++u) {
+                const float4 v = make_float4(acc[4 * u] + bias, acc[4 * u + 1] + bias,
+                                             acc[4 * u + 2] + bias, acc[4 * u + 3] + bias);
+                const int wo = wo0 + 4 * u;
+                if (vec && wo + 3 < a.Wout) {
+                    store4(dst + 4 * u, v);
+                } else {
+                    if (wo < a.Wout) dst[4 * u] = v.x;
+                    if (wo + 1 < a.Wout) dst[4 * u + 1] = v.y;
+                    if (wo + 2 < a.Wout) dst[4 * u + 2] = v.z;
+                    if (wo + 3 < a.Wout) dst[4 * u + 3] = v.w;
+                }
+            }
+        }
+    }
+    if (tma_store && lane == 0) bulk_wait_group<0>();
+}
+
+template <class K>
+dw_status_t launch_chl(const Problem& p, const float* in, const void* w, const float* b,
+                       float* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
+                       int pl_eff) {
+    const int64_t Hin = K::REV ? p.Ho : p.H, Win = K::REV ? p.Wo : p.W;
+    Args a;
+    a.w = w;
+    a.b = K::REV ? nullptr : b;
+    a.out = out;
+    a.err = err;
+    a.wtype = p.wtype;
+    a.N = static_cast<int>(p.N);
+    a.C = static_cast<int>(p.C);
+    a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
+    a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
+    a.pt = pt_eff;
+    a.pl = pl_eff;
+    const int64_t tx = (a.Wout + K::TW - 1) / K::TW;
+    const int64_t ty = a.Hout;
+    const int64_t tc = (p.C + K::CH - 1) / K::CH;
+    const int64_t nt = tx * ty * tc * p.N;
+    if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.tiles_x = make_fastdiv(static_cast<int>(tx));
+    a.tiles_y = make_fastdiv(static_cast<int>(ty));
+    a.tiles_c = make_fastdiv(static_cast<int>(tc));
+    a.ntiles = static_cast<int>(nt);
+    if (dry_run) return DW_OK;
+
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&chl_kernel<K>), K::NT, K::SMEM,
+                                   cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+    CUtensorMap map;
+    const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t strides[3] = {cuuint64_t(Win) * 4, cuuint64_t(Win * Hin) * 4,
+                                   cuuint64_t(Win * Hin * p.C) * 4};
+    const cuuint32_t box[4] = {K::IWB, 1, K::CH, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
+                          strides, box, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+    // output map for the per-warp bulk stores (row pitch must be a multiple
+    // of 16 bytes, as for every tensor map)
+    CUtensorMap omap = map;
+    int tma_store = 0;
+    if ((a.Wout & 3) == 0) {
+        const cuuint64_t odims[4] = {cuuint64_t(a.Wout), cuuint64_t(a.Hout), cuuint64_t(p.C),
+                                     cuuint64_t(p.N)};
+        const cuuint64_t ostrides[3] = {cuuint64_t(a.Wout) * 4, cuuint64_t(a.Wout) * a.Hout * 4,
+                                        cuuint64_t(a.Wout) * a.Hout * p.C * 4};
+        const cuuint32_t obox[4] = {K::TWT, 1, K::CH, 1};
+        if (encode_tensor_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out, odims, ostrides,
+                              obox, estr) != CUDA_SUCCESS)
+            return DW_ERR_CUDA;
+        tma_store = 1;
+    }
+    int64_t grid = int64_t(sm_count(dev)) * occ;
+    if (grid > a.ntiles) grid = a.ntiles;
+    if (launch_pdl(chl_kernel<K>, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream,
+                   map, omap, a, tma_store) != cudaSuccess)
+        return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+template <int KW, bool REV, int TWT, int NCW, int NS>
+dw_status_t launch_chl_rem(const Problem& p, const float* in, const void* w, const float* b,
+                           float* out, cudaStream_t stream, int32_t* err, bool dry_run,
+                           int pt_eff, int pl_eff) {
+    switch (((-pl_eff) % 4 + 4) % 4) {
+        case 0: return launch_chl<ClCfg<KW, REV, 0, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 1: return launch_chl<ClCfg<KW, REV, 1, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 2: return launch_chl<ClCfg<KW, REV, 2, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        default: return launch_chl<ClCfg<KW, REV, 3, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+    }
+}
+
+template <int KW, int TWT, int NCW, int NS>
+dw_status_t launch_chl_op(const Problem& p, Op op, const float* in, const void* w, const float* b,
+                          float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (op == OP_FWD)
+        return launch_chl_rem<KW, false, TWT, NCW, NS>(p, in, w, b, out, stream, err, dry_run,
+                                                       p.pt, p.pl);
+    return launch_chl_rem<KW, true, TWT, NCW, NS>(p, in, w, b, out, stream, err, dry_run, -p.pt,
+                                                  (KW - 1) - p.pl);
+}
+
 template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS>
 dw_status_t launch_rem(const Problem& p, const float* in, const void* w, const float* b,
                        float* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
@@ -337,8 +616,9 @@ dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const vo
     if (p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 7 && p.kW == 7) return launch_op<7, 7, 4, 32, 4, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    if (p.kH == 1 && p.kW == 15) return launch_op<1, 15, 1, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    if (p.kH == 1 && p.kW == 31) return launch_op<1, 31, 1, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    //                                           KW TWT NCW NS
+    if (p.kH == 1 && p.kW == 15) return launch_chl_op<15, 16, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 1 && p.kW == 31) return launch_chl_op<31, 16, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
     return DW_ERR_UNSUPPORTED;
 }
 

@@ -342,3 +342,25 @@ def test_dependent_calls_keep_stream_order(layout, graph):
     err = np.abs(got.cpu().double().numpy() - ref)
     # six chained float32 passes: compare relative to the reference's scale
     assert err.max() <= 1e-4 * np.abs(ref).max(), err.max()
+
+
+@pytest.mark.parametrize("case", [
+    Case("rw_nchw_1x31", 3, 2, 132, 40, 1, 31, padding=(0, 0, 3, 2), layout="nchw",
+         act="normal", seed=61),
+    Case("rw_nchw_1x15", 2, 3, 260, 36, 1, 15, padding=(1, 0, 0, 1), layout="nchw",
+         act="normal", seed=62),
+    Case("rw_nchw_3x3", 2, 33, 132, 6, 3, 3, padding=(1, 1, 1, 0), layout="nchw", seed=63),
+], ids=lambda c: c.name)
+def test_tiled_forward_with_ragged_output_width(case):
+    """Forward on the tiled path where the output row pitch is not a
+    multiple of 16 bytes (the epilogue falls back to register stores)."""
+    inp = gu.inputs(case)
+    x = inp["x"].cuda()
+    w = inp["w"].cuda()
+    y = torch.empty(case.out_shape(*gu.out_hw(case)), device="cuda")
+    assert gu.out_hw(case)[1] % 4 != 0
+    assert gu.chosen_algo(case, 0, x, w, y) == dw.DW_ALGO_TILED
+    ref, sc = gu.reference_fwd(case, inp)
+    got = gu.gpu_fwd(case, inp, algo="tiled")
+    torch.cuda.synchronize()
+    gu.assert_close(got.cpu().numpy(), ref, sc, case.name)
