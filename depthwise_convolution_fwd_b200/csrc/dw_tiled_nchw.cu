@@ -39,8 +39,10 @@ struct Args {
     int ntiles;
 };
 
-template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_>
+template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
+          int MINB_ = 1>
 struct Cfg {
+    static constexpr int MINB = MINB_;  // CTAs per SM the register budget is sized for
     static constexpr int KH = KH_, KW = KW_, D = D_, REM = REM_;
     static constexpr bool REV = REV_;
     static constexpr bool ROWS = KH == 1;  // 1-D: thread rows are channels
@@ -88,7 +90,7 @@ __device__ __forceinline__ void decode_tile(int t, const Args& a, int& tx, int& 
 }
 
 template <class K>
-__global__ void __launch_bounds__(K::NT, 1)
+__global__ void __launch_bounds__(K::NT, K::MINB)
     tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
     extern __shared__ __align__(128) unsigned char smem[];
     float* stages = reinterpret_cast<float*>(smem);
@@ -574,26 +576,26 @@ dw_status_t launch_chl_op(const Problem& p, Op op, const float* in, const void* 
                                                   (KW - 1) - p.pl);
 }
 
-template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS>
+template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB>
 dw_status_t launch_rem(const Problem& p, const float* in, const void* w, const float* b,
                        float* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
                        int pl_eff) {
     const int rem = ((-pl_eff) % 4 + 4) % 4;
     switch (rem) {
-        case 0: return launch<Cfg<KH, KW, 1, REV, 0, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        case 1: return launch<Cfg<KH, KW, 1, REV, 1, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        case 2: return launch<Cfg<KH, KW, 1, REV, 2, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        default: return launch<Cfg<KH, KW, 1, REV, 3, THT, WX, WY, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 0: return launch<Cfg<KH, KW, 1, REV, 0, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 1: return launch<Cfg<KH, KW, 1, REV, 1, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        case 2: return launch<Cfg<KH, KW, 1, REV, 2, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
+        default: return launch<Cfg<KH, KW, 1, REV, 3, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
     }
 }
 
-template <int KH, int KW, int THT, int WX, int WY, int NS>
+template <int KH, int KW, int THT, int WX, int WY, int NS, int MINB = 1>
 dw_status_t launch_op(const Problem& p, Op op, const float* in, const void* w, const float* b,
                       float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     if (op == OP_FWD)
-        return launch_rem<KH, KW, false, THT, WX, WY, NS>(p, in, w, b, out, stream, err, dry_run,
+        return launch_rem<KH, KW, false, THT, WX, WY, NS, MINB>(p, in, w, b, out, stream, err, dry_run,
                                                           p.pt, p.pl);
-    return launch_rem<KH, KW, true, THT, WX, WY, NS>(p, in, w, b, out, stream, err, dry_run,
+    return launch_rem<KH, KW, true, THT, WX, WY, NS, MINB>(p, in, w, b, out, stream, err, dry_run,
                                                      (KH - 1) - p.pt, (KW - 1) - p.pl);
 }
 
