@@ -1,4 +1,5 @@
-"""Float64 CPU oracle for depthwise 2-D convolution (forward and input gradient).
+"""Float64 CPU oracle for depthwise 2-D convolution (forward, input gradient,
+weight and bias gradients).
 
 TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and the CPU
 (reference / cpu_baseline) legs of ``bench.py`` may import this package; the
@@ -8,8 +9,10 @@ arrays through ctypes.  Nothing here is shared with the CUDA library.
 
 Source of every definition: page "LeanMlir Proofs/Architectures/Depthwise"
 (lean.brettkoonce.com), sections "Depthwise conv2d forward", "Closed-form
-input gradient ... direct formula", "Depthwise conv input-VJP", "Stride-2
-SAME depthwise conv" and "Stride-2 XLA-SAME depthwise conv".  Readings where
+input gradient ... direct formula", "Depthwise conv input-VJP", "Depthwise
+weight-VJP", "Depthwise bias gradient - closed-form formula", "Stride-2 SAME
+depthwise conv" and "Stride-2 XLA-SAME depthwise conv" with their VJP
+sections.  Readings where
 the page leaves a step open (SAME at stride > 1, bias dtype, batch axis,
 layouts) are documented in ``dw_oracle.c``.
 
@@ -70,6 +73,8 @@ def _load():
     lib.dwo_bwd_input.argtypes = [p_i64, p_f64, p_f64, p_f64]
     lib.dwo_fwd_at.restype = None
     lib.dwo_fwd_at.argtypes = [p_i64, p_f64, p_f64, p_f64, i64, p_i64, p_f64]
+    lib.dwo_bwd_weight.restype = None
+    lib.dwo_bwd_weight.argtypes = [p_i64, p_f64, p_f64, p_f64, p_f64]
     lib.dwo_bwd_input_at.restype = None
     lib.dwo_bwd_input_at.argtypes = [p_i64, p_f64, p_f64, i64, p_i64, p_f64]
     _lib = lib
@@ -208,3 +213,15 @@ def bwd_input_at(prob, dy, w, flat_idx):
     _load().dwo_bwd_input_at(_ptr(prob, ctypes.c_int64), _ptr(dy), _ptr(w),
                              idx.shape[0], _ptr(idx, ctypes.c_int64), _ptr(out))
     return out
+
+
+def bwd_weight(prob, x, dy):
+    """(dW [C,kH,kW], db [C]): weight and bias gradients of the forward (float64)."""
+    prob = np.ascontiguousarray(prob, dtype=np.int64)
+    x = _f64(x).reshape(in_shape(prob))
+    dy = _f64(dy).reshape(out_shape(prob))
+    C, kH, kW = int(prob[3]), int(prob[4]), int(prob[5])
+    dw = np.empty((C, kH, kW), dtype=np.float64)
+    db = np.empty(C, dtype=np.float64)
+    _load().dwo_bwd_weight(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(dy), _ptr(dw), _ptr(db))
+    return dw, db

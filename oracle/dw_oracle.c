@@ -25,6 +25,12 @@
  *     evaluates the section's closed-form "direct formula", a sum over output
  *     positions (ho,wo) with the kernel offset reconstructed from
  *     hi + pt = ho*sh + kh*dh.
+ *   - weight and bias gradients, sections "Depthwise weight-VJP" and "Depthwise
+ *     bias gradient - closed-form formula": the forward is affine in W and in b,
+ *     so dW[c,kh,kw] = sum_{n,ho,wo} dy[n,ho,wo,c] * X(n, ho*sh + kh*dh - pt,
+ *     wo*sw + kw*dw - pl, c) (the x_pad term that multiplies W[c,kh,kw]) and
+ *     db[c] = sum_{n,ho,wo} dy[n,ho,wo,c]; the strided and XLA-SAME variants
+ *     are the same sums with the strided index map (dwo_bwd_weight()).
  *   - stride-2 "SAME" and "XLA-SAME" (sections "Stride-2 SAME depthwise conv"
  *     and "Stride-2 XLA-SAME depthwise conv") fix which input rows a strided
  *     output reads; dwo_same_pads() implements the XLA rule
@@ -219,5 +225,40 @@ void dwo_bwd_input_at(const int64_t* p, const double* dy, const double* wt,
             }
         }
         out[i] = acc;
+    }
+}
+
+/* Weight and bias gradients: for each channel, the sum over every output
+ * position of dy times the input value each tap read there (0 where the tap
+ * read padding), and the plain sum of dy.  db may be NULL. */
+void dwo_bwd_weight(const int64_t* p, const double* x, const double* dy, double* dw,
+                    double* db) {
+    int64_t N = p[P_N], C = p[P_C], H = p[P_H], W = p[P_W];
+    int64_t kH = p[P_KH], kW = p[P_KW];
+    int64_t Ho = out_h(p), Wo = out_w(p);
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        for (int64_t kh = 0; kh < kH; ++kh)
+            for (int64_t kw = 0; kw < kW; ++kw) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n)
+                    for (int64_t ho = 0; ho < Ho; ++ho)
+                        for (int64_t wo = 0; wo < Wo; ++wo) {
+                            int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];
+                            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];
+                            if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;
+                            acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *
+                                   x[act_index(p, n, c, hi, wi, H, W)];
+                        }
+                dw[(c * kH + kh) * kW + kw] = acc;
+            }
+        if (db) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                for (int64_t ho = 0; ho < Ho; ++ho)
+                    for (int64_t wo = 0; wo < Wo; ++wo)
+                        acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)];
+            db[c] = acc;
+        }
     }
 }

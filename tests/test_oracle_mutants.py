@@ -38,6 +38,9 @@ MUTANTS = {
     "same_odd_half_on_top": ("*lo = total / 2;\n    *hi = total - *lo;", "*hi = total / 2;\n    *lo = total - *hi;"),
     "extent_off_by_one": ("return last_reach / s + 1;", "return last_reach / s;"),
     "bwd_at_no_divisibility": ("if (kh_nat % dh != 0) continue;", ""),
+    "wgrad_pad_sign": ("int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];\n                            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n                            if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;\n                            acc +=",
+                       "int64_t hi = ho * p[P_SH] + kh * p[P_DH] + p[P_PT];\n                            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n                            if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;\n                            acc +="),
+    "wgrad_transposed_taps": ("dw[(c * kH + kh) * kW + kw] = acc;", "dw[(c * kW + kw) * kH + kh] = acc;"),
     "bwd_at_channel_mix": ("acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *\n                       wt[(c * kH + kh) * kW + kw];",
                            "acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *\n                       wt[(((c + 1) % p[P_C]) * kH + kh) * kW + kw];"),
 }
@@ -70,6 +73,8 @@ def run_pin_subset():
         ("torch_bwd", lambda: pins.test_bwd_equals_torch_autograd(None)),
         ("adjoint", lambda: pins.test_adjoint_identity(None)),
         ("sampled", lambda: pins.test_sampled_evaluators_match_full(None)),
+        ("golden_wgrad", lambda: pins.test_golden_weight_gradient(None)),
+        ("wgrad_linearity", lambda: pins.test_weight_gradient_linearity_identity(None)),
     ]
     for name, fn in checks:
         try:

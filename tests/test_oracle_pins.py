@@ -466,3 +466,60 @@ def test_bias_absent_is_zero(oracle_mod):
     x = rng.standard_normal((1, 5, 5, 3))
     w = rng.standard_normal((3, 3, 3))
     np.testing.assert_array_equal(oracle.fwd(p, x, w, None), oracle.fwd(p, x, w, np.zeros(3)))
+
+
+# ------------------------------------------------ weight / bias gradients --
+
+def test_golden_weight_gradient(oracle_mod):
+    g = load_golden("orientation_2x2.json")
+    p = prob1(g["H"], g["W"], 1, g["kH"], g["kW"], g["stride"], g["dilation"], g["pads"])
+    dw, db = oracle.bwd_weight(p, chw_to("nhwc", [g["x"]]), chw_to("nhwc", [g["bwd_weight"]["dy"]]))
+    assert np.array_equal(dw[0], np.array(g["bwd_weight"]["dw"]))
+    assert db[0] == g["bwd_weight"]["db"]
+    g = load_golden("stride2_4x4.json")
+    for layout in ("nhwc", "nchw"):
+        for key in ("even", "xla_same"):
+            case = g[key]
+            p = prob1(4, 4, 1, 3, 3, case["stride"], 1, case["pads"], layout=layout)
+            dw, db = oracle.bwd_weight(p, chw_to(layout, [g["x"]]), chw_to(layout, [case["dy"]]))
+            assert np.array_equal(dw[0], np.array(case["dw"])), (layout, key)
+            assert db[0] == case["db"]
+
+
+def test_weight_gradient_equals_torch_autograd(oracle_mod):
+    for p, layout, rng in valid_cases(141, 50):
+        N, H, W, C, kH, kW, sh, sw, dh, dw_, pt, pb, pl, pr, _ = (int(v) for v in p)
+        x = rng.standard_normal(oracle.in_shape(p))
+        dy = rng.standard_normal(oracle.out_shape(p))
+        wt = torch.from_numpy(rng.standard_normal((C, 1, kH, kW))).requires_grad_(True)
+        bt = torch.from_numpy(rng.standard_normal(C)).requires_grad_(True)
+        xn = torch.from_numpy(np.ascontiguousarray(to_nchw(p, x)))
+        y = F.conv2d(F.pad(xn, (pl, pr, pt, pb)), wt, bt, (sh, sw), 0, (dh, dw_), groups=C)
+        gw, gb = torch.autograd.grad(y, (wt, bt), torch.from_numpy(np.ascontiguousarray(to_nchw(p, dy))))
+        dw, db = oracle.bwd_weight(p, x, dy)
+        np.testing.assert_allclose(dw, gw.numpy()[:, 0], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(db, gb.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_weight_gradient_linearity_identity(oracle_mod):
+    """The forward is linear in (W, b) for fixed x, so
+    <dW, V> + <db, u> = <dy, fwd(x; V, u)> for any V, u."""
+    for p, layout, rng in valid_cases(151, 60, max_hw=12, max_k=5, max_c=4):
+        C, kH, kW = int(p[3]), int(p[4]), int(p[5])
+        x = rng.standard_normal(oracle.in_shape(p))
+        dy = rng.standard_normal(oracle.out_shape(p))
+        V = rng.standard_normal((C, kH, kW))
+        u = rng.standard_normal(C)
+        dw, db = oracle.bwd_weight(p, x, dy)
+        lhs = float(np.sum(dw * V) + np.sum(db * u))
+        rhs = float(np.sum(dy * oracle.fwd(p, x, V, u)))
+        assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(rhs)), (lhs, rhs)
+
+
+def test_bias_gradient_closed_form(oracle_mod):
+    """db[c] = sum over n, h, w of dy[c] (the page's closed form)."""
+    for p, layout, rng in valid_cases(161, 30):
+        dy = rng.standard_normal(oracle.out_shape(p))
+        _, db = oracle.bwd_weight(p, rng.standard_normal(oracle.in_shape(p)), dy)
+        axes = (0, 1, 2) if layout == "nhwc" else (0, 2, 3)
+        np.testing.assert_allclose(db, dy.sum(axis=axes), rtol=1e-13, atol=1e-13)
