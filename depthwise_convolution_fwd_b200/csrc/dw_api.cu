@@ -246,8 +246,67 @@ dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy, const voi
                false, nullptr);
 }
 
+dw_status_t dwconv2d_bwd_weight_workspace_size(const dw_desc_t* desc, uint64_t* bytes) {
+    Problem p;
+    const dw_status_t st = resolve(desc, &p);
+    if (st != DW_OK) return st;
+    if (!bytes) return DW_ERR_INVALID_ARG;
+    *bytes = bwd_weight_workspace_bytes(p);
+    return DW_OK;
+}
+
+static dw_status_t run_bwd_weight(const dw_desc_t* desc, const float* x, const float* dy,
+                                  float* dw, float* db, void* ws, uint64_t ws_bytes,
+                                  cudaStream_t stream, bool dry_run, int32_t* chosen) {
+    Problem p;
+    dw_status_t st = resolve(desc, &p);
+    if (st != DW_OK) return st;
+    if (!x || !dy || !dw || !ws) return DW_ERR_INVALID_ARG;
+    if (ws_bytes < bwd_weight_workspace_bytes(p)) return DW_ERR_INVALID_ARG;
+    const size_t xb = size_t(p.N) * size_t(p.C) * size_t(p.H) * size_t(p.W) * 4;
+    const size_t gb = size_t(p.N) * size_t(p.C) * size_t(p.Ho) * size_t(p.Wo) * 4;
+    const size_t wb = size_t(p.C) * size_t(p.kH) * size_t(p.kW) * 4;
+    const size_t bb = size_t(p.C) * 4;
+    const void* ins[2] = {x, dy};
+    const size_t inb[2] = {xb, gb};
+    void* outs[3] = {dw, db, ws};
+    const size_t outb[3] = {wb, bb, size_t(ws_bytes)};
+    for (int o = 0; o < 3; ++o) {
+        for (int i = 0; i < 2; ++i)
+            if (overlaps(outs[o], outb[o], ins[i], inb[i])) return DW_ERR_ALIAS;
+        for (int o2 = o + 1; o2 < 3; ++o2)
+            if (overlaps(outs[o], outb[o], outs[o2], outb[o2])) return DW_ERR_ALIAS;
+    }
+    int32_t* err = nullptr;
+    if (!dry_run) {
+        err = device_error_ptr(current_device());
+        if (!err) return DW_ERR_CUDA;
+    }
+    return bwd_weight_launch(p, desc->algo, x, dy, dw, db, ws, stream, err, dry_run, chosen);
+}
+
+dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const float* x, const float* dy, float* dw,
+                                float* db, void* workspace, uint64_t workspace_bytes,
+                                void* stream) {
+    return run_bwd_weight(desc, x, dy, dw, db, workspace, workspace_bytes,
+                          static_cast<cudaStream_t>(stream), false, nullptr);
+}
+
 int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void* in, const void* w,
                             const void* out) {
+    if (op == 2) {
+        int32_t chosen = 0;
+        Problem p;
+        dw_status_t st = resolve(desc, &p);
+        if (st != DW_OK) return -st;
+        const uint64_t need = bwd_weight_workspace_bytes(p);
+        // a workspace address far from the tensors, only used for the checks
+        st = run_bwd_weight(desc, static_cast<const float*>(in), static_cast<const float*>(w),
+                            static_cast<float*>(const_cast<void*>(out)), nullptr,
+                            reinterpret_cast<void*>(uintptr_t(1) << 62), need, nullptr, true,
+                            &chosen);
+        return st == DW_OK ? chosen : -st;
+    }
     if (op != OP_FWD && op != OP_BWD_INPUT) return -DW_ERR_INVALID_ARG;
     int32_t chosen = 0;
     const dw_status_t st =

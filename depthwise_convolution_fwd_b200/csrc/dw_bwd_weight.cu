@@ -1,0 +1,546 @@
+// Weight and bias gradients (page "LeanMlir Proofs/Architectures/Depthwise",
+// sections "Depthwise weight-VJP", "Depthwise bias gradient - closed-form
+// formula" and the stride-2 / XLA-SAME weight and bias VJP sections):
+//
+//   dW[c,kh,kw] = sum_{n,ho,wo} dy[n,ho,wo,c] * X(n, ho*sh + kh*dh - pt,
+//                                                 wo*sw + kw*dw - pl, c)
+//   db[c]       = sum_{n,ho,wo} dy[n,ho,wo,c]
+//
+// A per-channel reduction over every output position, done in two levels
+// with a deterministic order (no atomics):
+//   1. partial kernels write one float64 partial per (block of work, tap,
+//      channel) into the caller's workspace.  Inside a thread, products are
+//      summed in float32 over at most a handful of outputs and then folded
+//      into float64, so the result is accurate to well below float32
+//      rounding of the final value.
+//   2. a finalize kernel sums each channel's partials in a fixed order and
+//      writes dW / db as float32.
+// The tiled partial kernel (NHWC, TMA) loads, per tile, the input halo box
+// and the matching dy box into one pipeline stage; lane = channel (a warp
+// covers the 32 channels of a pixel), each thread owns THT x TWT outputs and
+// streams its input window once, feeding every (output, tap) pair at
+// compile-time offsets.  The direct partial kernels cover every other shape.
+#include <climits>
+
+#include "dw_common.cuh"
+
+namespace dw {
+namespace wgrad {
+
+constexpr int kLanes = 32;          // channels per tiled work block
+constexpr int kMaxTiledCtas = 1024; // cap on the tiled grid (sizes the workspace)
+constexpr int kMaxChunks = 128;     // direct kernels: position chunks per (tap, channel)
+constexpr int64_t kMinChunk = 256;  // direct kernels: positions per chunk at least
+constexpr int kFold = 16;           // direct kernels: float32 terms per float64 fold
+
+// ----------------------------------------------------------- direct kernels --
+
+struct DArgs {
+    int64_t N, C, H, W, Ho, Wo;
+    int kH, kW, sh, sw, dh, dw, pt, pl;
+    int T;           // taps + 1 (the last slot is the bias)
+    int64_t P;       // output positions per channel = N*Ho*Wo
+    int64_t chunk;   // positions per chunk
+    int64_t chunks;  // number of chunks
+    int64_t items;   // chunks * T * C
+};
+
+// NHWC: one thread per (chunk, tap, channel), channel fastest, so a warp reads
+// 32 consecutive channels of one pixel.
+__global__ void __launch_bounds__(256) partial_direct_nhwc(const float* __restrict__ x,
+                                                           const float* __restrict__ dy,
+                                                           double* __restrict__ part, DArgs a) {
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.items; i += stride) {
+        const int64_t c = i % a.C;
+        const int64_t r = i / a.C;
+        const int t = int(r % a.T);
+        const int64_t j = r / a.T;
+        const bool bias = t == a.T - 1;
+        const int kh = bias ? 0 : t / a.kW, kw = bias ? 0 : t % a.kW;
+        const int64_t p0 = j * a.chunk;
+        const int64_t p1 = p0 + a.chunk < a.P ? p0 + a.chunk : a.P;
+        int64_t wo = p0 % a.Wo, q = p0 / a.Wo;
+        int64_t ho = q % a.Ho, n = q / a.Ho;
+        double acc = 0.0;
+        float part32 = 0.f;
+        int cnt = 0;
+        for (int64_t pp = p0; pp < p1; ++pp) {
+            const float g = __ldg(dy + ((n * a.Ho + ho) * a.Wo + wo) * a.C + c);
+            if (bias) {
+                part32 += g;
+            } else {
+                const int64_t hi = ho * a.sh + int64_t(kh) * a.dh - a.pt;
+                const int64_t wi = wo * a.sw + int64_t(kw) * a.dw - a.pl;
+                if (hi >= 0 && hi < a.H && wi >= 0 && wi < a.W)
+                    part32 = fmaf(g, __ldg(x + ((n * a.H + hi) * a.W + wi) * a.C + c), part32);
+            }
+            if (++cnt == kFold) {
+                acc += double(part32);
+                part32 = 0.f;
+                cnt = 0;
+            }
+            if (++wo == a.Wo) {
+                wo = 0;
+                if (++ho == a.Ho) {
+                    ho = 0;
+                    ++n;
+                }
+            }
+        }
+        part[i] = acc + double(part32);
+    }
+}
+
+// NCHW: one warp per (chunk, tap, channel); lanes walk consecutive output
+// positions (W innermost), then the warp sums its lanes.
+__global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restrict__ x,
+                                                           const float* __restrict__ dy,
+                                                           double* __restrict__ part, DArgs a) {
+    grid_dependency_wait();
+    allow_dependents();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < a.items;
+         i += warps) {
+        const int64_t c = i % a.C;
+        const int64_t r = i / a.C;
+        const int t = int(r % a.T);
+        const int64_t j = r / a.T;
+        const bool bias = t == a.T - 1;
+        const int kh = bias ? 0 : t / a.kW, kw = bias ? 0 : t % a.kW;
+        const int64_t p0 = j * a.chunk;
+        const int64_t p1 = p0 + a.chunk < a.P ? p0 + a.chunk : a.P;
+        double acc = 0.0;
+        float part32 = 0.f;
+        int cnt = 0;
+        for (int64_t pp = p0 + lane; pp < p1; pp += 32) {
+            const int64_t wo = pp % a.Wo, q = pp / a.Wo;
+            const int64_t ho = q % a.Ho, n = q / a.Ho;
+            const float g = __ldg(dy + ((n * a.C + c) * a.Ho + ho) * a.Wo + wo);
+            if (bias) {
+                part32 += g;
+            } else {
+                const int64_t hi = ho * a.sh + int64_t(kh) * a.dh - a.pt;
+                const int64_t wi = wo * a.sw + int64_t(kw) * a.dw - a.pl;
+                if (hi >= 0 && hi < a.H && wi >= 0 && wi < a.W)
+                    part32 = fmaf(g, __ldg(x + ((n * a.C + c) * a.H + hi) * a.W + wi), part32);
+            }
+            if (++cnt == kFold) {
+                acc += double(part32);
+                part32 = 0.f;
+                cnt = 0;
+            }
+        }
+        acc += double(part32);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) part[i] = acc;
+    }
+}
+
+// part[(j*T + t)*C + c] summed over j in order.
+__global__ void __launch_bounds__(256) finalize_direct(const double* __restrict__ part,
+                                                       float* __restrict__ dw,
+                                                       float* __restrict__ db, int64_t C, int T,
+                                                       int64_t chunks) {
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t n = C * T;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t c = i % C;
+        const int t = int(i / C);
+        double s = 0.0;
+        for (int64_t j = 0; j < chunks; ++j) s += part[(j * T + t) * C + c];
+        if (t == T - 1) {
+            if (db) db[c] = float(s);
+        } else {
+            dw[c * (T - 1) + t] = float(s);
+        }
+    }
+}
+
+// ------------------------------------------------------------ tiled kernel --
+
+struct TArgs {
+    double* part;
+    int32_t* err;
+    int C;
+    int pt, pl;
+    FastDiv tiles_c, tiles_x, tiles_y;
+    int ntiles;
+};
+
+template <int KH_, int KW_, int S_, int D_, int THT_, int TWT_, int WX_, int WY_, int NS_>
+struct WCfg {
+    static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
+    static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
+    static constexpr int T = KH * KW + 1;
+    static constexpr int NCW = WX * WY;  // consumer warps (one 32-channel pixel row each)
+    static constexpr int NCT = NCW * 32;
+    static constexpr int NT = NCT + 32;  // + producer warp
+    static constexpr int TH = THT * WY, TW = TWT * WX;
+    static constexpr int IH = (TH - 1) * S + (KH - 1) * D + 1;
+    static constexpr int IW = (TW - 1) * S + (KW - 1) * D + 1;
+    static constexpr int RH = (THT - 1) * S + (KH - 1) * D + 1;
+    static constexpr int RW = (TWT - 1) * S + (KW - 1) * D + 1;
+    static constexpr int XBYTES = IH * IW * kLanes * 4;
+    static constexpr int GBYTES = TH * TW * kLanes * 4;
+    static constexpr int STAGE_BYTES = XBYTES + GBYTES;
+    static constexpr int RED_BYTES = NCW * T * kLanes * 8;
+    static constexpr int AREA = NS * STAGE_BYTES > RED_BYTES ? NS * STAGE_BYTES : RED_BYTES;
+    static constexpr size_t SMEM = size_t(AREA) + size_t(2 * NS) * 8 + 16;
+    static_assert(XBYTES % 128 == 0 && GBYTES % 128 == 0, "TMA shared-memory alignment");
+    static_assert(IH <= 256 && IW <= 256 && TW <= 256 && TH <= 256, "TMA box limit");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <class K>
+__host__ __device__ constexpr int tap_of(int r, int j) {  // tap reading window cell r for output j
+    const int num = r - j * K::S;
+    if (num < 0 || num % K::D != 0) return -1;
+    return num / K::D;
+}
+
+struct WTile {
+    int cb, n, oy0, ox0, iy0, ix0;
+};
+
+template <class K>
+__device__ __forceinline__ WTile decode(int t, const TArgs& a) {
+    WTile T;
+    const int q = fast_div(t, a.tiles_c);
+    T.cb = t - q * a.tiles_c.d;
+    const int r = fast_div(q, a.tiles_x);
+    const int tx = q - r * a.tiles_x.d;
+    T.n = fast_div(r, a.tiles_y);
+    const int ty = r - T.n * a.tiles_y.d;
+    T.oy0 = ty * K::TH;
+    T.ox0 = tx * K::TW;
+    T.iy0 = T.oy0 * K::S - a.pt;
+    T.ix0 = T.ox0 * K::S - a.pl;
+    return T;
+}
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    partial_tiled(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap gmap,
+                  const TArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + K::AREA);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    allow_dependents();
+
+    if (warp == K::NCW) {
+        if (lane == 0) {
+            prefetch_tensor_map(&xmap);
+            prefetch_tensor_map(&gmap);
+            int k = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
+                const int s = k % K::NS;
+                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const WTile T = decode<K>(t, a);
+                unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+                tma_load_4d(st, &xmap, &full[s], T.cb * kLanes, T.ix0, T.iy0, T.n);
+                tma_load_4d(st + K::XBYTES, &gmap, &full[s], T.cb * kLanes, T.ox0, T.oy0, T.n);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
+        }
+        return;
+    }
+
+    const int xi = warp % K::WX, yi = warp / K::WX;
+    const int j0 = yi * K::THT, i0 = xi * K::TWT;
+    double acc64[K::T];
+#pragma unroll
+    for (int t = 0; t < K::T; ++t) acc64[t] = 0.0;
+
+    int k = 0;
+    for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
+        const int s = k % K::NS;
+        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+            }
+            break;
+        }
+        const float* xb = reinterpret_cast<const float*>(smem + size_t(s) * K::STAGE_BYTES);
+        const float* gb = xb + K::XBYTES / 4;
+        float g[K::THT][K::TWT];
+#pragma unroll
+        for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+            for (int i = 0; i < K::TWT; ++i) g[j][i] = gb[((j0 + j) * K::TW + i0 + i) * kLanes + lane];
+        float acc[K::KH][K::KW];
+#pragma unroll
+        for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+            for (int kw = 0; kw < K::KW; ++kw) acc[kh][kw] = 0.f;
+        const float* win = xb + ((j0 * K::S) * K::IW + i0 * K::S) * kLanes + lane;
+        static_for<0, K::RH>([&](auto r_) {
+            constexpr int r = decltype(r_)::value;
+            static_for<0, K::RW>([&](auto q_) {
+                constexpr int q = decltype(q_)::value;
+                const float v = win[(r * K::IW + q) * kLanes];
+                static_for<0, K::THT>([&](auto j_) {
+                    constexpr int j = decltype(j_)::value;
+                    constexpr int kh = tap_of<K>(r, j);
+                    if constexpr (kh >= 0 && kh < K::KH) {
+                        static_for<0, K::TWT>([&](auto i_) {
+                            constexpr int i = decltype(i_)::value;
+                            constexpr int kw = tap_of<K>(q, i);
+                            if constexpr (kw >= 0 && kw < K::KW)
+                                acc[kh][kw] = fmaf(g[j][i], v, acc[kh][kw]);
+                        });
+                    }
+                });
+            });
+        });
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        float gs = 0.f;
+#pragma unroll
+        for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+            for (int i = 0; i < K::TWT; ++i) gs += g[j][i];
+#pragma unroll
+        for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+            for (int kw = 0; kw < K::KW; ++kw) acc64[kh * K::KW + kw] += double(acc[kh][kw]);
+        acc64[K::T - 1] += double(gs);
+    }
+
+    // every consumer is past its last tile (no copy in flight any more): sum
+    // the warps' float64 partials through shared memory, in warp order
+    named_barrier_sync(1, K::NCT);
+    double* red = reinterpret_cast<double*>(smem);
+#pragma unroll
+    for (int t = 0; t < K::T; ++t) red[(warp * K::T + t) * kLanes + lane] = acc64[t];
+    named_barrier_sync(1, K::NCT);
+    for (int t = warp; t < K::T; t += K::NCW) {
+        double sum = 0.0;
+        for (int w = 0; w < K::NCW; ++w) sum += red[(w * K::T + t) * kLanes + lane];
+        a.part[(int64_t(blockIdx.x) * K::T + t) * kLanes + lane] = sum;
+    }
+}
+
+// part[(b*T + t)*32 + lane], b = cb, cb + tiles_c, ... < G, summed in order.
+__global__ void __launch_bounds__(256) finalize_tiled(const double* __restrict__ part,
+                                                      float* __restrict__ dw,
+                                                      float* __restrict__ db, int C, int T,
+                                                      int tiles_c, int G) {
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t n = int64_t(C) * T;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int c = int(i % C);
+        const int t = int(i / C);
+        const int cb = c / kLanes, lane = c % kLanes;
+        double s = 0.0;
+        for (int b = cb; b < G; b += tiles_c) s += part[(int64_t(b) * T + t) * kLanes + lane];
+        if (t == T - 1) {
+            if (db) db[c] = float(s);
+        } else {
+            dw[int64_t(c) * (T - 1) + t] = float(s);
+        }
+    }
+}
+
+// ------------------------------------------------------------------- host --
+
+int64_t direct_chunks(const Problem& p, int64_t& chunk) {
+    const int64_t P = p.N * p.Ho * p.Wo;
+    int64_t chunks = (P + kMinChunk - 1) / kMinChunk;
+    if (chunks > kMaxChunks) chunks = kMaxChunks;
+    if (chunks < 1) chunks = 1;
+    chunk = (P + chunks - 1) / chunks;
+    chunks = (P + chunk - 1) / chunk;
+    return chunks;
+}
+
+size_t direct_workspace(const Problem& p) {
+    int64_t chunk;
+    const int64_t chunks = direct_chunks(p, chunk);
+    return size_t(chunks) * size_t(p.kH * p.kW + 1) * size_t(p.C) * sizeof(double);
+}
+
+size_t tiled_workspace(const Problem& p) {
+    const int64_t tc = (p.C + kLanes - 1) / kLanes;
+    const int64_t g = tc >= kMaxTiledCtas ? tc : (kMaxTiledCtas / tc) * tc;
+    return size_t(g) * size_t(p.kH * p.kW + 1) * kLanes * sizeof(double);
+}
+
+dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, float* dw, float* db,
+                          void* ws, cudaStream_t stream) {
+    DArgs a;
+    a.N = p.N; a.C = p.C; a.H = p.H; a.W = p.W; a.Ho = p.Ho; a.Wo = p.Wo;
+    a.kH = p.kH; a.kW = p.kW; a.sh = p.sh; a.sw = p.sw; a.dh = p.dh; a.dw = p.dw;
+    a.pt = p.pt; a.pl = p.pl;
+    a.T = p.kH * p.kW + 1;
+    a.P = p.N * p.Ho * p.Wo;
+    a.chunks = direct_chunks(p, a.chunk);
+    a.items = a.chunks * a.T * p.C;
+    double* part = static_cast<double*>(ws);
+    const int dev = current_device();
+    const int64_t cap = int64_t(sm_count(dev)) * 8;
+    const int64_t threads_needed = p.layout == DW_NHWC ? a.items : a.items * 32;
+    int64_t blocks = (threads_needed + 255) / 256;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    cudaError_t e = p.layout == DW_NHWC
+                        ? launch_pdl(partial_direct_nhwc, dim3(unsigned(blocks)), dim3(256), 0,
+                                     stream, x, dy, part, a)
+                        : launch_pdl(partial_direct_nchw, dim3(unsigned(blocks)), dim3(256), 0,
+                                     stream, x, dy, part, a);
+    if (e != cudaSuccess) return DW_ERR_CUDA;
+    int64_t fb = (p.C * a.T + 255) / 256;
+    if (fb > cap) fb = cap;
+    e = launch_pdl(finalize_direct, dim3(unsigned(fb)), dim3(256), 0, stream,
+                   static_cast<const double*>(part), dw, db, int64_t(p.C), a.T, a.chunks);
+    if (e != cudaSuccess) return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+template <class K>
+dw_status_t launch_tiled(const Problem& p, const float* x, const float* dy, float* dw, float* db,
+                         void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    TArgs a;
+    a.part = static_cast<double*>(ws);
+    a.err = err;
+    a.C = static_cast<int>(p.C);
+    a.pt = p.pt;
+    a.pl = p.pl;
+    const int64_t ty = (p.Ho + K::TH - 1) / K::TH;
+    const int64_t tx = (p.Wo + K::TW - 1) / K::TW;
+    const int64_t tc = (p.C + kLanes - 1) / kLanes;
+    const int64_t spatial = ty * tx * p.N;
+    const int64_t nt = spatial * tc;
+    if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.tiles_y = make_fastdiv(int(ty));
+    a.tiles_x = make_fastdiv(int(tx));
+    a.tiles_c = make_fastdiv(int(tc));
+    a.ntiles = int(nt);
+    if (dry_run) return DW_OK;
+
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&partial_tiled<K>), K::NT,
+                                   K::SMEM, cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+    // every CTA keeps one channel block: the grid is a multiple of tiles_c,
+    // at most kMaxTiledCtas (the bound the workspace size assumes)
+    int64_t reps = (int64_t(sm_count(dev)) * occ) / tc;
+    const int64_t reps_cap = tc >= kMaxTiledCtas ? 1 : kMaxTiledCtas / tc;
+    if (reps > reps_cap) reps = reps_cap;
+    if (reps > spatial) reps = spatial;
+    if (reps < 1) reps = 1;
+    const int64_t G = reps * tc;
+
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap xmap, gmap;
+    const cuuint64_t xd[4] = {cuuint64_t(p.C), cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.N)};
+    const cuuint64_t xs[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * p.W) * 4,
+                              cuuint64_t(p.C * p.W * p.H) * 4};
+    const cuuint32_t xbox[4] = {kLanes, K::IW, K::IH, 1};
+    const cuuint64_t gd[4] = {cuuint64_t(p.C), cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.N)};
+    const cuuint64_t gs[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * p.Wo) * 4,
+                              cuuint64_t(p.C * p.Wo * p.Ho) * 4};
+    const cuuint32_t gbox[4] = {kLanes, K::TW, K::TH, 1};
+    if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
+                          xbox, estr) != CUDA_SUCCESS ||
+        encode_tensor_map(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(dy), gd, gs,
+                          gbox, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+    if (launch_pdl(partial_tiled<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap, gmap,
+                   a) != cudaSuccess)
+        return DW_ERR_CUDA;
+    int64_t fb = (p.C * K::T + 255) / 256;
+    const int64_t cap = int64_t(sm_count(dev)) * 8;
+    if (fb > cap) fb = cap;
+    if (launch_pdl(finalize_tiled, dim3(unsigned(fb)), dim3(256), 0, stream,
+                   static_cast<const double*>(a.part), dw, db, int(p.C), K::T, int(tc),
+                   int(G)) != cudaSuccess)
+        return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+//                         KH KW  S  D THT TWT WX WY NS
+using W33s1 = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4>;
+using W33s2 = WCfg<3, 3, 2, 1, 1, 2, 4, 2, 4>;
+using W55s1 = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3>;
+using W77s1 = WCfg<7, 7, 1, 1, 1, 4, 4, 2, 3>;
+using W1x15 = WCfg<1, 15, 1, 1, 1, 8, 8, 1, 4>;
+using W1x31 = WCfg<1, 31, 1, 1, 1, 8, 8, 1, 4>;
+
+dw_status_t tiled_pick(const Problem& p, const float* x, const float* dy, float* dw, float* db,
+                       void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.layout != DW_NHWC || p.C % 4 != 0) return DW_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
+        return DW_ERR_UNSUPPORTED;
+    if (p.sh != p.sw || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
+    if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.C >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    const int S = p.sh;
+    if (p.kH == 3 && p.kW == 3 && S == 1) return launch_tiled<W33s1>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && S == 2) return launch_tiled<W33s2>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 5 && p.kW == 5 && S == 1) return launch_tiled<W55s1>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 7 && p.kW == 7 && S == 1) return launch_tiled<W77s1>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 1 && p.kW == 15 && S == 1) return launch_tiled<W1x15>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 1 && p.kW == 31 && S == 1) return launch_tiled<W1x31>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
+}  // namespace wgrad
+
+size_t bwd_weight_workspace_bytes(const Problem& p) {
+    const size_t a = wgrad::direct_workspace(p), b = wgrad::tiled_workspace(p);
+    return a > b ? a : b;
+}
+
+dw_status_t bwd_weight_launch(const Problem& p, int algo, const float* x, const float* dy,
+                              float* dw, float* db, void* ws, cudaStream_t stream, int32_t* err,
+                              bool dry_run, int32_t* chosen) {
+    if (algo == DW_ALGO_AUTO || algo == DW_ALGO_TILED) {
+        const dw_status_t t = wgrad::tiled_pick(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (t == DW_OK) {
+            if (chosen) *chosen = DW_ALGO_TILED;
+            return DW_OK;
+        }
+        if (t != DW_ERR_UNSUPPORTED || algo == DW_ALGO_TILED) return t;
+    }
+    if (chosen) *chosen = DW_ALGO_DIRECT;
+    if (dry_run) return DW_OK;
+    return wgrad::launch_direct(p, x, dy, dw, db, ws, stream);
+}
+
+}  // namespace dw

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
 #include <utility>
 
 #include "dwconv2d.h"
@@ -38,7 +39,14 @@ dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const vo
                               const float* b, float* out, cudaStream_t stream,
                               int32_t* dev_err, bool dry_run);
 
-// Host helpers (dw_host.cu).
+// Weight / bias gradient (dw_bwd_weight.cu): workspace bytes the call needs,
+// and the launch (partials into `ws`, then the fixed-order finalize).
+size_t bwd_weight_workspace_bytes(const Problem& p);
+dw_status_t bwd_weight_launch(const Problem& p, int algo, const float* x, const float* dy,
+                              float* dw, float* db, void* ws, cudaStream_t stream,
+                              int32_t* dev_err, bool dry_run, int32_t* chosen);
+
+// Host helpers (dw_api.cu).
 int current_device();
 int sm_count(int dev);
 // cuTensorMapEncodeTiled fetched through the runtime (no link-time libcuda
@@ -246,6 +254,15 @@ __device__ __forceinline__ void grid_dependency_wait() {
 }
 __device__ __forceinline__ void allow_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Compile-time loop: calls f(integral_constant<int, i>) for i in [I, N).
+template <int I, int N, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for<I + 1, N>(f);
+    }
 }
 
 __device__ __forceinline__ void fma4(float4& acc, const float4& v, const float4& w) {

@@ -69,13 +69,6 @@ struct Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-template <int I, int N, class F>
-__device__ __forceinline__ void static_for(F&& f) {
-    if constexpr (I < N) {
-        f(std::integral_constant<int, I>{});
-        static_for<I + 1, N>(f);
-    }
-}
 
 // tile t -> (tx, ty or output row h, plane or channel group, n)
 template <class K>

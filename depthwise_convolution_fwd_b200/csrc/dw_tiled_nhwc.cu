@@ -134,13 +134,6 @@ struct Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-template <int I, int N, class F>
-__device__ __forceinline__ void static_for(F&& f) {
-    if constexpr (I < N) {
-        f(std::integral_constant<int, I>{});
-        static_for<I + 1, N>(f);
-    }
-}
 
 // Tap index that maps output offset j (within a thread block) to window
 // row r, or -1.  Forward: r = j*S + k*D.  Transposed: r - A = (j - k*D)/S

@@ -27,8 +27,9 @@ _ALGOS = {"auto": DW_ALGO_AUTO, "direct": DW_ALGO_DIRECT, "tiled": DW_ALGO_TILED
 
 # Every symbol include/dwconv2d.h declares.
 EXPORTS = ("dwconv2d_out_shape", "dwconv2d_resolved_pads", "dwconv2d_fwd",
-           "dwconv2d_bwd_input", "dwconv2d_query_algo", "dwconv2d_take_device_error",
-           "dwconv2d_status_string", "dwconv2d_version")
+           "dwconv2d_bwd_input", "dwconv2d_bwd_weight", "dwconv2d_bwd_weight_workspace_size",
+           "dwconv2d_query_algo", "dwconv2d_take_device_error", "dwconv2d_status_string",
+           "dwconv2d_version")
 
 
 class DwDesc(ctypes.Structure):
@@ -73,6 +74,10 @@ def lib() -> ctypes.CDLL:
     L.dwconv2d_fwd.argtypes = [P(DwDesc), vp, vp, vp, vp, vp]
     L.dwconv2d_bwd_input.restype = i32
     L.dwconv2d_bwd_input.argtypes = [P(DwDesc), vp, vp, vp, vp]
+    L.dwconv2d_bwd_weight.restype = i32
+    L.dwconv2d_bwd_weight.argtypes = [P(DwDesc), vp, vp, vp, vp, vp, ctypes.c_uint64, vp]
+    L.dwconv2d_bwd_weight_workspace_size.restype = i32
+    L.dwconv2d_bwd_weight_workspace_size.argtypes = [P(DwDesc), P(ctypes.c_uint64)]
     L.dwconv2d_query_algo.restype = i32
     L.dwconv2d_query_algo.argtypes = [P(DwDesc), i32, vp, vp, vp]
     L.dwconv2d_take_device_error.restype = i32
@@ -169,6 +174,21 @@ def bwd_input_raw(desc: DwDesc, dy_ptr: int, w_ptr: int, dx_ptr: int, stream: in
     """dwconv2d_bwd_input on raw device pointers; returns the status."""
     return int(lib().dwconv2d_bwd_input(ctypes.byref(desc), dy_ptr, w_ptr, dx_ptr,
                                         stream or None))
+
+
+def bwd_weight_raw(desc: DwDesc, x_ptr: int, dy_ptr: int, dw_ptr: int, db_ptr: Optional[int],
+                   ws_ptr: int, ws_bytes: int, stream: int) -> int:
+    """dwconv2d_bwd_weight on raw device pointers; returns the status."""
+    return int(lib().dwconv2d_bwd_weight(ctypes.byref(desc), x_ptr, dy_ptr, dw_ptr, db_ptr or None,
+                                         ws_ptr, int(ws_bytes), stream or None))
+
+
+def dwconv2d_bwd_weight_workspace_size(desc: DwDesc) -> int:
+    n = ctypes.c_uint64()
+    st = lib().dwconv2d_bwd_weight_workspace_size(ctypes.byref(desc), ctypes.byref(n))
+    if st != DW_OK:
+        raise DwError(st, "dwconv2d_bwd_weight_workspace_size")
+    return int(n.value)
 
 
 # ------------------------------------------------------------ tensor calls --
@@ -272,3 +292,47 @@ def dwconv2d_bwd_input(dy: torch.Tensor, w: torch.Tensor, input_hw: Tuple[int, i
     if st != DW_OK:
         raise DwError(st, "dwconv2d_bwd_input")
     return out
+
+
+def dwconv2d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel_hw: Tuple[int, int], *,
+                        stride=1, dilation=1, padding="same", layout: str = "nhwc",
+                        algo: str = "auto", bias: bool = True,
+                        dw: Optional[torch.Tensor] = None, db: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None):
+    """(dW [C,kH,kW], db [C] or None): weight and bias gradients of the
+    forward with input x and output cotangent dy.  `workspace` (a CUDA byte
+    tensor of at least dwconv2d_bwd_weight_workspace_size bytes) is allocated
+    when not given."""
+    _check_act(x, "x")
+    _check_act(dy, "dy")
+    if dy.device != x.device:
+        raise ValueError("x and dy must be on the same device")
+    kH, kW = (int(v) for v in kernel_hw)
+    if layout.lower() == "nhwc":
+        N, H, W, C = x.shape
+    else:
+        N, C, H, W = x.shape
+    desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
+                     layout=layout, algo=algo)
+    Ho, Wo = dwconv2d_out_shape(desc)
+    want = (N, Ho, Wo, C) if desc.layout == DW_NHWC else (N, C, Ho, Wo)
+    if tuple(dy.shape) != want:
+        raise ValueError(f"dy must have shape {want}, got {tuple(dy.shape)}")
+    if dw is None:
+        dw = torch.empty((C, kH, kW), device=x.device, dtype=torch.float32)
+    elif dw.dtype != torch.float32 or dw.numel() != C * kH * kW or not dw.is_contiguous():
+        raise ValueError("dw must be a contiguous float32 tensor of C*kH*kW elements")
+    if bias and db is None:
+        db = torch.empty((C,), device=x.device, dtype=torch.float32)
+    need = dwconv2d_bwd_weight_workspace_size(desc)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), device=x.device, dtype=torch.uint8)
+    elif workspace.device != x.device or workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace must hold at least {need} bytes on {x.device}")
+    with torch.cuda.device(x.device):
+        st = bwd_weight_raw(desc, x.data_ptr(), dy.data_ptr(), dw.data_ptr(),
+                            None if db is None else db.data_ptr(), workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream_ptr(x.device))
+    if st != DW_OK:
+        raise DwError(st, "dwconv2d_bwd_weight")
+    return dw, db

@@ -144,10 +144,41 @@ DW_API dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy,
                                const void* w, float* dx, void* stream);
 
 /*
+ * Weight and bias gradients of the forward of `desc`:
+ *   dW[c,kh,kw] = sum_{n,ho,wo} dy[n,ho,wo,c] * X(n, ho*sh + kh*dh - pt,
+ *                                                 wo*sw + kw*dw - pl, c)
+ *   db[c]       = sum_{n,ho,wo} dy[n,ho,wo,c]
+ *   x:  [N,H,W,C] or [N,C,H,W] float32, read only.
+ *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] float32, read only.
+ *   dw: [C,kH,kW] float32, every element written (also when desc->wtype is
+ *       DW_F16: gradients are produced in float32).
+ *   db: [C] float32 or NULL (then the bias gradient is not produced).
+ *   workspace: device memory of at least dwconv2d_bwd_weight_workspace_size()
+ *       bytes, caller-owned; its contents on entry do not matter and are
+ *       overwritten.
+ * The sums are reduced in a fixed order (float32 products over a few
+ * outputs folded into float64, then float64 partials summed in order), so
+ * repeated calls give bit-identical results on the same device.
+ * dw, db and workspace must not overlap x, dy or each other (DW_ERR_ALIAS);
+ * a workspace smaller than required returns DW_ERR_INVALID_ARG.
+ * Page: LeanMlir Depthwise, "Depthwise weight-VJP", "Depthwise bias gradient
+ * - closed-form formula" and the stride-2 / XLA-SAME weight and bias VJP
+ * sections.
+ */
+DW_API dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const float* x, const float* dy,
+                                       float* dw, float* db, void* workspace,
+                                       uint64_t workspace_bytes, void* stream);
+
+/* Workspace bytes dwconv2d_bwd_weight needs for `desc` (host only; depends
+ * on the problem, not on the device or the pointers). */
+DW_API dw_status_t dwconv2d_bwd_weight_workspace_size(const dw_desc_t* desc, uint64_t* bytes);
+
+/*
  * Which kernel family a call with these arguments would run (host only, no
  * launch): returns DW_ALGO_DIRECT or DW_ALGO_TILED, or -DW_ERR_* when the call
  * would fail.  op: 0 = forward (in = x, out = y), 1 = input gradient
- * (in = dy, out = dx).  Pointers are only inspected for alignment.
+ * (in = dy, out = dx), 2 = weight gradient (in = x, w = dy, out = dw).
+ * Pointers are only inspected for alignment.
  */
 DW_API int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void* in,
                             const void* w, const void* out);

@@ -156,3 +156,31 @@ def test_binding_refuses_cpu_tensors(lib):
     w = torch.zeros(4, 3, 3)
     with pytest.raises(TypeError):
         dw.dwconv2d_fwd(x, w)
+
+
+def test_weight_gradient_host_checks(lib):
+    desc = dw.make_desc(2, 16, 16, 32, 3, 3)
+    need = dw.dwconv2d_bwd_weight_workspace_size(desc)
+    assert need > 0
+    # the workspace size depends on the problem only
+    assert need == dw.dwconv2d_bwd_weight_workspace_size(dw.make_desc(2, 16, 16, 32, 3, 3))
+    base = 1 << 40
+    x, dy, dwp, db, ws = base, base + (1 << 24), base + (2 << 24), base + (3 << 24), base + (4 << 24)
+    # too small a workspace, NULL tensors, invalid descriptor: rejected before launch
+    assert dw.bwd_weight_raw(desc, x, dy, dwp, db, ws, need - 1, 0) == dw.DW_ERR_INVALID_ARG
+    assert dw.bwd_weight_raw(desc, 0, dy, dwp, db, ws, need, 0) == dw.DW_ERR_INVALID_ARG
+    assert dw.bwd_weight_raw(desc, x, dy, dwp, db, 0, need, 0) == dw.DW_ERR_INVALID_ARG
+    bad = dw.make_desc(2, 16, 16, 32, 3, 3)
+    bad.C = 0
+    assert dw.bwd_weight_raw(bad, x, dy, dwp, db, ws, need, 0) == dw.DW_ERR_INVALID_ARG
+    # outputs overlapping inputs or each other
+    assert dw.bwd_weight_raw(desc, x, dy, x + 64, db, ws, need, 0) == dw.DW_ERR_ALIAS
+    assert dw.bwd_weight_raw(desc, x, dy, dwp, dy + 4, ws, need, 0) == dw.DW_ERR_ALIAS
+    assert dw.bwd_weight_raw(desc, x, dy, dwp, db, dwp + 8, need, 0) == dw.DW_ERR_ALIAS
+    assert dw.bwd_weight_raw(desc, x, dy, dwp, db, x, need, 0) == dw.DW_ERR_ALIAS
+    # kernel family selection (op 2 = weight gradient; no launch)
+    T, D = dw.DW_ALGO_TILED, dw.DW_ALGO_DIRECT
+    assert dw.dwconv2d_query_algo(desc, 2, x, dy, dwp) == T
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 3, 3, layout="nchw"), 2, x, dy, dwp) == D
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 7, 3, 3), 2, x, dy, dwp) == D
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 3, 3, dilation=2), 2, x, dy, dwp) == D

@@ -1,0 +1,130 @@
+"""GPU parity of the weight and bias gradients against the float64 oracle.
+
+Rule as for the other calls: |gpu - ref| <= 1e-5 * sum|terms| per element,
+the scale being the oracle's gradient of |x| and |dy| (every term
+non-negative), exact where there is no term.  Both kernel families; calls
+repeat bit-identically (fixed reduction order)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import depthwise_convolution_fwd_b200 as dw
+from depthwise_convolution_fwd_b200 import build as dwbuild
+from depthwise_convolution_fwd_b200 import workloads as wl
+from depthwise_convolution_fwd_b200.workloads import Case
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dwbuild.build()
+    dw.lib()
+    yield
+    torch.cuda.synchronize()
+    assert dw.dwconv2d_take_device_error() == 0
+
+
+def reference(case, inp):
+    p = gu.problem(case)
+    x, dy = gu.f64(inp["x"]), gu.f64(inp["dy"])
+    dwr, dbr = oracle.bwd_weight(p, x, dy)
+    dws, dbs = oracle.bwd_weight(p, np.abs(x), np.abs(dy))
+    return dwr, dbr, dws, dbs
+
+
+def gpu(case, inp, algo="auto"):
+    return dw.dwconv2d_bwd_weight(inp["x"].cuda(), inp["dy"].cuda(), (case.kH, case.kW),
+                                  stride=case.stride, dilation=case.dilation,
+                                  padding=case.padding, layout=case.layout, algo=algo)
+
+
+def check(case, algos=("auto", "direct")):
+    inp = gu.inputs(case)
+    dwr, dbr, dws, dbs = reference(case, inp)
+    for algo in algos:
+        g_w, g_b = gpu(case, inp, algo)
+        torch.cuda.synchronize()
+        gu.assert_close(g_w.cpu().numpy(), dwr, dws, f"{case.name} dW [{algo}]")
+        gu.assert_close(g_b.cpu().numpy(), dbr, dbs, f"{case.name} db [{algo}]")
+
+
+CONFIGS = wl.tiny() + wl.mobilenet() + [c for c in wl.conformer() if c.W == 24] + \
+    [c for c in wl.large() if c.H == 30] + [c for c in wl.edge() if c.wtype == "f32"]
+
+
+@pytest.mark.parametrize("case", CONFIGS, ids=lambda c: c.name)
+def test_config_cases(case):
+    check(case)
+
+
+TILED = [
+    Case("w_3x3_s1", 3, 37, 45, 72, 3, 3, seed=71),
+    Case("w_3x3_s1_pad", 2, 23, 70, 36, 3, 3, padding=(0, 2, 2, 1), seed=72),
+    Case("w_3x3_s2", 4, 29, 41, 44, 3, 3, stride=2, padding=1, seed=73),
+    Case("w_3x3_s2_same", 2, 30, 34, 40, 3, 3, stride=2, seed=74),
+    Case("w_5x5", 2, 17, 39, 68, 5, 5, seed=75),
+    Case("w_7x7", 2, 19, 23, 36, 7, 7, seed=76),
+    Case("w_1x15", 4, 2, 300, 44, 1, 15, act="normal", seed=77),
+    Case("w_1x31", 3, 3, 290, 68, 1, 31, act="normal", seed=78),
+    Case("w_many_tiles", 16, 64, 64, 96, 3, 3, seed=79),
+]
+
+
+@pytest.mark.parametrize("case", TILED, ids=lambda c: c.name)
+def test_tiled_weight_gradient(case):
+    inp = gu.inputs(case)
+    x, dy = inp["x"].cuda(), inp["dy"].cuda()
+    dwt = torch.empty(case.C, case.kH, case.kW, device="cuda")
+    assert dw.dwconv2d_query_algo(gu.desc_of(case), 2, x.data_ptr(), dy.data_ptr(),
+                                  dwt.data_ptr()) == dw.DW_ALGO_TILED
+    check(case, algos=("tiled", "direct"))
+
+
+def test_repeatable_bit_for_bit():
+    case = wl.mobilenet()[2]
+    inp = gu.inputs(case)
+    a = gpu(case, inp)
+    b = gpu(case, inp)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_large_full_size():
+    case = [c for c in wl.large() if c.H == 512 and c.layout == "nhwc"][0]
+    check(case, algos=("auto",))
+
+
+def test_random_sweep():
+    rng = np.random.default_rng(303)
+    count = 0
+    while count < 40:
+        layout = "nhwc" if rng.random() < 0.5 else "nchw"
+        k = int(rng.choice([1, 2, 3, 5]))
+        case = Case(f"wsweep{count}", int(rng.integers(1, 4)), int(rng.integers(1, 30)),
+                    int(rng.integers(1, 30)), int(rng.choice([1, 4, 7, 32, 36])), k,
+                    int(rng.choice([1, k])), stride=int(rng.integers(1, 3)),
+                    dilation=int(rng.integers(1, 3)),
+                    padding="same" if rng.random() < 0.5 else int(rng.integers(0, 3)),
+                    layout=layout, seed=7000 + count)
+        ho, wo = gu.out_hw(case)
+        if ho < 1 or wo < 1:
+            continue
+        check(case)
+        count += 1
+
+
+def test_no_bias_gradient_and_small_workspace_error():
+    case = Case("wnob", 2, 12, 12, 32, 3, 3, seed=80)
+    inp = gu.inputs(case)
+    dwr, _, dws, _ = reference(case, inp)
+    g_w, g_b = dw.dwconv2d_bwd_weight(inp["x"].cuda(), inp["dy"].cuda(), (3, 3), bias=False)
+    torch.cuda.synchronize()
+    assert g_b is None
+    gu.assert_close(g_w.cpu().numpy(), dwr, dws, "dW without db")
+    with pytest.raises(ValueError):
+        dw.dwconv2d_bwd_weight(inp["x"].cuda(), inp["dy"].cuda(), (3, 3),
+                               workspace=torch.empty(8, dtype=torch.uint8, device="cuda"))
