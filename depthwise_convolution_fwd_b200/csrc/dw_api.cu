@@ -88,6 +88,24 @@ static int32_t* device_error_ptr(int dev) {
     return p;
 }
 
+// Fixed device scratch of dwconv2d_bwd_weight_noalloc: one array per device
+// that loads the library, held until the process exits.  Host code only ever
+// uses its device address, looked up once per device (with that device
+// current) and cached; the array's name in host code is not that address.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DW_NOALLOC_SCRATCH_BYTES];
+
+static void* noalloc_scratch_ptr(int dev) {
+    static std::atomic<void*> cache[64];
+    if (dev < 0 || dev >= 64) return nullptr;
+    void* p = cache[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr)
+        return nullptr;
+    cache[dev].store(addr, std::memory_order_release);
+    return addr;
+}
+
 // ---------------------------------------------------------------- validation
 
 static int64_t out_extent(int64_t in, int k, int s, int d, int lo, int hi) {
@@ -292,6 +310,18 @@ dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const float* x, const flo
                           static_cast<cudaStream_t>(stream), false, nullptr);
 }
 
+dw_status_t dwconv2d_bwd_weight_noalloc(const dw_desc_t* desc, const float* x, const float* dy,
+                                        float* dw, float* db, void* stream) {
+    Problem p;
+    const dw_status_t st = resolve(desc, &p);
+    if (st != DW_OK) return st;
+    if (bwd_weight_workspace_bytes(p) > DW_NOALLOC_SCRATCH_BYTES) return DW_ERR_TOO_LARGE;
+    void* scratch = noalloc_scratch_ptr(current_device());
+    if (!scratch) return DW_ERR_CUDA;
+    return run_bwd_weight(desc, x, dy, dw, db, scratch, DW_NOALLOC_SCRATCH_BYTES,
+                          static_cast<cudaStream_t>(stream), false, nullptr);
+}
+
 int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void* in, const void* w,
                             const void* out) {
     if (op == 2) {
@@ -338,6 +368,8 @@ const char* dwconv2d_status_string(dw_status_t status) {
         case DW_ERR_ALIAS: return "DW_ERR_ALIAS: output overlaps an input";
         case DW_ERR_CUDA: return "DW_ERR_CUDA: CUDA launch or runtime error";
         case DW_ERR_DEVICE_TIMEOUT: return "DW_ERR_DEVICE_TIMEOUT: a kernel gave up waiting on a copy";
+        case DW_ERR_TOO_LARGE:
+            return "DW_ERR_TOO_LARGE: the problem needs more scratch than the fixed device array holds";
         default: return "unknown dw_status_t";
     }
 }

@@ -16,7 +16,9 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdwconv2d.so")
 _lib = None
 
-DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_ALIAS, DW_ERR_CUDA, DW_ERR_DEVICE_TIMEOUT = range(6)
+(DW_OK, DW_ERR_INVALID_ARG, DW_ERR_UNSUPPORTED, DW_ERR_ALIAS, DW_ERR_CUDA,
+ DW_ERR_DEVICE_TIMEOUT, DW_ERR_TOO_LARGE) = range(7)
+DW_NOALLOC_SCRATCH_BYTES = 16 << 20
 DW_NHWC, DW_NCHW = 0, 1
 DW_F32, DW_F16 = 0, 1
 DW_PAD_EXPLICIT, DW_PAD_SAME = 0, 1
@@ -28,6 +30,7 @@ _ALGOS = {"auto": DW_ALGO_AUTO, "direct": DW_ALGO_DIRECT, "tiled": DW_ALGO_TILED
 # Every symbol include/dwconv2d.h declares.
 EXPORTS = ("dwconv2d_out_shape", "dwconv2d_resolved_pads", "dwconv2d_fwd",
            "dwconv2d_bwd_input", "dwconv2d_bwd_weight", "dwconv2d_bwd_weight_workspace_size",
+           "dwconv2d_bwd_weight_noalloc",
            "dwconv2d_query_algo", "dwconv2d_take_device_error", "dwconv2d_status_string",
            "dwconv2d_version")
 
@@ -76,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.dwconv2d_bwd_input.argtypes = [P(DwDesc), vp, vp, vp, vp]
     L.dwconv2d_bwd_weight.restype = i32
     L.dwconv2d_bwd_weight.argtypes = [P(DwDesc), vp, vp, vp, vp, vp, ctypes.c_uint64, vp]
+    L.dwconv2d_bwd_weight_noalloc.restype = i32
+    L.dwconv2d_bwd_weight_noalloc.argtypes = [P(DwDesc), vp, vp, vp, vp, vp]
     L.dwconv2d_bwd_weight_workspace_size.restype = i32
     L.dwconv2d_bwd_weight_workspace_size.argtypes = [P(DwDesc), P(ctypes.c_uint64)]
     L.dwconv2d_query_algo.restype = i32
@@ -181,6 +186,15 @@ def bwd_weight_raw(desc: DwDesc, x_ptr: int, dy_ptr: int, dw_ptr: int, db_ptr: O
     """dwconv2d_bwd_weight on raw device pointers; returns the status."""
     return int(lib().dwconv2d_bwd_weight(ctypes.byref(desc), x_ptr, dy_ptr, dw_ptr, db_ptr or None,
                                          ws_ptr, int(ws_bytes), stream or None))
+
+
+def bwd_weight_noalloc_raw(desc: DwDesc, x_ptr: int, dy_ptr: int, dw_ptr: int,
+                           db_ptr: Optional[int], stream: int) -> int:
+    """dwconv2d_bwd_weight_noalloc on raw device pointers; returns the status.
+    For callers that cannot allocate device memory: the scratch is a fixed
+    array inside the library (see include/dwconv2d.h)."""
+    return int(lib().dwconv2d_bwd_weight_noalloc(ctypes.byref(desc), x_ptr, dy_ptr, dw_ptr,
+                                                 db_ptr or None, stream or None))
 
 
 def dwconv2d_bwd_weight_workspace_size(desc: DwDesc) -> int:

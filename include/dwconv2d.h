@@ -75,7 +75,8 @@ enum {
     DW_ERR_UNSUPPORTED = 2,
     DW_ERR_ALIAS = 3,
     DW_ERR_CUDA = 4,
-    DW_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up waiting on a copy */
+    DW_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting on a copy */
+    DW_ERR_TOO_LARGE = 6       /* needs more scratch than the fixed device array holds */
 };
 
 enum { DW_NHWC = 0, DW_NCHW = 1 };                 /* dw_desc_t.layout   */
@@ -172,6 +173,35 @@ DW_API dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const float* x, co
 /* Workspace bytes dwconv2d_bwd_weight needs for `desc` (host only; depends
  * on the problem, not on the device or the pointers). */
 DW_API dw_status_t dwconv2d_bwd_weight_workspace_size(const dw_desc_t* desc, uint64_t* bytes);
+
+/*
+ * Weight and bias gradients for callers that cannot allocate device memory.
+ * The source pages have no counterpart to this entry point: it is the same
+ * computation as dwconv2d_bwd_weight, but its scratch is a fixed array inside
+ * the library instead of a caller workspace.  It is meant for code that
+ * cannot allocate at the call site: programs whose device memory is an arena
+ * reserved up front and that may not allocate more, and latency-critical
+ * paths where cudaMalloc / cudaFree are not acceptable because they can
+ * synchronise the device.
+ *   - Arguments and results as dwconv2d_bwd_weight (x, dy, dw, db are the
+ *     caller's device buffers; db may be NULL).
+ *   - The scratch is one array of DW_NOALLOC_SCRATCH_BYTES bytes per device;
+ *     every GPU that loads the library holds it until the process exits.
+ *     A problem whose dwconv2d_bwd_weight_workspace_size() exceeds it returns
+ *     DW_ERR_TOO_LARGE and launches nothing.
+ *   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *     library routine.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents;
+ *     the kernels write every scratch element before reading it, so nothing
+ *     has to be cleared between calls.  Calls that overlap on the GPU (for
+ *     example on two streams) race on the array: the caller must order them.
+ */
+#define DW_NOALLOC_SCRATCH_BYTES (16u << 20)
+DW_API dw_status_t dwconv2d_bwd_weight_noalloc(const dw_desc_t* desc, const float* x,
+                                               const float* dy, float* dw, float* db,
+                                               void* stream);
 
 /*
  * Which kernel family a call with these arguments would run (host only, no

@@ -42,7 +42,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert dw.dwconv2d_version() >= 10000
-    for st in range(6):
+    for st in range(7):
         assert dw.status_string(st).startswith("DW_")
 
 
