@@ -15,11 +15,14 @@
 //      rounding of the final value.
 //   2. a finalize kernel sums each channel's partials in a fixed order and
 //      writes dW / db as float32.
-// The tiled partial kernel (NHWC, TMA) loads, per tile, the input halo box
-// and the matching dy box into one pipeline stage; lane = channel (a warp
-// covers the 32 channels of a pixel), each thread owns THT x TWT outputs and
-// streams its input window once, feeding every (output, tap) pair at
-// compile-time offsets.  The direct partial kernels cover every other shape.
+// The tiled partial kernels load, per tile, the input halo box and the
+// matching dy box into one pipeline stage (TMA).  NHWC: lane = channel (a
+// warp covers the 32 channels of a pixel), each thread owns THT x TWT outputs
+// and streams its input window once, feeding every (output, tap) pair at
+// compile-time offsets.  NCHW (stride 1): lanes run along W, 4 outputs per
+// lane; a CTA works through whole units (one row band of one (n, c) plane)
+// and reduces each unit to one float64 partial per tap.  The direct partial
+// kernels cover every other shape.
 #include <climits>
 
 #include "dw_common.cuh"
@@ -495,9 +498,322 @@ dw_status_t launch_tiled(const Problem& p, const float* x, const float* dy, floa
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
+// ------------------------------------------------- tiled kernel, NCHW ------
+
+struct NArgs {
+    double* part;
+    int32_t* err;
+    int C, pt, pl;
+    int tiles_x, tiles_y;  // tiles per plane
+    int bands, band_rows;  // row bands per plane, tile rows per band
+    int units;             // N * C * bands
+};
+
+template <int KH_, int KW_, int REM_, int THT_, int WY_, int NS_>
+struct NWCfg {
+    static constexpr int KH = KH_, KW = KW_, REM = REM_, THT = THT_, WY = WY_, NS = NS_;
+    static constexpr int T = KH * KW + 1;
+    static constexpr int NCW = WY;  // consumer warps, one 128-column row strip each
+    static constexpr int NCT = NCW * 32;
+    static constexpr int NT = NCT + 32;
+    static constexpr int TW = 128, TH = THT * WY;
+    static constexpr int IH = TH + KH - 1;
+    static constexpr int IWB = (REM + TW + KW - 1 + 3) / 4 * 4;
+    static constexpr int NV = (REM + 3 + KW - 1) / 4 + 1;  // float4 per window row
+    static constexpr int XBYTES = IWB * IH * 4;
+    static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;
+    static constexpr int GBYTES = TW * TH * 4;
+    static constexpr int STAGE_BYTES = XPITCH + GBYTES;
+    static constexpr int RED_BYTES = NCW * T * 8;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + RED_BYTES + size_t(2 * NS) * 8 + 16;
+    static_assert(GBYTES % 128 == 0, "TMA shared-memory alignment");
+    static_assert(IWB <= 256 && IH <= 256, "TMA box limit");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    partial_tiled_nchw(const __grid_constant__ CUtensorMap xmap,
+                       const __grid_constant__ CUtensorMap gmap, const NArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    double* red = reinterpret_cast<double*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES + K::RED_BYTES);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    allow_dependents();
+
+    // unit u = (n*C + c) * bands + band; its tiles: rows of the band x all columns
+    auto unit_tiles = [&](int u, int& plane, int& ty0, int& rows) {
+        plane = u / a.bands;
+        const int band = u - plane * a.bands;
+        ty0 = band * a.band_rows;
+        rows = a.tiles_y - ty0 < a.band_rows ? a.tiles_y - ty0 : a.band_rows;
+    };
+
+    if (warp == K::NCW) {
+        if (lane == 0) {
+            prefetch_tensor_map(&xmap);
+            prefetch_tensor_map(&gmap);
+            int k = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < a.units && ok; u += G) {
+                int plane, ty0, rows;
+                unit_tiles(u, plane, ty0, rows);
+                const int c = plane % a.C, n = plane / a.C;
+                for (int r = 0; r < rows && ok; ++r)
+                    for (int tx = 0; tx < a.tiles_x; ++tx, ++k) {
+                        const int s = k % K::NS;
+                        if (k >= K::NS &&
+                            !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const int ty = ty0 + r;
+                        unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
+                        mbar_arrive_expect_tx(&full[s], K::XBYTES + K::GBYTES);
+                        tma_load_4d(st, &xmap, &full[s], tx * K::TW - a.pl - K::REM,
+                                    ty * K::TH - a.pt, c, n);
+                        tma_load_4d(st + K::XPITCH, &gmap, &full[s], tx * K::TW, ty * K::TH, c, n);
+                    }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
+        }
+        return;
+    }
+
+    const int row0 = warp * K::THT;
+    int k = 0;
+    bool failed = false;
+    for (int u = blockIdx.x; u < a.units; u += G) {
+        int plane, ty0, rows;
+        unit_tiles(u, plane, ty0, rows);
+        double acc64[K::T];
+#pragma unroll
+        for (int t = 0; t < K::T; ++t) acc64[t] = 0.0;
+        const int ntile = rows * a.tiles_x;
+        for (int i = 0; i < ntile && !failed; ++i, ++k) {
+            const int s = k % K::NS;
+            if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                }
+                failed = true;
+                break;
+            }
+            const unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
+            const float4* xw = reinterpret_cast<const float4*>(st) + row0 * (K::IWB / 4) + lane;
+            const float4* gw = reinterpret_cast<const float4*>(st + K::XPITCH) + row0 * (K::TW / 4) + lane;
+            float g[K::THT][4];
+#pragma unroll
+            for (int j = 0; j < K::THT; ++j) {
+                const float4 f = gw[j * (K::TW / 4)];
+                g[j][0] = f.x; g[j][1] = f.y; g[j][2] = f.z; g[j][3] = f.w;
+            }
+            float acc[K::KH][K::KW];
+#pragma unroll
+            for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw) acc[kh][kw] = 0.f;
+            static_for<0, K::THT + K::KH - 1>([&](auto r_) {
+                constexpr int r = decltype(r_)::value;
+                float v[4 * K::NV];
+#pragma unroll
+                for (int q = 0; q < K::NV; ++q) {
+                    const float4 f = xw[r * (K::IWB / 4) + q];
+                    v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+                }
+                static_for<0, K::THT>([&](auto j_) {
+                    constexpr int j = decltype(j_)::value;
+                    constexpr int kh = r - j;
+                    if constexpr (kh >= 0 && kh < K::KH) {
+#pragma unroll
+                        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                            for (int kw = 0; kw < K::KW; ++kw)
+                                acc[kh][kw] = fmaf(g[j][ii], v[K::REM + ii + kw], acc[kh][kw]);
+                    }
+                });
+            });
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            float gs = 0.f;
+#pragma unroll
+            for (int j = 0; j < K::THT; ++j) gs += (g[j][0] + g[j][1]) + (g[j][2] + g[j][3]);
+#pragma unroll
+            for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw) acc64[kh * K::KW + kw] += double(acc[kh][kw]);
+            acc64[K::T - 1] += double(gs);
+        }
+        // the unit's partial: warp sums, then the warps in order
+#pragma unroll
+        for (int t = 0; t < K::T; ++t) {
+            double v = acc64[t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) red[warp * K::T + t] = v;
+        }
+        named_barrier_sync(1, K::NCT);
+        if (tid < K::T) {
+            double sum = 0.0;
+            for (int w = 0; w < K::NCW; ++w) sum += red[w * K::T + tid];
+            a.part[int64_t(u) * K::T + tid] = sum;
+        }
+        named_barrier_sync(1, K::NCT);
+        if (failed) break;
+    }
+}
+
+// part[u*T + t], u = (n*C + c)*bands + band, summed over n and band in order.
+__global__ void __launch_bounds__(256) finalize_tiled_nchw(const double* __restrict__ part,
+                                                           float* __restrict__ dw,
+                                                           float* __restrict__ db, int N, int C,
+                                                           int T, int bands) {
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t n_items = int64_t(C) * T;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_items;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int c = int(i % C);
+        const int t = int(i / C);
+        double s = 0.0;
+        for (int n = 0; n < N; ++n)
+            for (int b = 0; b < bands; ++b) s += part[((int64_t(n) * C + c) * bands + b) * T + t];
+        if (t == T - 1) {
+            if (db) db[c] = float(s);
+        } else {
+            dw[int64_t(c) * (T - 1) + t] = float(s);
+        }
+    }
+}
+
+constexpr int kNchwUnitsCap = 2048;  // bands are added until N*C*bands reaches this
+
+int nchw_bands_cap(const Problem& p) {
+    const int64_t planes = p.N * p.C;
+    int64_t r = (kNchwUnitsCap + planes - 1) / planes;
+    return int(r < 1 ? 1 : r);
+}
+
+size_t tiled_nchw_workspace(const Problem& p) {
+    if (p.layout != DW_NCHW) return 0;
+    return size_t(p.N) * size_t(p.C) * size_t(nchw_bands_cap(p)) * size_t(p.kH * p.kW + 1) *
+           sizeof(double);
+}
+
+template <class K>
+dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy, float* dw,
+                              float* db, void* ws, cudaStream_t stream, int32_t* err,
+                              bool dry_run) {
+    NArgs a;
+    a.part = static_cast<double*>(ws);
+    a.err = err;
+    a.C = int(p.C);
+    a.pt = p.pt;
+    a.pl = p.pl;
+    const int64_t ty = (p.Ho + K::TH - 1) / K::TH, tx = (p.Wo + K::TW - 1) / K::TW;
+    if (ty >= INT_MAX || tx >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.tiles_x = int(tx);
+    a.tiles_y = int(ty);
+    const int64_t planes = p.N * p.C;
+    // enough units to spread over every SM, never more bands than tile rows
+    int64_t bands = (2 * 148 + planes - 1) / planes;
+    if (bands > nchw_bands_cap(p)) bands = nchw_bands_cap(p);
+    if (bands > ty) bands = ty;
+    if (bands < 1) bands = 1;
+    a.band_rows = int((ty + bands - 1) / bands);
+    a.bands = int((ty + a.band_rows - 1) / a.band_rows);
+    const int64_t units = planes * a.bands;
+    if (units >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.units = int(units);
+    if (dry_run) return DW_OK;
+
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&partial_tiled_nchw<K>), K::NT,
+                                   K::SMEM, cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+    int64_t G = int64_t(sm_count(dev)) * occ;
+    if (G > units) G = units;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap xmap, gmap;
+    const cuuint64_t xd[4] = {cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t xs[3] = {cuuint64_t(p.W) * 4, cuuint64_t(p.W * p.H) * 4,
+                              cuuint64_t(p.W * p.H * p.C) * 4};
+    const cuuint32_t xbox[4] = {K::IWB, K::IH, 1, 1};
+    const cuuint64_t gd[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * 4, cuuint64_t(p.Wo * p.Ho) * 4,
+                              cuuint64_t(p.Wo * p.Ho * p.C) * 4};
+    const cuuint32_t gbox[4] = {K::TW, K::TH, 1, 1};
+    if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
+                          xbox, estr) != CUDA_SUCCESS ||
+        encode_tensor_map(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(dy), gd, gs,
+                          gbox, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+    if (launch_pdl(partial_tiled_nchw<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap,
+                   gmap, a) != cudaSuccess)
+        return DW_ERR_CUDA;
+    int64_t fb = (p.C * K::T + 255) / 256;
+    const int64_t cap = int64_t(sm_count(dev)) * 8;
+    if (fb > cap) fb = cap;
+    if (launch_pdl(finalize_tiled_nchw, dim3(unsigned(fb)), dim3(256), 0, stream,
+                   static_cast<const double*>(a.part), dw, db, int(p.N), int(p.C), K::T,
+                   a.bands) != cudaSuccess)
+        return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+template <int KH, int KW, int THT, int WY, int NS>
+dw_status_t launch_nchw_rem(const Problem& p, const float* x, const float* dy, float* dw,
+                            float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    switch (((-p.pl) % 4 + 4) % 4) {
+        case 0: return launch_tiled_nchw<NWCfg<KH, KW, 0, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 1: return launch_tiled_nchw<NWCfg<KH, KW, 1, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 2: return launch_tiled_nchw<NWCfg<KH, KW, 2, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        default: return launch_tiled_nchw<NWCfg<KH, KW, 3, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    }
+}
+
+dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, float* dw,
+                            float* db, void* ws, cudaStream_t stream, int32_t* err,
+                            bool dry_run) {
+    if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
+    if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
+    if (p.W % 4 != 0 || p.Wo % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row pitches
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
+        return DW_ERR_UNSUPPORTED;
+    if (p.N >= INT_MAX || p.C >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    //                                                    KH KW THT WY NS
+    if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 5 && p.kW == 5) return launch_nchw_rem<5, 5, 4, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 7 && p.kW == 7) return launch_nchw_rem<7, 7, 2, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
 //                         KH KW  S  D THT TWT WX WY NS
 using W33s1 = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4>;
-using W33s2 = WCfg<3, 3, 2, 1, 1, 2, 4, 2, 4>;
+using W33s2 = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4>;
 using W55s1 = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3>;
 using W77s1 = WCfg<7, 7, 1, 1, 1, 4, 4, 2, 3>;
 using W1x15 = WCfg<1, 15, 1, 1, 1, 8, 8, 1, 4>;
@@ -505,6 +821,7 @@ using W1x31 = WCfg<1, 31, 1, 1, 1, 8, 8, 1, 4>;
 
 dw_status_t tiled_pick(const Problem& p, const float* x, const float* dy, float* dw, float* db,
                        void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.layout == DW_NCHW) return tiled_pick_nchw(p, x, dy, dw, db, ws, stream, err, dry_run);
     if (p.layout != DW_NHWC || p.C % 4 != 0) return DW_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
         return DW_ERR_UNSUPPORTED;
@@ -523,8 +840,11 @@ dw_status_t tiled_pick(const Problem& p, const float* x, const float* dy, float*
 }  // namespace wgrad
 
 size_t bwd_weight_workspace_bytes(const Problem& p) {
-    const size_t a = wgrad::direct_workspace(p), b = wgrad::tiled_workspace(p);
-    return a > b ? a : b;
+    size_t m = wgrad::direct_workspace(p);
+    const size_t b = wgrad::tiled_workspace(p), c = wgrad::tiled_nchw_workspace(p);
+    if (b > m) m = b;
+    if (c > m) m = c;
+    return m;
 }
 
 dw_status_t bwd_weight_launch(const Problem& p, int algo, const float* x, const float* dy,

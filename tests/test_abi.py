@@ -181,6 +181,11 @@ def test_weight_gradient_host_checks(lib):
     # kernel family selection (op 2 = weight gradient; no launch)
     T, D = dw.DW_ALGO_TILED, dw.DW_ALGO_DIRECT
     assert dw.dwconv2d_query_algo(desc, 2, x, dy, dwp) == T
-    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 3, 3, layout="nchw"), 2, x, dy, dwp) == D
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 3, 3, layout="nchw"), 2, x, dy, dwp) == T
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 7, 7, layout="nchw"), 2, x, dy, dwp) == T
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 18, 32, 3, 3, layout="nchw"), 2, x, dy, dwp) == D
+    assert dw.dwconv2d_query_algo(
+        dw.make_desc(2, 16, 16, 32, 3, 3, stride=2, layout="nchw"), 2, x, dy, dwp) == D
+    assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 1, 31, layout="nchw"), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 7, 3, 3), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 3, 3, dilation=2), 2, x, dy, dwp) == D

@@ -71,6 +71,15 @@ TILED = [
     Case("w_1x15", 4, 2, 300, 44, 1, 15, act="normal", seed=77),
     Case("w_1x31", 3, 3, 290, 68, 1, 31, act="normal", seed=78),
     Case("w_many_tiles", 16, 64, 64, 96, 3, 3, seed=79),
+    # NCHW, stride 1: the four column phases of the input box, bands, ragged edges
+    Case("w_nchw_3x3_same", 3, 37, 44, 20, 3, 3, layout="nchw", seed=81),
+    Case("w_nchw_3x3_pl0", 2, 29, 40, 12, 3, 3, padding=(0, 1, 0, 2), layout="nchw", seed=82),
+    Case("w_nchw_3x3_pl2", 2, 31, 36, 12, 3, 3, padding=(2, 0, 2, 0), layout="nchw", seed=83),
+    Case("w_nchw_3x3_pl3", 2, 26, 40, 12, 3, 3, padding=(1, 3, 3, 3), layout="nchw", seed=84),
+    Case("w_nchw_5x5", 2, 35, 52, 10, 5, 5, layout="nchw", seed=85),
+    Case("w_nchw_7x7", 2, 33, 28, 9, 7, 7, layout="nchw", seed=86),
+    Case("w_nchw_wide", 1, 70, 300, 3, 3, 3, layout="nchw", seed=87),
+    Case("w_nchw_planes", 8, 20, 24, 64, 3, 3, layout="nchw", seed=88),
 ]
 
 
@@ -93,8 +102,9 @@ def test_repeatable_bit_for_bit():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_large_full_size():
-    case = [c for c in wl.large() if c.H == 512 and c.layout == "nhwc"][0]
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+def test_large_full_size(layout):
+    case = [c for c in wl.large() if c.H == 512 and c.layout == layout][0]
     check(case, algos=("auto",))
 
 
