@@ -16,6 +16,11 @@ sections.  Readings where
 the page leaves a step open (SAME at stride > 1, bias dtype, batch axis,
 layouts) are documented in ``dw_oracle.c``.
 
+The fused forward epilogue (``bn_act``, ``fwd_bn_act``) follows the same
+page's section on the MLIR lowering, which names a depthwise conv + batch-norm
+emitter; it is read as inference-mode batch normalisation with running
+statistics followed by an optional activation (see ``dw_oracle.c``).
+
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 (hand-derived golden values, dense grouped-conv library routine, adjoint
 identity, decimation identities, closed forms).
@@ -47,7 +52,7 @@ def build(force: bool = False) -> str:
         return _LIB_PATH
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-shared", "-fPIC", _SRC, "-o", tmp]
+           "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -77,6 +82,9 @@ def _load():
     lib.dwo_bwd_weight.argtypes = [p_i64, p_f64, p_f64, p_f64, p_f64]
     lib.dwo_bwd_input_at.restype = None
     lib.dwo_bwd_input_at.argtypes = [p_i64, p_f64, p_f64, i64, p_i64, p_f64]
+    lib.dwo_bn_act.restype = None
+    lib.dwo_bn_act.argtypes = [i64, p_f64, p_i64, p_f64, p_f64, p_f64, p_f64,
+                               ctypes.c_double, i64, p_f64]
     _lib = lib
     return lib
 
@@ -225,3 +233,46 @@ def bwd_weight(prob, x, dy):
     db = np.empty(C, dtype=np.float64)
     _load().dwo_bwd_weight(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(dy), _ptr(dw), _ptr(db))
     return dw, db
+
+
+ACTS = {"none": 0, "relu": 1, "relu6": 2, "silu": 3}
+
+
+def channel_of(prob, flat_idx, out=True):
+    """Channel of each flat index of y (out=True) or x, in the problem's layout."""
+    idx = np.asarray(flat_idx, dtype=np.int64)
+    shape = out_shape(prob) if out else in_shape(prob)
+    if int(prob[14]) == 0:
+        return idx % shape[3]
+    return (idx // (shape[2] * shape[3])) % shape[1]
+
+
+def bn_act(prob, z, flat_idx=None, bn=None, act="none"):
+    """Fused epilogue applied to forward values z (float64).
+
+    z holds the forward output at the flat y indices `flat_idx` (all of y, in
+    layout order, when None).  bn = (gamma, beta, mean, var, eps) or None.
+    """
+    z = _f64(z)
+    flat = z.reshape(-1)
+    idx = np.arange(flat.size, dtype=np.int64) if flat_idx is None else \
+        np.ascontiguousarray(flat_idx, dtype=np.int64)
+    ch = np.ascontiguousarray(channel_of(prob, idx), dtype=np.int64)
+    out = np.empty_like(flat)
+    C = int(prob[3])
+    if bn is None:
+        g = be = mu = var = None
+        eps = 0.0
+    else:
+        g, be, mu, var = (_f64(v).reshape(C) for v in bn[:4])
+        eps = float(bn[4])
+    _load().dwo_bn_act(flat.size, _ptr(flat), _ptr(ch, ctypes.c_int64),
+                       None if g is None else _ptr(g), None if g is None else _ptr(be),
+                       None if g is None else _ptr(mu), None if g is None else _ptr(var),
+                       eps, ACTS[act], _ptr(out))
+    return out.reshape(z.shape)
+
+
+def fwd_bn_act(prob, x, w, b=None, bn=None, act="none"):
+    """act(batch_norm(forward(x)))  (float64); bn = (gamma, beta, mean, var, eps) or None."""
+    return bn_act(prob, fwd(prob, x, w, b), None, bn, act)

@@ -44,6 +44,7 @@
  */
 #include <stddef.h>
 #include <stdint.h>
+#include <math.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -260,5 +261,40 @@ void dwo_bwd_weight(const int64_t* p, const double* x, const double* dy, double*
                         acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)];
             db[c] = acc;
         }
+    }
+}
+
+/* Fused forward epilogue.  The page's section on the MLIR lowering names a
+ * depthwise-convolution-plus-batch-norm emitter without spelling the
+ * normalisation out; it is read here as inference-mode batch normalisation
+ * with per-channel running statistics, followed by an optional activation:
+ *     u = gamma[c] * (z - mean[c]) / sqrt(var[c] + eps) + beta[c]
+ *     out = act(u),  act in {identity, relu, relu6 = min(max(u,0),6),
+ *                            silu = u / (1 + exp(-u))}
+ * where z is the forward output (bias included) at an element of channel c.
+ * gamma == NULL skips the normalisation (u = z).  Applied element by element:
+ * z[i] belongs to channel ch[i]. */
+enum { DWO_ACT_NONE = 0, DWO_ACT_RELU = 1, DWO_ACT_RELU6 = 2, DWO_ACT_SILU = 3 };
+
+static double activation(double u, int64_t act) {
+    switch (act) {
+        case DWO_ACT_RELU: return u < 0.0 ? 0.0 : u;
+        case DWO_ACT_RELU6: return u < 0.0 ? 0.0 : (u > 6.0 ? 6.0 : u);
+        case DWO_ACT_SILU: return u / (1.0 + exp(-u));
+        default: return u;
+    }
+}
+
+void dwo_bn_act(int64_t count, const double* z, const int64_t* ch, const double* gamma,
+                const double* beta, const double* mean, const double* var, double eps,
+                int64_t act, double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        double u = z[i];
+        if (gamma) {
+            int64_t c = ch[i];
+            u = gamma[c] * (u - mean[c]) / sqrt(var[c] + eps) + beta[c];
+        }
+        out[i] = activation(u, act);
     }
 }

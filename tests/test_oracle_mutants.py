@@ -43,6 +43,13 @@ MUTANTS = {
     "wgrad_transposed_taps": ("dw[(c * kH + kh) * kW + kw] = acc;", "dw[(c * kW + kw) * kH + kh] = acc;"),
     "bwd_at_channel_mix": ("acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *\n                       wt[(c * kH + kh) * kW + kw];",
                            "acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *\n                       wt[(((c + 1) % p[P_C]) * kH + kh) * kW + kw];"),
+    "bn_dropped_eps": ("(u - mean[c]) / sqrt(var[c] + eps)", "(u - mean[c]) / sqrt(var[c])"),
+    "bn_mean_sign": ("(u - mean[c])", "(u + mean[c])"),
+    "bn_channel_ignored": ("int64_t c = ch[i];", "int64_t c = 0;"),
+    "bn_bias_after_norm": ("gamma[c] * (u - mean[c]) / sqrt(var[c] + eps) + beta[c]",
+                           "gamma[c] * u / sqrt(var[c] + eps) + beta[c] - mean[c]"),
+    "relu6_no_upper_clamp": ("(u > 6.0 ? 6.0 : u)", "u"),
+    "silu_wrong_sign": ("u / (1.0 + exp(-u))", "u / (1.0 + exp(u))"),
 }
 
 
@@ -56,7 +63,7 @@ def build_variant(tmp_path, name, patch):
     c_path.write_text(src)
     so_path = tmp_path / f"lib{name}.so"
     subprocess.run(["gcc", "-O1", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC",
-                    str(c_path), "-o", str(so_path)], check=True)
+                    str(c_path), "-o", str(so_path), "-lm"], check=True)
     return str(so_path)
 
 
@@ -75,6 +82,8 @@ def run_pin_subset():
         ("sampled", lambda: pins.test_sampled_evaluators_match_full(None)),
         ("golden_wgrad", lambda: pins.test_golden_weight_gradient(None)),
         ("wgrad_linearity", lambda: pins.test_weight_gradient_linearity_identity(None)),
+        ("golden_bn_act", lambda: [pins.test_golden_bn_act(None, l) for l in ("nhwc", "nchw")]),
+        ("torch_bn_act", lambda: pins.test_bn_act_equals_torch_batch_norm_and_activations(None)),
     ]
     for name, fn in checks:
         try:

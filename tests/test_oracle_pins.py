@@ -523,3 +523,82 @@ def test_bias_gradient_closed_form(oracle_mod):
         _, db = oracle.bwd_weight(p, rng.standard_normal(oracle.in_shape(p)), dy)
         axes = (0, 1, 2) if layout == "nhwc" else (0, 2, 3)
         np.testing.assert_allclose(db, dy.sum(axis=axes), rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------- fused batch norm + activation ---
+
+ACTS = ["none", "relu", "relu6", "silu"]
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+def test_golden_bn_act(oracle_mod, layout):
+    g = load_golden("bn_act_2ch.json")
+    p = prob1(g["H"], g["W"], g["C"], g["kH"], g["kW"], 1, 1, g["pads"], layout=layout)
+    x = chw_to(layout, g["x"])
+    bn = (g["gamma"], g["beta"], g["mean"], g["var"], g["eps"])
+    for act in ACTS:
+        y = to_chw(layout, oracle.fwd_bn_act(p, x, g["w"], g["b"], bn, act))
+        want = np.array(g["out"][act])
+        tol = g["silu_tolerance"] if act == "silu" else 0.0
+        assert np.allclose(y, want, rtol=0, atol=tol), (act, y, want)
+
+
+def random_bn(rng, C):
+    return (rng.uniform(-1.5, 1.5, C), rng.uniform(-0.5, 0.5, C), rng.uniform(-0.3, 0.3, C),
+            rng.uniform(0.2, 2.0, C), float(rng.choice([1e-5, 1e-3, 0.1])))
+
+
+def torch_bn_act(z_nchw, bn, act):
+    g, be, mu, var = (torch.tensor(np.asarray(v), dtype=torch.float64) for v in bn[:4])
+    eps = bn[4]
+    u = F.batch_norm(torch.from_numpy(z_nchw), mu, var, g, be, training=False, eps=eps)
+    return {"none": lambda t: t, "relu": F.relu, "relu6": F.relu6, "silu": F.silu}[act](u).numpy()
+
+
+def test_bn_act_equals_torch_batch_norm_and_activations(oracle_mod):
+    # the library's eval-mode batch norm and activation functions, float64
+    rng = np.random.default_rng(404)
+    for p, _, _ in valid_cases(405, 20):
+        x = rng.uniform(-2, 2, oracle.in_shape(p))
+        C = int(p[3])
+        w = rng.normal(0, 1, (C, int(p[4]), int(p[5])))
+        b = rng.uniform(-0.5, 0.5, C)
+        bn = random_bn(rng, C)
+        z = to_nchw(p, oracle.fwd(p, x, w, b))
+        for act in ACTS:
+            got = to_nchw(p, oracle.fwd_bn_act(p, x, w, b, bn, act))
+            want = torch_bn_act(z, bn, act)
+            assert np.allclose(got, want, rtol=1e-13, atol=1e-14), act
+
+
+def test_bn_identity_statistics_reduce_to_plain_forward(oracle_mod):
+    # gamma = sqrt(var + eps), beta = mean: the normalisation is the identity
+    rng = np.random.default_rng(406)
+    for p, _, _ in valid_cases(407, 10):
+        C = int(p[3])
+        x = rng.uniform(-1, 1, oracle.in_shape(p))
+        w = rng.normal(0, 1, (C, int(p[4]), int(p[5])))
+        var, eps = rng.uniform(0.5, 3, C), 1e-3
+        mean = rng.uniform(-1, 1, C)
+        bn = (np.sqrt(var + eps), mean, mean, var, eps)
+        y = oracle.fwd(p, x, w, None)
+        assert np.allclose(oracle.fwd_bn_act(p, x, w, None, bn, "none"), y, rtol=1e-13, atol=1e-13)
+        assert np.array_equal(oracle.fwd_bn_act(p, x, w, None, None, "relu"), np.maximum(y, 0))
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+def test_bn_act_constant_input_closed_form(oracle_mod, layout):
+    # x = a everywhere, 3x3 SAME: an interior output is a*sum(W[c]) + b[c]
+    a, C = 0.75, 3
+    p = oracle.problem((1, 5, 5, C) if layout == "nhwc" else (1, C, 5, 5), 3, 3, layout=layout)
+    w = np.arange(C * 9, dtype=np.float64).reshape(C, 3, 3) / 20.0 - 0.4
+    b = np.array([0.1, -0.2, 0.3])
+    bn = ([1.5, -2.0, 0.5], [0.25, 0.0, -1.0], [1.0, -0.5, 2.0], [0.44, 3.0, 0.01], 0.06)
+    for act in ACTS:
+        y = to_chw(layout, oracle.fwd_bn_act(p, np.full(oracle.in_shape(p), a), w, b, bn, act))
+        for c in range(C):
+            z = a * w[c].sum() + b[c]
+            u = bn[0][c] * (z - bn[2][c]) / np.sqrt(bn[3][c] + bn[4]) + bn[1][c]
+            want = {"none": u, "relu": max(u, 0.0), "relu6": min(max(u, 0.0), 6.0),
+                    "silu": u / (1.0 + np.exp(-u))}[act]
+            assert abs(y[c, 2, 2] - want) <= 1e-12 * max(1.0, abs(want)), (act, c)
