@@ -76,6 +76,10 @@ def algorithmic_bytes(case, Ho, Wo, op):
     wbytes = case.C * case.kH * case.kW * (2 if case.wtype == "f16" else 4)
     if op == "fwd":
         return 4 * n_in + 4 * n_out + wbytes + (4 * case.C if case.bias else 0)
+    if op == "fused":  # forward + four [C] batch-norm statistics
+        return 4 * n_in + 4 * n_out + wbytes + (4 * case.C if case.bias else 0) + 16 * case.C
+    if op == "wgrad":  # read x and dy, write dW [C,kH,kW] and db [C] (f32)
+        return 4 * n_in + 4 * n_out + 4 * case.C * case.kH * case.kW + 4 * case.C
     return 4 * n_out + 4 * n_in + wbytes
 
 
@@ -200,9 +204,33 @@ class Shape:
                 "dx": torch.empty(case.in_shape(), device=device)})
         self.set_bytes = sum(t.numel() * 4 for t in self.sets[0].values())
 
+    def prepare_next_rows(self, dw, torch, device, act):
+        """Buffers of the calls measured beside the step: the weight gradient
+        and the forward with the fused batch-norm / activation epilogue."""
+        from depthwise_convolution_fwd_b200.workloads import make_bn
+        c = self.case
+        self.act = act
+        self.bn = [t.to(device) for t in make_bn(c.C, c.seed + 500)[:4]]
+        self.ws_bytes = dw.dwconv2d_bwd_weight_workspace_size(self.desc)
+        self.ws = torch.empty(max(1, self.ws_bytes), dtype=torch.uint8, device=device)
+        self.dW = torch.empty(c.C * c.kH * c.kW, device=device)
+        self.db = torch.empty(c.C, device=device)
+        for op in ("fused", "wgrad"):
+            self.bytes[op] = algorithmic_bytes(c, self.Ho, self.Wo, op)
+
     def call(self, dw, op, r, stream):
         s = self.sets[r % len(self.sets)]
-        if op == "fwd":
+        if op == "fused":
+            acts = {"relu": dw.DW_ACT_RELU, "relu6": dw.DW_ACT_RELU6, "silu": dw.DW_ACT_SILU}
+            st = dw.fwd_bn_act_raw(self.desc, s["x"].data_ptr(), self.w.data_ptr(),
+                                   None if self.b is None else self.b.data_ptr(),
+                                   [t.data_ptr() for t in self.bn], 1e-5, acts[self.act],
+                                   s["y"].data_ptr(), stream)
+        elif op == "wgrad":
+            st = dw.bwd_weight_raw(self.desc, s["x"].data_ptr(), s["dy"].data_ptr(),
+                                   self.dW.data_ptr(), self.db.data_ptr(), self.ws.data_ptr(),
+                                   self.ws_bytes, stream)
+        elif op == "fwd":
             st = dw.fwd_raw(self.desc, s["x"].data_ptr(), self.w.data_ptr(),
                             None if self.b is None else self.b.data_ptr(), s["y"].data_ptr(), stream)
         else:
@@ -292,26 +320,7 @@ def run_ours(args, rank, world, local_rank):
     # one kernel over enough buffer copies that its inputs come from HBM
     kernels = {}
     for sh, op in ops:
-        per = sh.bytes[op]
-        reuse = max(len(sh.sets), -(-int(3 * l2) // max(1, per)))
-        extra = []
-        if reuse > len(sh.sets):
-            for _ in range(reuse - len(sh.sets)):
-                extra.append({k: torch.empty_like(v).copy_(v) for k, v in sh.sets[0].items()})
-        pool = sh.sets + extra
-        saved = sh.sets
-        sh.sets = pool
-        launches = len(pool)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for r in range(launches):
-                sh.call(dw, op, r, stream.cuda_stream)
-        reps = max(3, int(60e-3 / max(1e-6, per / 6e12) / launches))
-        ms_k = time_graph(torch, g, reps, stream) / (reps * launches)
-        sh.sets = saved
-        del g, extra, pool
-        key = f"{sh.case.name}:{op}"
-        kernels[key] = {"us": ms_k * 1e3, "bytes": per, "gbs": per / (ms_k * 1e-3) / 1e9}
+        kernels[f"{sh.case.name}:{op}"] = time_kernel(torch, dw, sh, op, l2, stream)
     total_us = sum(v["us"] for v in kernels.values())
     for v in kernels.values():
         v["share"] = v["us"] / total_us
@@ -319,6 +328,24 @@ def run_ours(args, rank, world, local_rank):
     dom = kernels[dom_key]
     peak, peak_kind = load_peaks()
     traffic = load_traffic(args.workload).get(dom_key)
+
+    # the rows measured beside the step (not part of it): weight gradient, and
+    # the forward with the fused batch-norm + activation epilogue
+    next_rows = {}
+    if not args.no_next_rows:
+        act = "silu" if args.workload == "conformer" else "relu6"
+        for sh in shapes:
+            sh.prepare_next_rows(dw, torch, device, act)
+            with torch.cuda.stream(stream):
+                for op in ("fused", "wgrad"):
+                    sh.call(dw, op, 0, sptr)
+            torch.cuda.synchronize()
+            for op in ("fused", "wgrad"):
+                k = time_kernel(torch, dw, sh, op, l2, stream)
+                k["frac"] = k["gbs"] / peak
+                if op == "fused":
+                    k["epilogue"] = f"inference batch norm + {act}"
+                next_rows[f"{sh.case.name}:{op}"] = k
 
     # end to end through the public tensor API: pinned host inputs -> device,
     # forward + input gradient, outputs -> pinned host, every step
@@ -346,6 +373,7 @@ def run_ours(args, rank, world, local_rank):
                      "timing": "avg launch of a CUDA graph of back-to-back launches, inputs "
                                "rotated over buffer copies > 3x L2, CUDA events"},
         "kernels": kernels,
+        "next_rows": next_rows,
         "e2e": e2e,
         "gpu_launches": len(ops) * args.steps,
         "clocks": clocks,
@@ -356,6 +384,30 @@ def run_ours(args, rank, world, local_rank):
     for g in graphs:
         del g
     return result
+
+
+def time_kernel(torch, dw, sh, op, l2, stream):
+    """Average launch time of one call: a CUDA graph of back-to-back launches
+    over enough buffer copies (> 3x L2) that its inputs come from HBM."""
+    per = sh.bytes[op]
+    reuse = max(len(sh.sets), -(-int(3 * l2) // max(1, per)))
+    extra = []
+    if reuse > len(sh.sets):
+        for _ in range(reuse - len(sh.sets)):
+            extra.append({k: torch.empty_like(v).copy_(v) for k, v in sh.sets[0].items()})
+    pool = sh.sets + extra
+    saved = sh.sets
+    sh.sets = pool
+    launches = len(pool)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for r in range(launches):
+            sh.call(dw, op, r, stream.cuda_stream)
+    reps = max(3, int(60e-3 / max(1e-6, per / 6e12) / launches))
+    ms_k = time_graph(torch, g, reps, stream) / (reps * launches)
+    sh.sets = saved
+    del g, extra, pool
+    return {"us": ms_k * 1e3, "bytes": per, "gbs": per / (ms_k * 1e-3) / 1e9}
 
 
 def run_e2e(args, torch, dw, shapes, device, stream, world):
@@ -537,6 +589,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=8.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the weight-gradient and fused-epilogue measurements")
     ap.add_argument("--profile", metavar="SHAPE:OP", default=None,
                     help="launch only this kernel (e.g. mobilenet_32x56x56x144_3x3_s2:fwd) "
                          "--steps times on one buffer set, untimed; for ncu captures")

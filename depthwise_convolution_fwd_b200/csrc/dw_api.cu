@@ -201,12 +201,20 @@ static dw_status_t check_buffers(const Problem& p, Op op, const Buffers& bf) {
 }
 
 static dw_status_t run(const dw_desc_t* desc, Op op, const Buffers& bf, cudaStream_t stream,
-                       bool dry_run, int32_t* chosen) {
+                       bool dry_run, int32_t* chosen, const Epilogue* epi = nullptr) {
     Problem p;
     dw_status_t st = resolve(desc, &p);
     if (st != DW_OK) return st;
     st = check_buffers(p, op, bf);
     if (st != DW_OK) return st;
+    if (epi) {
+        // every statistics array must stay clear of y
+        const size_t yb = size_t(p.N) * size_t(p.C) * size_t(p.Ho) * size_t(p.Wo) * 4;
+        const float* stats[4] = {epi->gamma, epi->beta, epi->mean, epi->var};
+        for (const float* v : stats)
+            if (overlaps(bf.out, yb, v, size_t(p.C) * 4)) return DW_ERR_ALIAS;
+        p.epi = *epi;
+    }
     const int algo = desc->algo;
     int32_t* err = nullptr;
     if (!dry_run) {
@@ -256,6 +264,25 @@ dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const float* x, const void* w, c
                          float* y, void* stream) {
     return run(desc, OP_FWD, Buffers{x, w, b, y}, static_cast<cudaStream_t>(stream), false,
                nullptr);
+}
+
+dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const float* x, const void* w,
+                                const float* b, const float* gamma, const float* beta,
+                                const float* mean, const float* var, float eps, int32_t act,
+                                float* y, void* stream) {
+    const int given = (gamma != nullptr) + (beta != nullptr) + (mean != nullptr) + (var != nullptr);
+    if (given != 0 && given != 4) return DW_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !(eps <= 3.402823466e38f)) return DW_ERR_INVALID_ARG;  // NaN, inf, < 0
+    if (act < DW_ACT_NONE || act > DW_ACT_SILU) return DW_ERR_INVALID_ARG;
+    Epilogue e;
+    e.gamma = gamma;
+    e.beta = beta;
+    e.mean = mean;
+    e.var = var;
+    e.eps = eps;
+    e.act = act;
+    return run(desc, OP_FWD, Buffers{x, w, b, y}, static_cast<cudaStream_t>(stream), false,
+               nullptr, &e);
 }
 
 dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy, const void* w, float* dx,

@@ -14,6 +14,18 @@
 
 namespace dw {
 
+// Fused forward epilogue: inference-mode batch normalisation (per-channel
+// running statistics; gamma == nullptr means none) and an activation.
+struct Epilogue {
+    const float* gamma = nullptr;
+    const float* beta = nullptr;
+    const float* mean = nullptr;
+    const float* var = nullptr;
+    float eps = 0.f;
+    int act = DW_ACT_NONE;
+    __host__ __device__ bool on() const { return gamma != nullptr || act != DW_ACT_NONE; }
+};
+
 // A resolved problem: everything the kernels need, pads already resolved.
 // H, W, C, N are the extents of x (forward input) / dx (gradient output);
 // Ho, Wo the extents of y / dy.
@@ -23,6 +35,7 @@ struct Problem {
     int pt, pb, pl, pr;
     int layout;  // DW_NHWC / DW_NCHW
     int wtype;   // DW_F32 / DW_F16
+    Epilogue epi;  // forward only; off for every other call
 };
 
 enum Op { OP_FWD = 0, OP_BWD_INPUT = 1 };
@@ -54,6 +67,59 @@ int sm_count(int dev);
 CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank,
                            void* base, const cuuint64_t* dims, const cuuint64_t* strides,
                            const cuuint32_t* box, const cuuint32_t* elem_strides);
+
+// Per-channel scale and shift of the epilogue's normalisation:
+// scale = gamma / sqrt(var + eps), shift = beta - mean * scale (IEEE division
+// and square root); without statistics scale = 1 and shift = -0, so that
+// fmaf(z, scale, shift) == z for every z, -0 included.
+__device__ __forceinline__ void bn_scale_shift(const Epilogue& e, int c, float& scale,
+                                               float& shift) {
+    if (e.gamma != nullptr) {
+        scale = __ldg(e.gamma + c) / sqrtf(__ldg(e.var + c) + e.eps);
+        shift = fmaf(-__ldg(e.mean + c), scale, __ldg(e.beta + c));
+    } else {
+        scale = 1.f;
+        shift = -0.f;
+    }
+}
+
+// The activation; comparisons written so that NaN passes through.
+// silu: u / (1 + e^-u) with expf (at most 2 ulp) and the fast division
+// __fdividef (at most 2 ulp while the divisor stays below 2^126; beyond, at
+// u < -87.3, it returns 0 where the true value is below 1e-35 in magnitude).
+// The correctly rounded division or reciprocal costs a third of the large
+// NHWC forward's time; this form keeps the epilogue near the memory bound.
+template <int ACT>
+__device__ __forceinline__ float activate(float u) {
+    if constexpr (ACT == DW_ACT_RELU) return u < 0.f ? 0.f : u;
+    if constexpr (ACT == DW_ACT_RELU6) return u < 0.f ? 0.f : (u > 6.f ? 6.f : u);
+    if constexpr (ACT == DW_ACT_SILU) return __fdividef(u, 1.f + expf(-u));
+    return u;
+}
+
+// act(z * scale + shift)
+template <int ACT>
+__device__ __forceinline__ float epilogue_act(float z, float scale, float shift) {
+    return activate<ACT>(fmaf(z, scale, shift));
+}
+
+// Run-time activation (the direct kernels).
+__device__ __forceinline__ float epilogue_apply(float z, float scale, float shift, int act) {
+    switch (act) {
+        case DW_ACT_RELU: return epilogue_act<DW_ACT_RELU>(z, scale, shift);
+        case DW_ACT_RELU6: return epilogue_act<DW_ACT_RELU6>(z, scale, shift);
+        case DW_ACT_SILU: return epilogue_act<DW_ACT_SILU>(z, scale, shift);
+        default: return epilogue_act<DW_ACT_NONE>(z, scale, shift);
+    }
+}
+
+// Kernel instantiation of an epilogue: -1 = none (plain forward, and every
+// gradient kernel), else the activation.  The tiled kernels fold the
+// normalisation into the filter and bias they hold in registers (W' = scale *
+// W, b' = scale * b + shift, exact when the statistics are absent: scale 1,
+// shift -0), so the only per-output work left is the activation.
+constexpr int kNoEpilogue = -1;
+inline int epilogue_variant(const Epilogue& e) { return e.on() ? e.act : kNoEpilogue; }
 
 // Launch with programmatic stream serialization (see grid_dependency_wait).
 template <class... KArgs, class... Actual>

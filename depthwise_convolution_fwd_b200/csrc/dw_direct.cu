@@ -19,6 +19,7 @@ struct DirectArgs {
     int kH, kW, sh, sw, dh, dw, pt, pl;
     int wtype;
     int64_t total;
+    Epilogue epi;  // forward only
 };
 
 template <int LAYOUT>
@@ -65,6 +66,11 @@ __global__ void __launch_bounds__(256) direct_fwd_kernel(const float* __restrict
             }
         }
         if (b) acc += __ldg(b + c);
+        if (a.epi.on()) {
+            float scale, shift;
+            bn_scale_shift(a.epi, int(c), scale, shift);
+            acc = epilogue_apply(acc, scale, shift, a.epi.act);
+        }
         y[i] = acc;
     }
 }
@@ -107,6 +113,7 @@ dw_status_t direct_launch(const Problem& p, Op op, const float* in, const void* 
     a.N = p.N; a.C = p.C; a.H = p.H; a.W = p.W; a.Ho = p.Ho; a.Wo = p.Wo;
     a.kH = p.kH; a.kW = p.kW; a.sh = p.sh; a.sw = p.sw; a.dh = p.dh; a.dw = p.dw;
     a.pt = p.pt; a.pl = p.pl; a.wtype = p.wtype;
+    a.epi = op == OP_FWD ? p.epi : Epilogue{};
     a.total = p.N * p.C * (op == OP_FWD ? p.Ho * p.Wo : p.H * p.W);
     const int threads = 256;
     const int dev = current_device();

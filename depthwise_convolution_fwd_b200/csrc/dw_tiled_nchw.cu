@@ -37,6 +37,7 @@ struct Args {
     int pt, pl;  // effective low pads of the correlation this kernel runs
     FastDiv tiles_x, tiles_y, tiles_c;
     int ntiles;
+    Epilogue epi;  // used by the EPI instantiations only
 };
 
 template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
@@ -82,9 +83,12 @@ __device__ __forceinline__ void decode_tile(int t, const Args& a, int& tx, int& 
     c = r - n * a.tiles_c.d;   // ROWS: channel group; else channel
 }
 
-template <class K>
+// EPI: kNoEpilogue, or the activation of the fused batch-norm / activation
+// epilogue of the forward.
+template <class K, int EPI>
 __global__ void __launch_bounds__(K::NT, K::MINB)
     tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
+    static_assert(EPI == kNoEpilogue || !K::REV, "the epilogue belongs to the forward");
     extern __shared__ __align__(128) unsigned char smem[];
     float* stages = reinterpret_cast<float*>(smem);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH);
@@ -150,6 +154,11 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     float bias = 0.f;
     int cur_key = -1;
     bool live = false;
+    // the value stored for one output: acc + bias (-> epilogue)
+    auto finish = [&](float v) -> float {
+        if constexpr (EPI != kNoEpilogue) return activate<EPI>(v + bias);
+        else return v + bias;
+    };
 
     int k = 0;
     for (int t = t_begin; t < t_end; ++t, ++k) {
@@ -171,6 +180,18 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     wr[kh][kw] = live ? load_weight(a.w, a.wtype, base + src) : 0.f;
                 }
             bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
+            if constexpr (EPI != kNoEpilogue) {
+                // fold the normalisation into the filter and the bias
+                if (live) {
+                    float sc, sh;
+                    bn_scale_shift(a.epi, c, sc, sh);
+#pragma unroll
+                    for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] *= sc;
+                    bias = fmaf(bias, sc, sh);
+                }
+            }
         }
 
         if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
@@ -225,8 +246,8 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 const int ho = K::ROWS ? ty : ty * K::TH + row0 + j;
                 if (ho >= a.Hout) continue;
                 float* dst = a.out + ((int64_t(n) * a.C + c) * a.Hout + ho) * a.Wout + wo0;
-                const float4 v = make_float4(acc[j][0] + bias, acc[j][1] + bias, acc[j][2] + bias,
-                                             acc[j][3] + bias);
+                const float4 v = make_float4(finish(acc[j][0]), finish(acc[j][1]),
+                                             finish(acc[j][2]), finish(acc[j][3]));
                 if ((a.Wout & 3) == 0 && wo0 + 3 < a.Wout) {
                     store4(dst, v);
                 } else {
@@ -265,12 +286,21 @@ dw_status_t launch(const Problem& p, const float* in, const void* w, const float
     a.tiles_y = make_fastdiv(static_cast<int>(ty));
     a.tiles_c = make_fastdiv(static_cast<int>(tc));
     a.ntiles = static_cast<int>(nt);
+    a.epi = K::REV ? Epilogue{} : p.epi;
     if (dry_run) return DW_OK;
 
-    static LaunchCache cache;
+    const int ev = epilogue_variant(a.epi);
+    void (*kern)(CUtensorMap, Args) = tiled_kernel<K, kNoEpilogue>;
+    if constexpr (!K::REV) {
+        if (ev == DW_ACT_NONE) kern = tiled_kernel<K, DW_ACT_NONE>;
+        if (ev == DW_ACT_RELU) kern = tiled_kernel<K, DW_ACT_RELU>;
+        if (ev == DW_ACT_RELU6) kern = tiled_kernel<K, DW_ACT_RELU6>;
+        if (ev == DW_ACT_SILU) kern = tiled_kernel<K, DW_ACT_SILU>;
+    }
+    static LaunchCache cache[5];
     const int dev = current_device();
-    const int occ = prepare_kernel(reinterpret_cast<const void*>(&tiled_kernel<K>), K::NT,
-                                   K::SMEM, cache, dev);
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(kern), K::NT, K::SMEM,
+                                   cache[ev + 1], dev);
     if (occ < 1) return DW_ERR_CUDA;
 
     CUtensorMap map;
@@ -284,8 +314,8 @@ dw_status_t launch(const Problem& p, const float* in, const void* w, const float
         return DW_ERR_CUDA;
     int64_t grid = int64_t(sm_count(dev)) * occ;
     if (grid > a.ntiles) grid = a.ntiles;
-    if (launch_pdl(tiled_kernel<K>, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM,
-                   stream, map, a) != cudaSuccess)
+    if (launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream, map,
+                   a) != cudaSuccess)
         return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
@@ -325,10 +355,11 @@ struct ClCfg {
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-template <class K>
+template <class K, int EPI>
 __global__ void __launch_bounds__(K::NT, 1)
     chl_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
                const Args a, const int tma_store) {
+    static_assert(EPI == kNoEpilogue || !K::REV, "the epilogue belongs to the forward");
     extern __shared__ __align__(128) unsigned char smem[];
     float* stages = reinterpret_cast<float*>(smem);
     float* outbuf = reinterpret_cast<float*>(smem + size_t(K::NS) * K::STAGE_PITCH);
@@ -386,6 +417,11 @@ __global__ void __launch_bounds__(K::NT, 1)
     float bias = 0.f;
     int cur_key = -1;
     bool live = false;
+    // the value stored for one output: acc + bias (-> epilogue)
+    auto finish = [&](float v) -> float {
+        if constexpr (EPI != kNoEpilogue) return activate<EPI>(v + bias);
+        else return v + bias;
+    };
     int k = 0;
     for (int t = t_begin; t < t_end; ++t, ++k) {
         const int s = k % K::NS;
@@ -408,6 +444,16 @@ __global__ void __launch_bounds__(K::NT, 1)
                 for (int kw = 0; kw < K::KW; ++kw) wr[kw] = __ldg(wp + (K::REV ? K::KW - 1 - kw : kw));
             }
             bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
+            if constexpr (EPI != kNoEpilogue) {
+                // fold the normalisation into the filter and the bias
+                if (live) {
+                    float sc, sh;
+                    bn_scale_shift(a.epi, c, sc, sh);
+#pragma unroll
+                    for (int kw = 0; kw < K::KW; ++kw) wr[kw] *= sc;
+                    bias = fmaf(bias, sc, sh);
+                }
+            }
         }
 
         if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
@@ -450,8 +496,8 @@ __global__ void __launch_bounds__(K::NT, 1)
                         lane * (K::TWT / 4);
 #pragma unroll
             for (int u = 0; u < K::TWT / 4; ++u)
-                o[u] = make_float4(acc[4 * u] + bias, acc[4 * u + 1] + bias, acc[4 * u + 2] + bias,
-                                   acc[4 * u + 3] + bias);
+                o[u] = make_float4(finish(acc[4 * u]), finish(acc[4 * u + 1]),
+                                   finish(acc[4 * u + 2]), finish(acc[4 * u + 3]));
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -465,8 +511,8 @@ __global__ void __launch_bounds__(K::NT, 1)
             const bool vec = (a.Wout & 3) == 0;
 #pragma unroll
             for (int u = 0; u < K::TWT / 4; ++u) {
-                const float4 v = make_float4(acc[4 * u] + bias, acc[4 * u + 1] + bias,
-                                             acc[4 * u + 2] + bias, acc[4 * u + 3] + bias);
+                const float4 v = make_float4(finish(acc[4 * u]), finish(acc[4 * u + 1]),
+                                             finish(acc[4 * u + 2]), finish(acc[4 * u + 3]));
                 const int wo = wo0 + 4 * u;
                 if (vec && wo + 3 < a.Wout) {
                     store4(dst + 4 * u, v);
@@ -508,12 +554,21 @@ dw_status_t launch_chl(const Problem& p, const float* in, const void* w, const f
     a.tiles_y = make_fastdiv(static_cast<int>(ty));
     a.tiles_c = make_fastdiv(static_cast<int>(tc));
     a.ntiles = static_cast<int>(nt);
+    a.epi = K::REV ? Epilogue{} : p.epi;
     if (dry_run) return DW_OK;
 
-    static LaunchCache cache;
+    const int ev = epilogue_variant(a.epi);
+    void (*kern)(CUtensorMap, CUtensorMap, Args, int) = chl_kernel<K, kNoEpilogue>;
+    if constexpr (!K::REV) {
+        if (ev == DW_ACT_NONE) kern = chl_kernel<K, DW_ACT_NONE>;
+        if (ev == DW_ACT_RELU) kern = chl_kernel<K, DW_ACT_RELU>;
+        if (ev == DW_ACT_RELU6) kern = chl_kernel<K, DW_ACT_RELU6>;
+        if (ev == DW_ACT_SILU) kern = chl_kernel<K, DW_ACT_SILU>;
+    }
+    static LaunchCache cache[5];
     const int dev = current_device();
-    const int occ = prepare_kernel(reinterpret_cast<const void*>(&chl_kernel<K>), K::NT, K::SMEM,
-                                   cache, dev);
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(kern), K::NT, K::SMEM,
+                                   cache[ev + 1], dev);
     if (occ < 1) return DW_ERR_CUDA;
     CUtensorMap map;
     const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.C), cuuint64_t(p.N)};
@@ -541,8 +596,8 @@ dw_status_t launch_chl(const Problem& p, const float* in, const void* w, const f
     }
     int64_t grid = int64_t(sm_count(dev)) * occ;
     if (grid > a.ntiles) grid = a.ntiles;
-    if (launch_pdl(chl_kernel<K>, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream,
-                   map, omap, a, tma_store) != cudaSuccess)
+    if (launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream, map,
+                   omap, a, tma_store) != cudaSuccess)
         return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }

@@ -61,6 +61,24 @@ struct VecOps<4> {
     static __device__ __forceinline__ T load_b(const float* b, int c) {
         return make_float4(__ldg(b + c), __ldg(b + c + 1), __ldg(b + c + 2), __ldg(b + c + 3));
     }
+    static __device__ __forceinline__ void scale_shift(const Epilogue& e, int c, T& s, T& t) {
+        bn_scale_shift(e, c, s.x, t.x);
+        bn_scale_shift(e, c + 1, s.y, t.y);
+        bn_scale_shift(e, c + 2, s.z, t.z);
+        bn_scale_shift(e, c + 3, s.w, t.w);
+    }
+    static __device__ __forceinline__ T mul(const T& a, const T& b) {
+        return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+    }
+    static __device__ __forceinline__ T fma(const T& a, const T& b, const T& c, int) {
+        return make_float4(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y), fmaf(a.z, b.z, c.z),
+                           fmaf(a.w, b.w, c.w));
+    }
+    template <int ACT>
+    static __device__ __forceinline__ T act(const T& u) {
+        return make_float4(activate<ACT>(u.x), activate<ACT>(u.y), activate<ACT>(u.z),
+                           activate<ACT>(u.w));
+    }
 };
 
 template <>
@@ -77,6 +95,17 @@ struct VecOps<1> {
         return float(w[o]);
     }
     static __device__ __forceinline__ T load_b(const float* b, int c) { return __ldg(b + c); }
+    static __device__ __forceinline__ void scale_shift(const Epilogue& e, int c, T& s, T& t) {
+        bn_scale_shift(e, c, s, t);
+    }
+    static __device__ __forceinline__ T mul(const T& a, const T& b) { return a * b; }
+    static __device__ __forceinline__ T fma(const T& a, const T& b, const T& c, int) {
+        return fmaf(a, b, c);
+    }
+    template <int ACT>
+    static __device__ __forceinline__ T act(const T& u) {
+        return activate<ACT>(u);
+    }
 };
 
 struct Args {
@@ -91,6 +120,7 @@ struct Args {
     int org_y, org_x;
     FastDiv tiles_c, tiles_x, tiles_y;
     int ntiles;
+    Epilogue epi;  // used by the EPI instantiations only
 };
 
 // NO: output staging buffers for the TMA-store epilogue (0 = results are
@@ -182,10 +212,13 @@ __device__ __forceinline__ Tile decode_tile(int t, const Args& a) {
     return T;
 }
 
-template <class K>
+// EPI: kNoEpilogue, or the activation of the fused batch-norm / activation
+// epilogue of the forward.
+template <class K, int EPI>
 __global__ void __launch_bounds__(K::NT, K::MINB)
     tiled_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
                  const Args a) {
+    static_assert(EPI == kNoEpilogue || !K::TR, "the epilogue belongs to the forward");
     using VO = VecOps<K::VEC>;
     using V = typename VO::T;
     constexpr int CV = K::CV;
@@ -255,6 +288,16 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     V wr[K::KH][K::KW];
     V bias = VO::zero();
     int cur_cb = -1;
+    // the value stored for one output: acc (+ bias) (-> activation)
+    auto finish = [&](const V& acc) -> V {
+        if constexpr (K::TR) {
+            return acc;
+        } else if constexpr (EPI != kNoEpilogue) {
+            return VO::template act<EPI>(VO::add(acc, bias));
+        } else {
+            return VO::add(acc, bias);
+        }
+    };
 
     int k = 0;
     for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
@@ -289,6 +332,18 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] = VO::zero();
             }
             if (!K::TR && a.b != nullptr && live) bias = VO::load_b(a.b, c);
+            if constexpr (EPI != kNoEpilogue) {
+                // fold the normalisation into the filter and the bias
+                if (live) {
+                    V sc, sh;
+                    VO::scale_shift(a.epi, c, sc, sh);
+#pragma unroll
+                    for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] = VO::mul(wr[kh][kw], sc);
+                    bias = VO::fma(bias, sc, sh, 0);
+                }
+            }
         }
 
         const bool ok = mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag);
@@ -358,7 +413,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
             for (int j = 0; j < K::THT; ++j)
 #pragma unroll
                 for (int i = 0; i < K::TWT; ++i)
-                    o[(j * K::TW + i) * CV] = K::TR ? acc[j][i] : VO::add(acc[j][i], bias);
+                    o[(j * K::TW + i) * CV] = finish(acc[j][i]);
             fence_proxy_async_smem();
             if (named_barrier_or(1, K::NCT, !ok)) {
                 if (tid == 0) {
@@ -382,8 +437,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 for (int i = 0; i < K::TWT; ++i) {
                     const int wo = wo0 + i;
                     if (wo < 0 || wo >= a.Wout) continue;
-                    const V v = K::TR ? acc[j][i] : VO::add(acc[j][i], bias);
-                    VO::store(base + j * row_pitch + int64_t(i) * a.C, v);
+                    VO::store(base + j * row_pitch + int64_t(i) * a.C, finish(acc[j][i]));
                 }
             }
         }
@@ -422,12 +476,22 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     a.tiles_x = make_fastdiv(static_cast<int>(tx));
     a.tiles_c = make_fastdiv(static_cast<int>(tc));
     a.ntiles = static_cast<int>(nt);
+    a.epi = tr ? Epilogue{} : p.epi;
     if (dry_run) return DW_OK;
 
-    static LaunchCache cache;
+    // the epilogue instantiations exist for the forward only
+    const int ev = epilogue_variant(a.epi);
+    void (*kern)(CUtensorMap, CUtensorMap, Args) = tiled_kernel<K, kNoEpilogue>;
+    if constexpr (!K::TR) {
+        if (ev == DW_ACT_NONE) kern = tiled_kernel<K, DW_ACT_NONE>;
+        if (ev == DW_ACT_RELU) kern = tiled_kernel<K, DW_ACT_RELU>;
+        if (ev == DW_ACT_RELU6) kern = tiled_kernel<K, DW_ACT_RELU6>;
+        if (ev == DW_ACT_SILU) kern = tiled_kernel<K, DW_ACT_SILU>;
+    }
+    static LaunchCache cache[5];
     const int dev = current_device();
-    const int occ = prepare_kernel(reinterpret_cast<const void*>(&tiled_kernel<K>), K::NT,
-                                   K::SMEM, cache, dev);
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(kern), K::NT, K::SMEM,
+                                   cache[ev + 1], dev);
     if (occ < 1) return DW_ERR_CUDA;
 
     const int64_t Hin = tr ? p.Ho : p.H, Win = tr ? p.Wo : p.W;
@@ -458,8 +522,8 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
     if (grid >= tc) grid -= grid % tc;
     if (grid > nt) grid = nt;
     if (grid < 1) grid = 1;
-    if (launch_pdl(tiled_kernel<K>, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM,
-                   stream, map, omap, a) != cudaSuccess)
+    if (launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream, map,
+                   omap, a) != cudaSuccess)
         return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }

@@ -23,12 +23,14 @@ DW_NHWC, DW_NCHW = 0, 1
 DW_F32, DW_F16 = 0, 1
 DW_PAD_EXPLICIT, DW_PAD_SAME = 0, 1
 DW_ALGO_AUTO, DW_ALGO_DIRECT, DW_ALGO_TILED = 0, 1, 2
+DW_ACT_NONE, DW_ACT_RELU, DW_ACT_RELU6, DW_ACT_SILU = 0, 1, 2, 3
 
 _LAYOUTS = {"nhwc": DW_NHWC, "nchw": DW_NCHW}
 _ALGOS = {"auto": DW_ALGO_AUTO, "direct": DW_ALGO_DIRECT, "tiled": DW_ALGO_TILED}
+_ACTS = {"none": DW_ACT_NONE, "relu": DW_ACT_RELU, "relu6": DW_ACT_RELU6, "silu": DW_ACT_SILU}
 
 # Every symbol include/dwconv2d.h declares.
-EXPORTS = ("dwconv2d_out_shape", "dwconv2d_resolved_pads", "dwconv2d_fwd",
+EXPORTS = ("dwconv2d_out_shape", "dwconv2d_resolved_pads", "dwconv2d_fwd", "dwconv2d_fwd_bn_act",
            "dwconv2d_bwd_input", "dwconv2d_bwd_weight", "dwconv2d_bwd_weight_workspace_size",
            "dwconv2d_bwd_weight_noalloc",
            "dwconv2d_query_algo", "dwconv2d_take_device_error", "dwconv2d_status_string",
@@ -77,6 +79,9 @@ def lib() -> ctypes.CDLL:
     L.dwconv2d_fwd.argtypes = [P(DwDesc), vp, vp, vp, vp, vp]
     L.dwconv2d_bwd_input.restype = i32
     L.dwconv2d_bwd_input.argtypes = [P(DwDesc), vp, vp, vp, vp]
+    L.dwconv2d_fwd_bn_act.restype = i32
+    L.dwconv2d_fwd_bn_act.argtypes = [P(DwDesc), vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32,
+                                      vp, vp]
     L.dwconv2d_bwd_weight.restype = i32
     L.dwconv2d_bwd_weight.argtypes = [P(DwDesc), vp, vp, vp, vp, vp, ctypes.c_uint64, vp]
     L.dwconv2d_bwd_weight_noalloc.restype = i32
@@ -173,6 +178,17 @@ def fwd_raw(desc: DwDesc, x_ptr: int, w_ptr: int, b_ptr: Optional[int], y_ptr: i
     """dwconv2d_fwd on raw device pointers; returns the status."""
     return int(lib().dwconv2d_fwd(ctypes.byref(desc), x_ptr, w_ptr, b_ptr or None, y_ptr,
                                   stream or None))
+
+
+def fwd_bn_act_raw(desc: DwDesc, x_ptr: int, w_ptr: int, b_ptr: Optional[int],
+                   bn_ptrs: Optional[Sequence[int]], eps: float, act: int, y_ptr: int,
+                   stream: int) -> int:
+    """dwconv2d_fwd_bn_act on raw device pointers (bn_ptrs = gamma, beta, mean,
+    var or None); returns the status."""
+    g, be, mu, var = bn_ptrs if bn_ptrs is not None else (None, None, None, None)
+    return int(lib().dwconv2d_fwd_bn_act(ctypes.byref(desc), x_ptr, w_ptr, b_ptr or None,
+                                         g or None, be or None, mu or None, var or None,
+                                         float(eps), int(act), y_ptr, stream or None))
 
 
 def bwd_input_raw(desc: DwDesc, dy_ptr: int, w_ptr: int, dx_ptr: int, stream: int) -> int:
@@ -273,6 +289,56 @@ def dwconv2d_fwd(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tensor] = N
                      out.data_ptr(), _stream_ptr(x.device))
     if st != DW_OK:
         raise DwError(st, "dwconv2d_fwd")
+    return out
+
+
+def dwconv2d_fwd_bn_act(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tensor] = None,
+                        bn: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor,
+                                           torch.Tensor, float]] = None,
+                        act: str = "none", *, stride=1, dilation=1, padding="same",
+                        layout: str = "nhwc", algo: str = "auto",
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = act(batch_norm(depthwise conv2d forward(x) + b)) in one kernel.
+
+    bn = (gamma, beta, running_mean, running_var, eps) with [C] float32 CUDA
+    tensors (inference-mode statistics) or None; act in "none", "relu",
+    "relu6", "silu".  Other arguments as for dwconv2d_fwd."""
+    _check_act(x, "x")
+    if layout.lower() == "nhwc":
+        N, H, W, C = x.shape
+    else:
+        N, C, H, W = x.shape
+    w, kH, kW, wt = _weights(w, C, x.device)
+    if b is not None:
+        if b.device != x.device or b.dtype != torch.float32 or b.numel() != C or not b.is_contiguous():
+            raise ValueError("b must be a contiguous float32 CUDA tensor of C elements")
+    ptrs, eps = None, 0.0
+    if bn is not None:
+        if len(bn) != 5:
+            raise ValueError("bn must be (gamma, beta, running_mean, running_var, eps)")
+        for t in bn[:4]:
+            if (not isinstance(t, torch.Tensor) or t.device != x.device or t.dtype != torch.float32
+                    or t.numel() != C or not t.is_contiguous()):
+                raise ValueError("batch-norm statistics must be contiguous float32 CUDA tensors of C elements")
+        ptrs = [t.data_ptr() for t in bn[:4]]
+        eps = float(bn[4])
+    if act not in _ACTS:
+        raise ValueError(f"act must be one of {sorted(_ACTS)}")
+    desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
+                     layout=layout, wtype=wt, algo=algo)
+    Ho, Wo = dwconv2d_out_shape(desc)
+    shape = (N, Ho, Wo, C) if desc.layout == DW_NHWC else (N, C, Ho, Wo)
+    if out is None:
+        out = torch.empty(shape, device=x.device, dtype=torch.float32)
+    else:
+        _check_act(out, "out")
+        if tuple(out.shape) != shape or out.device != x.device:
+            raise ValueError(f"out must have shape {shape} on {x.device}")
+    with torch.cuda.device(x.device):
+        st = fwd_bn_act_raw(desc, x.data_ptr(), w.data_ptr(), None if b is None else b.data_ptr(),
+                            ptrs, eps, _ACTS[act], out.data_ptr(), _stream_ptr(x.device))
+    if st != DW_OK:
+        raise DwError(st, "dwconv2d_fwd_bn_act")
     return out
 
 

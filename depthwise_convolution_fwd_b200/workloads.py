@@ -77,6 +77,20 @@ def make_inputs(case: Case, out_hw: Tuple[int, int]) -> Dict[str, Optional[torch
     return {"x": x, "w": w, "w32": w, "b": b, "dy": dy}
 
 
+def make_bn(C: int, seed: int, eps: float = 1e-5) -> Tuple[torch.Tensor, torch.Tensor,
+                                                          torch.Tensor, torch.Tensor, float]:
+    """Inference-mode batch-norm statistics for the fused epilogue (CPU float32):
+    gamma ~ U(0.25, 1.75), beta ~ U(-0.5, 0.5), running mean ~ U(-0.2, 0.2),
+    running var ~ U(0.25, 2), drawn in that order from their own seed."""
+    gen = torch.Generator().manual_seed(seed)
+    u = lambda lo, hi: torch.rand((C,), generator=gen, dtype=torch.float32) * (hi - lo) + lo
+    gamma = u(0.25, 1.75)
+    beta = u(-0.5, 0.5)
+    mean = u(-0.2, 0.2)
+    var = u(0.25, 2.0)
+    return gamma, beta, mean, var, eps
+
+
 # ------------------------------------------------------------ configurations
 
 def tiny() -> List[Case]:

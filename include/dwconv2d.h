@@ -83,6 +83,9 @@ enum { DW_NHWC = 0, DW_NCHW = 1 };                 /* dw_desc_t.layout   */
 enum { DW_F32 = 0, DW_F16 = 1 };                   /* dw_desc_t.wtype    */
 enum { DW_PAD_EXPLICIT = 0, DW_PAD_SAME = 1 };     /* dw_desc_t.pad_mode */
 enum { DW_ALGO_AUTO = 0, DW_ALGO_DIRECT = 1, DW_ALGO_TILED = 2 }; /* .algo */
+/* activation of dwconv2d_fwd_bn_act: identity, max(u,0), min(max(u,0),6),
+ * u / (1 + exp(-u)) */
+enum { DW_ACT_NONE = 0, DW_ACT_RELU = 1, DW_ACT_RELU6 = 2, DW_ACT_SILU = 3 };
 
 /*
  * Problem descriptor.  N,H,W,C are the INPUT (x / dx) extents.  pad_mode
@@ -129,6 +132,35 @@ DW_API dw_status_t dwconv2d_resolved_pads(const dw_desc_t* desc, int32_t pads[4]
  */
 DW_API dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const float* x, const void* w,
                          const float* b, float* y, void* stream);
+
+/*
+ * Forward with a fused epilogue: y = act(BN(depthwise(x; w) + b)), where BN
+ * is inference-mode batch normalisation with per-channel running statistics,
+ *   BN(z)[c] = gamma[c] * (z - mean[c]) / sqrt(var[c] + eps) + beta[c],
+ * and act one of DW_ACT_*.  The normalisation and the activation are applied
+ * to each output in registers before its single store, so y is written once
+ * and never re-read.
+ *   x, w, b, y: as for dwconv2d_fwd.
+ *   gamma, beta, mean, var: [C] float32 each, read only; either all four are
+ *       given or all four are NULL (then BN is the identity and only the
+ *       activation is applied).
+ *   eps: finite, >= 0.
+ *   act: DW_ACT_NONE .. DW_ACT_SILU.
+ * Each channel's scale gamma/sqrt(var+eps) and shift beta - mean*scale are
+ * formed in float32 (IEEE division and square root) and applied as one fused
+ * multiply-add (the tiled kernels fold them into the filter and bias they
+ * hold: scale*w and scale*b + shift); silu is u / (1 + expf(-u)) with a fast
+ * division (a few ulp).  y must not overlap any input (DW_ERR_ALIAS);
+ * a mixed set of NULL statistics, a negative or non-finite eps or an unknown
+ * act is DW_ERR_INVALID_ARG.
+ * Page: LeanMlir Depthwise, the section on the MLIR lowering, which names a
+ * depthwise conv + batch-norm emitter; the pages do not spell the
+ * normalisation out, and the inference-mode form above is the reading taken.
+ */
+DW_API dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const float* x, const void* w,
+                                       const float* b, const float* gamma, const float* beta,
+                                       const float* mean, const float* var, float eps,
+                                       int32_t act, float* y, void* stream);
 
 /*
  * Input gradient: dx = J^T dy for the forward of `desc` (bias plays no part).

@@ -189,3 +189,31 @@ def test_weight_gradient_host_checks(lib):
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 1, 31, layout="nchw"), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 7, 3, 3), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 3, 3, dilation=2), 2, x, dy, dwp) == D
+
+
+def test_fused_epilogue_host_checks(lib):
+    desc = dw.make_desc(1, 8, 8, 4, 3, 3)  # y: 1 KiB
+    base = 1 << 40
+    x, w, y = base, base + (1 << 20), base + (2 << 20)
+    st = [base + (3 << 20) + 4096 * i for i in range(4)]
+    R = dw.fwd_bn_act_raw
+    # mixed NULL statistics, bad eps, unknown activation: rejected before launch
+    for k in range(4):
+        part = list(st)
+        part[k] = 0
+        assert R(desc, x, w, None, part, 1e-5, dw.DW_ACT_RELU, y, 0) == dw.DW_ERR_INVALID_ARG
+    for eps in (-1e-3, float("nan"), float("inf")):
+        assert R(desc, x, w, None, st, eps, dw.DW_ACT_NONE, y, 0) == dw.DW_ERR_INVALID_ARG
+    for act in (-1, 4):
+        assert R(desc, x, w, None, st, 1e-5, act, y, 0) == dw.DW_ERR_INVALID_ARG
+    # y over any statistics array, or over x / w / b
+    for k in range(4):
+        part = list(st)
+        part[k] = y + 512
+        assert R(desc, x, w, None, part, 1e-5, dw.DW_ACT_NONE, y, 0) == dw.DW_ERR_ALIAS
+    assert R(desc, x, w, None, st, 1e-5, dw.DW_ACT_NONE, x + 8, 0) == dw.DW_ERR_ALIAS
+    assert R(desc, x, w, y + 16, st, 1e-5, dw.DW_ACT_NONE, y, 0) == dw.DW_ERR_ALIAS
+    # invalid descriptor
+    bad = dw.make_desc(1, 8, 8, 4, 3, 3)
+    bad.kH = 0
+    assert R(bad, x, w, None, st, 1e-5, dw.DW_ACT_NONE, y, 0) == dw.DW_ERR_INVALID_ARG
