@@ -145,6 +145,41 @@ __global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restri
 }
 
 // part[(j*T + t)*C + c] summed over j in order.
+// Fixed-order sum of `count` float64 terms by one warp: lane l adds terms
+// l, l+32, ... in order, then a fixed butterfly combines the lanes; lane 0's
+// value is the result (the same bits on every run).  32 independent load
+// streams hide the latency a single thread's sequential sum would expose.
+template <class F>
+__device__ __forceinline__ double warp_ordered_sum(int64_t count, F&& term) {
+    const int lane = threadIdx.x & 31;
+    double s = 0.0;
+#pragma unroll 4
+    for (int64_t j = lane; j < count; j += 32) s += term(j);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
+// Writes item i = t*C + c of the result: dW[c, t] for t < T-1, db[c] for t = T-1.
+__device__ __forceinline__ void store_item(float* dw, float* db, int64_t C, int T, int64_t c,
+                                           int t, double v) {
+    if (t == T - 1) {
+        if (db) db[c] = float(v);
+    } else {
+        dw[c * (T - 1) + t] = float(v);
+    }
+}
+
+// Finalize kernels: one warp per (channel, tap) item, grid-stride over items.
+constexpr int kFinalizeThreads = 256;
+
+int64_t finalize_blocks(int64_t items, int sms) {
+    int64_t fb = (items * 32 + kFinalizeThreads - 1) / kFinalizeThreads;
+    const int64_t cap = int64_t(sms) * 8;
+    if (fb > cap) fb = cap;
+    return fb < 1 ? 1 : fb;
+}
+
 __global__ void __launch_bounds__(256) finalize_direct(const double* __restrict__ part,
                                                        float* __restrict__ dw,
                                                        float* __restrict__ db, int64_t C, int T,
@@ -152,17 +187,13 @@ __global__ void __launch_bounds__(256) finalize_direct(const double* __restrict_
     grid_dependency_wait();
     allow_dependents();
     const int64_t n = C * T;
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32; i < n; i += warps) {
         const int64_t c = i % C;
         const int t = int(i / C);
-        double s = 0.0;
-        for (int64_t j = 0; j < chunks; ++j) s += part[(j * T + t) * C + c];
-        if (t == T - 1) {
-            if (db) db[c] = float(s);
-        } else {
-            dw[c * (T - 1) + t] = float(s);
-        }
+        const double s =
+            warp_ordered_sum(chunks, [&](int64_t j) { return part[(j * T + t) * C + c]; });
+        if ((threadIdx.x & 31) == 0) store_item(dw, db, C, T, c, t, s);
     }
 }
 
@@ -365,18 +396,17 @@ __global__ void __launch_bounds__(256) finalize_tiled(const double* __restrict__
     grid_dependency_wait();
     allow_dependents();
     const int64_t n = int64_t(C) * T;
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32; i < n; i += warps) {
         const int c = int(i % C);
         const int t = int(i / C);
         const int cb = c / kLanes, lane = c % kLanes;
-        double s = 0.0;
-        for (int b = cb; b < G; b += tiles_c) s += part[(int64_t(b) * T + t) * kLanes + lane];
-        if (t == T - 1) {
-            if (db) db[c] = float(s);
-        } else {
-            dw[int64_t(c) * (T - 1) + t] = float(s);
-        }
+        // the CTAs of channel block cb are cb, cb + tiles_c, ... < G
+        const int64_t count = (G - cb + tiles_c - 1) / tiles_c;
+        const double s = warp_ordered_sum(count, [&](int64_t j) {
+            return part[((cb + j * tiles_c) * T + t) * kLanes + lane];
+        });
+        if ((threadIdx.x & 31) == 0) store_item(dw, db, C, T, c, t, s);
     }
 }
 
@@ -427,9 +457,8 @@ dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, flo
                         : launch_pdl(partial_direct_nchw, dim3(unsigned(blocks)), dim3(256), 0,
                                      stream, x, dy, part, a);
     if (e != cudaSuccess) return DW_ERR_CUDA;
-    int64_t fb = (p.C * a.T + 255) / 256;
-    if (fb > cap) fb = cap;
-    e = launch_pdl(finalize_direct, dim3(unsigned(fb)), dim3(256), 0, stream,
+    const int64_t fb = finalize_blocks(p.C * a.T, sm_count(dev));
+    e = launch_pdl(finalize_direct, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
                    static_cast<const double*>(part), dw, db, int64_t(p.C), a.T, a.chunks);
     if (e != cudaSuccess) return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
@@ -488,10 +517,8 @@ dw_status_t launch_tiled(const Problem& p, const float* x, const float* dy, floa
     if (launch_pdl(partial_tiled<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap, gmap,
                    a) != cudaSuccess)
         return DW_ERR_CUDA;
-    int64_t fb = (p.C * K::T + 255) / 256;
-    const int64_t cap = int64_t(sm_count(dev)) * 8;
-    if (fb > cap) fb = cap;
-    if (launch_pdl(finalize_tiled, dim3(unsigned(fb)), dim3(256), 0, stream,
+    const int64_t fb = finalize_blocks(p.C * K::T, sm_count(dev));
+    if (launch_pdl(finalize_tiled, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
                    static_cast<const double*>(a.part), dw, db, int(p.C), K::T, int(tc),
                    int(G)) != cudaSuccess)
         return DW_ERR_CUDA;
@@ -693,18 +720,265 @@ __global__ void __launch_bounds__(256) finalize_tiled_nchw(const double* __restr
     grid_dependency_wait();
     allow_dependents();
     const int64_t n_items = int64_t(C) * T;
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_items;
-         i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32; i < n_items;
+         i += warps) {
         const int c = int(i % C);
         const int t = int(i / C);
-        double s = 0.0;
-        for (int n = 0; n < N; ++n)
-            for (int b = 0; b < bands; ++b) s += part[((int64_t(n) * C + c) * bands + b) * T + t];
-        if (t == T - 1) {
-            if (db) db[c] = float(s);
-        } else {
-            dw[int64_t(c) * (T - 1) + t] = float(s);
+        // term j = (n, band) = (j / bands, j % bands)
+        const double s = warp_ordered_sum(int64_t(N) * bands, [&](int64_t j) {
+            const int64_t n = j / bands, b = j - n * bands;
+            return part[((n * C + c) * bands + b) * T + t];
+        });
+        if ((threadIdx.x & 31) == 0) store_item(dw, db, C, T, c, t, s);
+    }
+}
+
+// ------------------------------------- tiled kernel, NCHW, 1 x kW filters --
+// With kH = 1 every row is an independent 1-D correlation.  A unit is (block
+// of n, group of 8 channels): consumer warp w owns channel cg*8 + w and walks,
+// for every n of the block, every output row and every 128-column strip; one
+// pipeline stage holds that row of the 8 channels' planes (a 4-D TMA box of
+// one row by 8 channels, zero-filled past C).  Lanes run along W with 4
+// outputs each, the kW taps at compile-time offsets of a register window.
+// Each warp's float64 sums over its unit become one partial per
+// (n block, tap, channel), laid out as the direct partials are, so the same
+// fixed-order finalize sums the n blocks.
+
+struct RArgs {
+    double* part;
+    int32_t* err;
+    int N, C, Ho, pt, pl;
+    int tiles_x;   // 128-column strips per row
+    int cgroups;   // groups of 8 channels
+    int nper;      // n per block
+    int units;     // n blocks * cgroups
+};
+
+template <int KW_, int REM_, int NS_>
+struct RCfg {
+    static constexpr int KW = KW_, REM = REM_, NS = NS_;
+    static constexpr int T = KW + 1;
+    static constexpr int NCW = 8;  // consumer warps = channels per unit
+    static constexpr int NT = NCW * 32 + 32;
+    static constexpr int TW = 128;
+    static constexpr int IWB = (REM + TW + KW - 1 + 3) / 4 * 4;
+    static constexpr int NV = (REM + 3 + KW - 1) / 4 + 1;  // float4 per window
+    static constexpr int XBYTES = IWB * NCW * 4;
+    static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;
+    static constexpr int GBYTES = TW * NCW * 4;
+    static constexpr int STAGE_BYTES = XPITCH + GBYTES;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(2 * NS) * 8 + 16;
+    static_assert(GBYTES % 128 == 0, "TMA shared-memory alignment");
+    static_assert(IWB <= 256, "TMA box limit");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    partial_rows_nchw(const __grid_constant__ CUtensorMap xmap,
+                      const __grid_constant__ CUtensorMap gmap, const RArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_BYTES);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
         }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    allow_dependents();
+
+    if (warp == K::NCW) {
+        if (lane == 0) {
+            prefetch_tensor_map(&xmap);
+            prefetch_tensor_map(&gmap);
+            int k = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < a.units && ok; u += G) {
+                const int nb = u / a.cgroups, cg = u - nb * a.cgroups;
+                const int n0 = nb * a.nper;
+                const int n1 = a.N - n0 < a.nper ? a.N : n0 + a.nper;
+                for (int n = n0; n < n1 && ok; ++n)
+                    for (int h = 0; h < a.Ho && ok; ++h)
+                        for (int tx = 0; tx < a.tiles_x; ++tx, ++k) {
+                            const int s = k % K::NS;
+                            if (k >= K::NS &&
+                                !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
+                            mbar_arrive_expect_tx(&full[s], K::XBYTES + K::GBYTES);
+                            tma_load_4d(st, &xmap, &full[s], tx * K::TW - a.pl - K::REM, h - a.pt,
+                                        cg * K::NCW, n);
+                            tma_load_4d(st + K::XPITCH, &gmap, &full[s], tx * K::TW, h,
+                                        cg * K::NCW, n);
+                        }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
+        }
+        return;
+    }
+
+    int k = 0;
+    bool failed = false;
+    for (int u = blockIdx.x; u < a.units && !failed; u += G) {
+        const int nb = u / a.cgroups, cg = u - nb * a.cgroups;
+        const int n0 = nb * a.nper;
+        const int n1 = a.N - n0 < a.nper ? a.N : n0 + a.nper;
+        const int c = cg * K::NCW + warp;
+        double acc64[K::T];
+#pragma unroll
+        for (int t = 0; t < K::T; ++t) acc64[t] = 0.0;
+        const int ntile = (n1 - n0) * a.Ho * a.tiles_x;
+        for (int i = 0; i < ntile; ++i, ++k) {
+            const int s = k % K::NS;
+            if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                }
+                failed = true;
+                break;
+            }
+            const unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
+            const float4* xw = reinterpret_cast<const float4*>(st) + warp * (K::IWB / 4) + lane;
+            const float4 gf =
+                reinterpret_cast<const float4*>(st + K::XPITCH)[warp * (K::TW / 4) + lane];
+            const float g[4] = {gf.x, gf.y, gf.z, gf.w};
+            float v[4 * K::NV];
+#pragma unroll
+            for (int q = 0; q < K::NV; ++q) {
+                const float4 f = xw[q];
+                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+            }
+            float acc[K::KW];
+#pragma unroll
+            for (int kw = 0; kw < K::KW; ++kw) {
+                float t0 = g[0] * v[K::REM + kw];
+                t0 = fmaf(g[1], v[K::REM + 1 + kw], t0);
+                t0 = fmaf(g[2], v[K::REM + 2 + kw], t0);
+                acc[kw] = fmaf(g[3], v[K::REM + 3 + kw], t0);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+            for (int kw = 0; kw < K::KW; ++kw) acc64[kw] += double(acc[kw]);
+            acc64[K::T - 1] += double((g[0] + g[1]) + (g[2] + g[3]));
+        }
+        // the warp's sums over the unit, lanes combined in a fixed order
+#pragma unroll
+        for (int t = 0; t < K::T; ++t) {
+            double v = acc64[t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0 && c < a.C) a.part[(int64_t(nb) * K::T + t) * a.C + c] = v;
+        }
+    }
+}
+
+// n blocks of the rows kernel: enough units to cover the SMs twice over (a
+// fixed count, so the workspace depends on the problem alone).
+constexpr int kRowsUnits = 296;
+
+int rows_nblocks(const Problem& p, int& nper) {
+    const int64_t cgroups = (p.C + 7) / 8;
+    int64_t nb = (kRowsUnits + cgroups - 1) / cgroups;
+    if (nb > p.N) nb = p.N;
+    if (nb < 1) nb = 1;
+    nper = int((p.N + nb - 1) / nb);
+    return int((p.N + nper - 1) / nper);
+}
+
+size_t rows_nchw_workspace(const Problem& p) {
+    if (p.layout != DW_NCHW || p.kH != 1) return 0;
+    int nper;
+    const int nb = rows_nblocks(p, nper);
+    return size_t(nb) * size_t(p.kW + 1) * size_t(p.C) * sizeof(double);
+}
+
+template <class K>
+dw_status_t launch_rows_nchw(const Problem& p, const float* x, const float* dy, float* dw,
+                             float* db, void* ws, cudaStream_t stream, int32_t* err,
+                             bool dry_run) {
+    RArgs a;
+    a.part = static_cast<double*>(ws);
+    a.err = err;
+    a.N = int(p.N);
+    a.C = int(p.C);
+    a.Ho = int(p.Ho);
+    a.pt = p.pt;
+    a.pl = p.pl;
+    const int64_t tx = (p.Wo + K::TW - 1) / K::TW;
+    const int64_t cgroups = (p.C + K::NCW - 1) / K::NCW;
+    int nper;
+    const int nb = rows_nblocks(p, nper);
+    const int64_t units = int64_t(nb) * cgroups;
+    if (units >= INT_MAX || tx >= INT_MAX || int64_t(nper) * p.Ho * tx >= INT_MAX)
+        return DW_ERR_UNSUPPORTED;
+    a.tiles_x = int(tx);
+    a.cgroups = int(cgroups);
+    a.nper = nper;
+    a.units = int(units);
+    if (dry_run) return DW_OK;
+
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&partial_rows_nchw<K>), K::NT,
+                                   K::SMEM, cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+    int64_t G = int64_t(sm_count(dev)) * occ;
+    if (G > units) G = units;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap xmap, gmap;
+    const cuuint64_t xd[4] = {cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t xs[3] = {cuuint64_t(p.W) * 4, cuuint64_t(p.W * p.H) * 4,
+                              cuuint64_t(p.W * p.H * p.C) * 4};
+    const cuuint32_t xbox[4] = {K::IWB, 1, K::NCW, 1};
+    const cuuint64_t gd[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * 4, cuuint64_t(p.Wo * p.Ho) * 4,
+                              cuuint64_t(p.Wo * p.Ho * p.C) * 4};
+    const cuuint32_t gbox[4] = {K::TW, 1, K::NCW, 1};
+    if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
+                          xbox, estr) != CUDA_SUCCESS ||
+        encode_tensor_map(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(dy), gd, gs,
+                          gbox, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+    if (launch_pdl(partial_rows_nchw<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap,
+                   gmap, a) != cudaSuccess)
+        return DW_ERR_CUDA;
+    const int64_t fb = finalize_blocks(p.C * K::T, sm_count(dev));
+    if (launch_pdl(finalize_direct, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
+                   static_cast<const double*>(a.part), dw, db, int64_t(p.C), K::T,
+                   int64_t(nb)) != cudaSuccess)
+        return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+template <int KW, int NS>
+dw_status_t launch_rows_rem(const Problem& p, const float* x, const float* dy, float* dw,
+                            float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    switch (((-p.pl) % 4 + 4) % 4) {
+        case 0: return launch_rows_nchw<RCfg<KW, 0, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 1: return launch_rows_nchw<RCfg<KW, 1, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 2: return launch_rows_nchw<RCfg<KW, 2, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        default: return launch_rows_nchw<RCfg<KW, 3, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
     }
 }
 
@@ -774,10 +1048,8 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     if (launch_pdl(partial_tiled_nchw<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap,
                    gmap, a) != cudaSuccess)
         return DW_ERR_CUDA;
-    int64_t fb = (p.C * K::T + 255) / 256;
-    const int64_t cap = int64_t(sm_count(dev)) * 8;
-    if (fb > cap) fb = cap;
-    if (launch_pdl(finalize_tiled_nchw, dim3(unsigned(fb)), dim3(256), 0, stream,
+    const int64_t fb = finalize_blocks(p.C * K::T, sm_count(dev));
+    if (launch_pdl(finalize_tiled_nchw, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
                    static_cast<const double*>(a.part), dw, db, int(p.N), int(p.C), K::T,
                    a.bands) != cudaSuccess)
         return DW_ERR_CUDA;
@@ -804,6 +1076,14 @@ dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, f
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
         return DW_ERR_UNSUPPORTED;
     if (p.N >= INT_MAX || p.C >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    if (p.kH == 1) {
+        if (p.kW == 3) return launch_rows_rem<3, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 5) return launch_rows_rem<5, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 7) return launch_rows_rem<7, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 15) return launch_rows_rem<15, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 31) return launch_rows_rem<31, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        return DW_ERR_UNSUPPORTED;
+    }
     //                                                    KH KW THT WY NS
     if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
     if (p.kH == 5 && p.kW == 5) return launch_nchw_rem<5, 5, 4, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
@@ -842,7 +1122,9 @@ dw_status_t tiled_pick(const Problem& p, const float* x, const float* dy, float*
 size_t bwd_weight_workspace_bytes(const Problem& p) {
     size_t m = wgrad::direct_workspace(p);
     const size_t b = wgrad::tiled_workspace(p), c = wgrad::tiled_nchw_workspace(p);
+    const size_t r = wgrad::rows_nchw_workspace(p);
     if (b > m) m = b;
+    if (r > m) m = r;
     if (c > m) m = c;
     return m;
 }

@@ -80,6 +80,12 @@ TILED = [
     Case("w_nchw_7x7", 2, 33, 28, 9, 7, 7, layout="nchw", seed=86),
     Case("w_nchw_wide", 1, 70, 300, 3, 3, 3, layout="nchw", seed=87),
     Case("w_nchw_planes", 8, 20, 24, 64, 3, 3, layout="nchw", seed=88),
+    # NCHW, 1 x kW: rows kernel (channel groups of 8 with a ragged last group)
+    Case("w_nchw_1x31", 3, 2, 300, 20, 1, 31, act="normal", layout="nchw", seed=89),
+    Case("w_nchw_1x15_pad", 2, 3, 64, 11, 1, 15, padding=(1, 0, 6, 8), act="normal",
+         layout="nchw", seed=90),
+    Case("w_nchw_1x3", 2, 5, 40, 9, 1, 3, padding=(0, 0, 0, 2), layout="nchw", seed=91),
+    Case("w_nchw_1x7", 5, 1, 44, 16, 1, 7, padding=(0, 0, 5, 1), layout="nchw", seed=92),
 ]
 
 
@@ -105,6 +111,12 @@ def test_repeatable_bit_for_bit():
 @pytest.mark.parametrize("layout", ["nhwc", "nchw"])
 def test_large_full_size(layout):
     case = [c for c in wl.large() if c.H == 512 and c.layout == layout][0]
+    check(case, algos=("auto",))
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+def test_conformer_full_size(layout):
+    case = [c for c in wl.conformer() if c.W == 512 and c.layout == layout][0]
     check(case, algos=("auto",))
 
 
