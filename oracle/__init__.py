@@ -133,8 +133,9 @@ def resolve_pads(H, W, kH, kW, stride=1, dilation=1, padding="same"):
     raise ValueError(f"bad padding {padding!r}")
 
 
-def problem(shape, kH, kW, stride=1, dilation=1, padding="same", layout="nhwc"):
-    """int64[15] problem vector from an activation shape in `layout` order."""
+def problem(shape, kH, kW, stride=1, dilation=1, padding="same", layout="nhwc", multiplier=1):
+    """int64[16] problem vector from the input activation shape in `layout`
+    order; `multiplier` M output channels per input channel (C*M in all)."""
     layout = layout.lower()
     if layout == "nhwc":
         N, H, W, C = shape
@@ -145,15 +146,21 @@ def problem(shape, kH, kW, stride=1, dilation=1, padding="same", layout="nhwc"):
     sh, sw = _pair(stride)
     dh, dw = _pair(dilation)
     pt, pb, pl, pr = resolve_pads(H, W, kH, kW, stride, dilation, padding)
+    if int(multiplier) < 1:
+        raise ValueError("multiplier must be >= 1")
     return np.array([N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr,
-                     LAYOUTS[layout]], dtype=np.int64)
+                     LAYOUTS[layout], int(multiplier)], dtype=np.int64)
+
+
+def out_channels(prob) -> int:
+    return int(prob[3]) * int(prob[15])
 
 
 def out_shape(prob) -> tuple[int, ...]:
-    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, lay = (int(v) for v in prob)
+    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, lay, M = (int(v) for v in prob)
     Ho = out_extent(H, kH, sh, dh, pt, pb)
     Wo = out_extent(W, kW, sw, dw, pl, pr)
-    return (N, Ho, Wo, C) if lay == 0 else (N, C, Ho, Wo)
+    return (N, Ho, Wo, C * M) if lay == 0 else (N, C * M, Ho, Wo)
 
 
 def in_shape(prob) -> tuple[int, ...]:
@@ -170,9 +177,8 @@ def _ptr(a, ty=ctypes.c_double):
 
 
 def _weights(w, prob):
-    C, kH, kW = int(prob[3]), int(prob[4]), int(prob[5])
-    w = _f64(w).reshape(C, kH, kW)
-    return w
+    kH, kW = int(prob[4]), int(prob[5])
+    return _f64(w).reshape(out_channels(prob), kH, kW)
 
 
 def fwd(prob, x, w, b=None):
@@ -180,7 +186,7 @@ def fwd(prob, x, w, b=None):
     prob = np.ascontiguousarray(prob, dtype=np.int64)
     x = _f64(x).reshape(in_shape(prob))
     w = _weights(w, prob)
-    bb = None if b is None else _f64(b).reshape(int(prob[3]))
+    bb = None if b is None else _f64(b).reshape(out_channels(prob))
     y = np.empty(out_shape(prob), dtype=np.float64)
     _load().dwo_fwd(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(w),
                     None if bb is None else _ptr(bb), _ptr(y))
@@ -202,7 +208,7 @@ def fwd_at(prob, x, w, b, flat_idx):
     prob = np.ascontiguousarray(prob, dtype=np.int64)
     x = _f64(x).reshape(in_shape(prob))
     w = _weights(w, prob)
-    bb = None if b is None else _f64(b).reshape(int(prob[3]))
+    bb = None if b is None else _f64(b).reshape(out_channels(prob))
     idx = np.ascontiguousarray(flat_idx, dtype=np.int64)
     out = np.empty(idx.shape[0], dtype=np.float64)
     _load().dwo_fwd_at(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(w),
@@ -224,11 +230,11 @@ def bwd_input_at(prob, dy, w, flat_idx):
 
 
 def bwd_weight(prob, x, dy):
-    """(dW [C,kH,kW], db [C]): weight and bias gradients of the forward (float64)."""
+    """(dW [C*M,kH,kW], db [C*M]): weight and bias gradients of the forward (float64)."""
     prob = np.ascontiguousarray(prob, dtype=np.int64)
     x = _f64(x).reshape(in_shape(prob))
     dy = _f64(dy).reshape(out_shape(prob))
-    C, kH, kW = int(prob[3]), int(prob[4]), int(prob[5])
+    C, kH, kW = out_channels(prob), int(prob[4]), int(prob[5])
     dw = np.empty((C, kH, kW), dtype=np.float64)
     db = np.empty(C, dtype=np.float64)
     _load().dwo_bwd_weight(_ptr(prob, ctypes.c_int64), _ptr(x), _ptr(dy), _ptr(dw), _ptr(db))
@@ -259,7 +265,7 @@ def bn_act(prob, z, flat_idx=None, bn=None, act="none"):
         np.ascontiguousarray(flat_idx, dtype=np.int64)
     ch = np.ascontiguousarray(channel_of(prob, idx), dtype=np.int64)
     out = np.empty_like(flat)
-    C = int(prob[3])
+    C = out_channels(prob)
     if bn is None:
         g = be = mu = var = None
         eps = 0.0

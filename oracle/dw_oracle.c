@@ -37,10 +37,21 @@
  *     (Ho = ceil(H/s), total pad = max((Ho-1)s + d(k-1) + 1 - H, 0), the odd
  *     half at the bottom/right), which reproduces the odd-position decimation.
  *
- * Problem vector `p` (int64[15]):
- *   N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, layout
- *   layout 0 = NHWC (c innermost), 1 = NCHW (w innermost).
- * Weights are W[c][kh][kw] row-major.  Bias may be NULL (treated as 0).
+ *   - channel multiplier M (page "Incorrect stableHLO for grouped convolution
+ *     gradient", the Reactant.jl issue: a 3x3 conv from 4 to 8 channels with
+ *     groups = 4): C input channels, C*M output channels, output channel
+ *     o = c*M + j (j < M) reads only input channel c = o / M through its own
+ *     filter W[o] - a grouped convolution with one input channel per group.
+ *     The forward, input gradient (dx[c] sums over the M output channels of
+ *     c) and weight gradient (dW[o] pairs dy[o] with x[o / M]) follow from
+ *     the same index map.  M = 1 is the plain depthwise convolution.
+ *
+ * Problem vector `p` (int64[16]):
+ *   N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, layout, M
+ *   layout 0 = NHWC (c innermost), 1 = NCHW (w innermost); C counts the
+ *   input channels, y and dy have C*M.
+ * Weights are W[o][kh][kw] row-major, o < C*M.  Bias (C*M) may be NULL
+ * (treated as 0).
  */
 #include <stddef.h>
 #include <stdint.h>
@@ -51,7 +62,7 @@
 #endif
 
 enum { P_N, P_H, P_W, P_C, P_KH, P_KW, P_SH, P_SW, P_DH, P_DW,
-       P_PT, P_PB, P_PL, P_PR, P_LAYOUT, P_COUNT };
+       P_PT, P_PB, P_PL, P_PR, P_LAYOUT, P_MULT, P_COUNT };
 
 /* Number of output positions along one axis: the largest o with
  * o*s + (k-1)*d - lo <= in - 1 + hi, plus one (0 if none). */
@@ -81,12 +92,15 @@ int dwo_num_threads(void) {
 #endif
 }
 
+/* Flat index of element (n, c, h, w) of a tensor with Cx channels and
+ * extents Hx, Wx, in the problem's layout. */
 static int64_t act_index(const int64_t* p, int64_t n, int64_t c, int64_t h,
-                         int64_t w, int64_t Hx, int64_t Wx) {
-    int64_t C = p[P_C];
-    if (p[P_LAYOUT] == 0) return ((n * Hx + h) * Wx + w) * C + c;
-    return ((n * C + c) * Hx + h) * Wx + w;
+                         int64_t w, int64_t Cx, int64_t Hx, int64_t Wx) {
+    if (p[P_LAYOUT] == 0) return ((n * Hx + h) * Wx + w) * Cx + c;
+    return ((n * Cx + c) * Hx + h) * Wx + w;
 }
+
+static int64_t out_c(const int64_t* p) { return p[P_C] * p[P_MULT]; }
 
 static int64_t out_h(const int64_t* p) {
     return dwo_out_extent(p[P_H], p[P_KH], p[P_SH], p[P_DH], p[P_PT], p[P_PB]);
@@ -95,11 +109,12 @@ static int64_t out_w(const int64_t* p) {
     return dwo_out_extent(p[P_W], p[P_KW], p[P_SW], p[P_DW], p[P_PL], p[P_PR]);
 }
 
-/* One forward output value, straight from the definition. */
+/* One forward output value (output channel o), straight from the definition. */
 static double fwd_one(const int64_t* p, const double* x, const double* wt,
-                      const double* b, int64_t n, int64_t c, int64_t ho,
+                      const double* b, int64_t n, int64_t o, int64_t ho,
                       int64_t wo) {
     int64_t H = p[P_H], W = p[P_W], kH = p[P_KH], kW = p[P_KW];
+    int64_t c = o / p[P_MULT];  /* the one input channel output o reads */
     double acc = 0.0;
     for (int64_t kh = 0; kh < kH; ++kh) {
         for (int64_t kw = 0; kw < kW; ++kw) {
@@ -107,60 +122,60 @@ static double fwd_one(const int64_t* p, const double* x, const double* wt,
             int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];
             double xv = 0.0;
             if (hi >= 0 && hi < H && wi >= 0 && wi < W)
-                xv = x[act_index(p, n, c, hi, wi, H, W)];
-            acc += xv * wt[(c * kH + kh) * kW + kw];
+                xv = x[act_index(p, n, c, hi, wi, p[P_C], H, W)];
+            acc += xv * wt[(o * kH + kh) * kW + kw];
         }
     }
-    return acc + (b ? b[c] : 0.0);
+    return acc + (b ? b[o] : 0.0);
 }
 
 void dwo_fwd(const int64_t* p, const double* x, const double* wt,
              const double* b, double* y) {
-    int64_t N = p[P_N], C = p[P_C];
+    int64_t N = p[P_N], Co = out_c(p);
     int64_t Ho = out_h(p), Wo = out_w(p);
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t n = 0; n < N; ++n)
-        for (int64_t c = 0; c < C; ++c)
+        for (int64_t o = 0; o < Co; ++o)
             for (int64_t ho = 0; ho < Ho; ++ho)
                 for (int64_t wo = 0; wo < Wo; ++wo)
-                    y[act_index(p, n, c, ho, wo, Ho, Wo)] =
-                        fwd_one(p, x, wt, b, n, c, ho, wo);
+                    y[act_index(p, n, o, ho, wo, Co, Ho, Wo)] =
+                        fwd_one(p, x, wt, b, n, o, ho, wo);
 }
 
 /* Transpose of the forward's linear part applied to dy: every output
- * cotangent dy[n,ho,wo,c] is sent back to each input position the forward
- * read for that output, weighted by the tap that read it.  Positions the
- * forward never reads receive 0. */
+ * cotangent dy[n,ho,wo,o] is sent back to each input position the forward
+ * read for that output (input channel o / M), weighted by the tap that read
+ * it.  Positions the forward never reads receive 0. */
 void dwo_bwd_input(const int64_t* p, const double* dy, const double* wt,
                    double* dx) {
     int64_t N = p[P_N], C = p[P_C], H = p[P_H], W = p[P_W];
-    int64_t kH = p[P_KH], kW = p[P_KW];
+    int64_t kH = p[P_KH], kW = p[P_KW], M = p[P_MULT], Co = out_c(p);
     int64_t Ho = out_h(p), Wo = out_w(p);
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t c = 0; c < C; ++c) {
             for (int64_t hi = 0; hi < H; ++hi)
                 for (int64_t wi = 0; wi < W; ++wi)
-                    dx[act_index(p, n, c, hi, wi, H, W)] = 0.0;
-            for (int64_t ho = 0; ho < Ho; ++ho)
-                for (int64_t wo = 0; wo < Wo; ++wo) {
-                    double g = dy[act_index(p, n, c, ho, wo, Ho, Wo)];
-                    for (int64_t kh = 0; kh < kH; ++kh)
-                        for (int64_t kw = 0; kw < kW; ++kw) {
-                            int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];
-                            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];
-                            if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;
-                            dx[act_index(p, n, c, hi, wi, H, W)] +=
-                                g * wt[(c * kH + kh) * kW + kw];
-                        }
-                }
+                    dx[act_index(p, n, c, hi, wi, C, H, W)] = 0.0;
+            for (int64_t o = c * M; o < (c + 1) * M; ++o)
+                for (int64_t ho = 0; ho < Ho; ++ho)
+                    for (int64_t wo = 0; wo < Wo; ++wo) {
+                        double g = dy[act_index(p, n, o, ho, wo, Co, Ho, Wo)];
+                        for (int64_t kh = 0; kh < kH; ++kh)
+                            for (int64_t kw = 0; kw < kW; ++kw) {
+                                int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];
+                                int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];
+                                if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;
+                                dx[act_index(p, n, c, hi, wi, C, H, W)] +=
+                                    g * wt[(o * kH + kh) * kW + kw];
+                            }
+                    }
         }
     }
 }
 
-static void decode(const int64_t* p, int64_t flat, int64_t Hx, int64_t Wx,
+static void decode(const int64_t* p, int64_t flat, int64_t C, int64_t Hx, int64_t Wx,
                    int64_t* n, int64_t* c, int64_t* h, int64_t* w) {
-    int64_t C = p[P_C];
     if (p[P_LAYOUT] == 0) {
         *c = flat % C; flat /= C;
         *w = flat % Wx; flat /= Wx;
@@ -179,9 +194,9 @@ void dwo_fwd_at(const int64_t* p, const double* x, const double* wt,
     int64_t Ho = out_h(p), Wo = out_w(p);
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < count; ++i) {
-        int64_t n, c, ho, wo;
-        decode(p, flat[i], Ho, Wo, &n, &c, &ho, &wo);
-        out[i] = fwd_one(p, x, wt, b, n, c, ho, wo);
+        int64_t n, o, ho, wo;
+        decode(p, flat[i], out_c(p), Ho, Wo, &n, &o, &ho, &wo);
+        out[i] = fwd_one(p, x, wt, b, n, o, ho, wo);
     }
 }
 
@@ -199,7 +214,7 @@ void dwo_bwd_input_at(const int64_t* p, const double* dy, const double* wt,
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < count; ++i) {
         int64_t n, c, hi, wi;
-        decode(p, flat[i], H, W, &n, &c, &hi, &wi);
+        decode(p, flat[i], p[P_C], H, W, &n, &c, &hi, &wi);
         int64_t rh = hi + p[P_PT], rw = wi + p[P_PL];
         /* ho*sh in [rh - (kH-1)dh, rh]  ->  ho in [ho_lo, ho_hi] */
         int64_t ho_lo = rh - (kH - 1) * dh;
@@ -211,20 +226,22 @@ void dwo_bwd_input_at(const int64_t* p, const double* dy, const double* wt,
         int64_t wo_hi = rw < 0 ? -1 : rw / sw;
         if (wo_hi > Wo - 1) wo_hi = Wo - 1;
         double acc = 0.0;
-        for (int64_t ho = ho_lo; ho <= ho_hi; ++ho) {
-            int64_t kh_nat = rh - ho * sh;          /* = kh * dh */
-            if (kh_nat % dh != 0) continue;
-            int64_t kh = kh_nat / dh;
-            if (kh < 0 || kh >= kH) continue;
-            for (int64_t wo = wo_lo; wo <= wo_hi; ++wo) {
-                int64_t kw_nat = rw - wo * sw;      /* = kw * dw */
-                if (kw_nat % dw != 0) continue;
-                int64_t kw = kw_nat / dw;
-                if (kw < 0 || kw >= kW) continue;
-                acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *
-                       wt[(c * kH + kh) * kW + kw];
+        /* every output channel of input channel c: o = c*M .. c*M + M-1 */
+        for (int64_t o = c * p[P_MULT]; o < (c + 1) * p[P_MULT]; ++o)
+            for (int64_t ho = ho_lo; ho <= ho_hi; ++ho) {
+                int64_t kh_nat = rh - ho * sh;          /* = kh * dh */
+                if (kh_nat % dh != 0) continue;
+                int64_t kh = kh_nat / dh;
+                if (kh < 0 || kh >= kH) continue;
+                for (int64_t wo = wo_lo; wo <= wo_hi; ++wo) {
+                    int64_t kw_nat = rw - wo * sw;      /* = kw * dw */
+                    if (kw_nat % dw != 0) continue;
+                    int64_t kw = kw_nat / dw;
+                    if (kw < 0 || kw >= kW) continue;
+                    acc += dy[act_index(p, n, o, ho, wo, out_c(p), Ho, Wo)] *
+                           wt[(o * kH + kh) * kW + kw];
+                }
             }
-        }
         out[i] = acc;
     }
 }
@@ -235,10 +252,11 @@ void dwo_bwd_input_at(const int64_t* p, const double* dy, const double* wt,
 void dwo_bwd_weight(const int64_t* p, const double* x, const double* dy, double* dw,
                     double* db) {
     int64_t N = p[P_N], C = p[P_C], H = p[P_H], W = p[P_W];
-    int64_t kH = p[P_KH], kW = p[P_KW];
+    int64_t kH = p[P_KH], kW = p[P_KW], Co = out_c(p);
     int64_t Ho = out_h(p), Wo = out_w(p);
 #pragma omp parallel for schedule(static)
-    for (int64_t c = 0; c < C; ++c) {
+    for (int64_t o = 0; o < Co; ++o) {
+        int64_t c = o / p[P_MULT];  /* the input channel filter o reads */
         for (int64_t kh = 0; kh < kH; ++kh)
             for (int64_t kw = 0; kw < kW; ++kw) {
                 double acc = 0.0;
@@ -248,18 +266,18 @@ void dwo_bwd_weight(const int64_t* p, const double* x, const double* dy, double*
                             int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];
                             int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];
                             if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;
-                            acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *
-                                   x[act_index(p, n, c, hi, wi, H, W)];
+                            acc += dy[act_index(p, n, o, ho, wo, Co, Ho, Wo)] *
+                                   x[act_index(p, n, c, hi, wi, C, H, W)];
                         }
-                dw[(c * kH + kh) * kW + kw] = acc;
+                dw[(o * kH + kh) * kW + kw] = acc;
             }
         if (db) {
             double acc = 0.0;
             for (int64_t n = 0; n < N; ++n)
                 for (int64_t ho = 0; ho < Ho; ++ho)
                     for (int64_t wo = 0; wo < Wo; ++wo)
-                        acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)];
-            db[c] = acc;
+                        acc += dy[act_index(p, n, o, ho, wo, Co, Ho, Wo)];
+            db[o] = acc;
         }
     }
 }

@@ -20,29 +20,37 @@ from tests import test_oracle_pins as pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "dw_oracle.c")
 
 MUTANTS = {
-    "fwd_flipped_kernel": ("acc += xv * wt[(c * kH + kh) * kW + kw];",
-                           "acc += xv * wt[(c * kH + (kH - 1 - kh)) * kW + (kW - 1 - kw)];"),
+    "fwd_flipped_kernel": ("acc += xv * wt[(o * kH + kh) * kW + kw];",
+                           "acc += xv * wt[(o * kH + (kH - 1 - kh)) * kW + (kW - 1 - kw)];"),
     "fwd_pad_sign": ("int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];\n            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n            double xv",
                      "int64_t hi = ho * p[P_SH] + kh * p[P_DH] + p[P_PT];\n            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n            double xv"),
-    "fwd_dropped_bias": ("return acc + (b ? b[c] : 0.0);", "return acc;"),
+    "fwd_dropped_bias": ("return acc + (b ? b[o] : 0.0);", "return acc;"),
     "fwd_swapped_strides": ("int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];\n            int64_t wi = wo * p[P_SW]",
                             "int64_t hi = ho * p[P_SW] + kh * p[P_DH] - p[P_PT];\n            int64_t wi = wo * p[P_SH]"),
-    "fwd_transposed_taps": ("acc += xv * wt[(c * kH + kh) * kW + kw];",
-                            "acc += xv * wt[(c * kW + kw) * kH + kh];"),
-    "bwd_flipped_kernel": ("g * wt[(c * kH + kh) * kW + kw];",
-                           "g * wt[(c * kH + (kH - 1 - kh)) * kW + (kW - 1 - kw)];"),
-    "bwd_dropped_dilation": ("int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];\n                            int64_t wi",
-                             "int64_t hi = ho * p[P_SH] + kh - p[P_PT];\n                            int64_t wi"),
-    "bwd_wrong_pad_side": ("int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n                            if (hi < 0",
-                           "int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PR];\n                            if (hi < 0"),
+    "fwd_transposed_taps": ("acc += xv * wt[(o * kH + kh) * kW + kw];",
+                            "acc += xv * wt[(o * kW + kw) * kH + kh];"),
+    "bwd_flipped_kernel": ("g * wt[(o * kH + kh) * kW + kw];",
+                           "g * wt[(o * kH + (kH - 1 - kh)) * kW + (kW - 1 - kw)];"),
+    "bwd_dropped_dilation": ("int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];\n                                int64_t wi",
+                             "int64_t hi = ho * p[P_SH] + kh - p[P_PT];\n                                int64_t wi"),
+    "bwd_wrong_pad_side": ("int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n                                if (hi < 0",
+                           "int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PR];\n                                if (hi < 0"),
     "same_odd_half_on_top": ("*lo = total / 2;\n    *hi = total - *lo;", "*hi = total / 2;\n    *lo = total - *hi;"),
     "extent_off_by_one": ("return last_reach / s + 1;", "return last_reach / s;"),
     "bwd_at_no_divisibility": ("if (kh_nat % dh != 0) continue;", ""),
     "wgrad_pad_sign": ("int64_t hi = ho * p[P_SH] + kh * p[P_DH] - p[P_PT];\n                            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n                            if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;\n                            acc +=",
                        "int64_t hi = ho * p[P_SH] + kh * p[P_DH] + p[P_PT];\n                            int64_t wi = wo * p[P_SW] + kw * p[P_DW] - p[P_PL];\n                            if (hi < 0 || hi >= H || wi < 0 || wi >= W) continue;\n                            acc +="),
-    "wgrad_transposed_taps": ("dw[(c * kH + kh) * kW + kw] = acc;", "dw[(c * kW + kw) * kH + kh] = acc;"),
-    "bwd_at_channel_mix": ("acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *\n                       wt[(c * kH + kh) * kW + kw];",
-                           "acc += dy[act_index(p, n, c, ho, wo, Ho, Wo)] *\n                       wt[(((c + 1) % p[P_C]) * kH + kh) * kW + kw];"),
+    "wgrad_transposed_taps": ("dw[(o * kH + kh) * kW + kw] = acc;", "dw[(o * kW + kw) * kH + kh] = acc;"),
+    "bwd_at_channel_mix": ("acc += dy[act_index(p, n, o, ho, wo, out_c(p), Ho, Wo)] *\n                           wt[(o * kH + kh) * kW + kw];",
+                           "acc += dy[act_index(p, n, o, ho, wo, out_c(p), Ho, Wo)] *\n                           wt[(((o + 1) % out_c(p)) * kH + kh) * kW + kw];"),
+    "mult_fwd_input_channel": ("int64_t c = o / p[P_MULT];  /* the one input channel output o reads */",
+                               "int64_t c = o % p[P_C];"),
+    "mult_bwd_first_output_only": ("for (int64_t o = c * M; o < (c + 1) * M; ++o)",
+                                   "for (int64_t o = c * M; o < c * M + 1; ++o)"),
+    "mult_bwd_at_first_output_only": ("for (int64_t o = c * p[P_MULT]; o < (c + 1) * p[P_MULT]; ++o)",
+                                      "for (int64_t o = c * p[P_MULT]; o < c * p[P_MULT] + 1; ++o)"),
+    "mult_wgrad_input_channel": ("int64_t c = o / p[P_MULT];  /* the input channel filter o reads */",
+                                 "int64_t c = o % p[P_C];"),
     "bn_dropped_eps": ("(u - mean[c]) / sqrt(var[c] + eps)", "(u - mean[c]) / sqrt(var[c])"),
     "bn_mean_sign": ("(u - mean[c])", "(u + mean[c])"),
     "bn_channel_ignored": ("int64_t c = ch[i];", "int64_t c = 0;"),
@@ -83,6 +91,9 @@ def run_pin_subset():
         ("golden_wgrad", lambda: pins.test_golden_weight_gradient(None)),
         ("wgrad_linearity", lambda: pins.test_weight_gradient_linearity_identity(None)),
         ("golden_bn_act", lambda: [pins.test_golden_bn_act(None, l) for l in ("nhwc", "nchw")]),
+        ("golden_multiplier", lambda: [pins.test_golden_multiplier(None, l) for l in ("nhwc", "nchw")]),
+        ("torch_multiplier", lambda: pins.test_multiplier_gradients_equal_torch_autograd(None)),
+        ("torch_multiplier_fwd", lambda: pins.test_multiplier_equals_torch_grouped_conv(None, False)),
         ("torch_bn_act", lambda: pins.test_bn_act_equals_torch_batch_norm_and_activations(None)),
     ]
     for name, fn in checks:

@@ -149,20 +149,20 @@ def from_nchw(p, a):
 
 def torch_fwd(p, x, w, b, dense=False):
     """Library routine: torch conv2d in float64 on an explicitly padded input."""
-    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _ = (int(v) for v in p)
+    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _, M = (int(v) for v in p)
     xt = torch.from_numpy(np.ascontiguousarray(to_nchw(p, x)))
     xt = F.pad(xt, (pl, pr, pt, pb))
-    wt = torch.from_numpy(np.asarray(w, dtype=np.float64).reshape(C, 1, kH, kW))
+    wt = torch.from_numpy(np.asarray(w, dtype=np.float64).reshape(C * M, 1, kH, kW))
     if dense:
-        # block-diagonal dense kernel Wd[o,i] = delta_oi W[o]: a regular conv
-        wd = torch.zeros(C, C, kH, kW, dtype=torch.float64)
-        for c in range(C):
-            wd[c, c] = wt[c, 0]
+        # dense kernel Wd[o,i] = delta_{i, o // M} W[o]: a regular conv
+        wd = torch.zeros(C * M, C, kH, kW, dtype=torch.float64)
+        for o in range(C * M):
+            wd[o, o // M] = wt[o, 0]
         y = F.conv2d(xt, wd, None, (sh, sw), 0, (dh, dw), groups=1)
     else:
         y = F.conv2d(xt, wt, None, (sh, sw), 0, (dh, dw), groups=C)
     if b is not None:
-        y = y + torch.from_numpy(np.asarray(b, dtype=np.float64)).view(1, C, 1, 1)
+        y = y + torch.from_numpy(np.asarray(b, dtype=np.float64)).view(1, C * M, 1, 1)
     return from_nchw(p, y.numpy())
 
 
@@ -184,7 +184,7 @@ def test_bwd_equals_torch_autograd(oracle_mod):
         w = rng.standard_normal((int(p[3]), int(p[4]), int(p[5])))
         dy = rng.standard_normal(oracle.out_shape(p))
         xt = torch.from_numpy(x).requires_grad_(True)
-        N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _ = (int(v) for v in p)
+        N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _, _ = (int(v) for v in p)
         xn = xt.permute(0, 3, 1, 2) if layout == "nhwc" else xt
         yt = F.conv2d(F.pad(xn, (pl, pr, pt, pb)),
                       torch.from_numpy(w).view(C, 1, kH, kW), None,
@@ -230,7 +230,7 @@ def test_fwd_equals_block_diagonal_dense_conv_bruteforce(oracle_mod):
     """Depthwise == a regular conv (groups = 1) whose kernel is block-diagonal,
     == a grouped conv with feature_group_count = C."""
     for p, layout, rng in valid_cases(31, 25, max_hw=6, max_k=3, max_c=3, max_n=1):
-        N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _ = (int(v) for v in p)
+        N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _, _ = (int(v) for v in p)
         x = rng.standard_normal(oracle.in_shape(p))
         w = rng.standard_normal((C, kH, kW))
         xc = to_nchw(p, x)[0]
@@ -249,7 +249,7 @@ def bwd_direct_formula_full(p, dy, w):
     over ALL output positions (ho,wo), with the kernel offset reconstructed
     from hi + pt = ho*sh + kh*dh; a term counts only when that offset is a
     whole tap in [0,kH) x [0,kW)."""
-    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _ = (int(v) for v in p)
+    N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _, _ = (int(v) for v in p)
     dyc = to_nchw(p, dy)
     Ho, Wo = dyc.shape[2], dyc.shape[3]
     dx = np.zeros((N, C, H, W))
@@ -287,7 +287,7 @@ def test_bwd_equals_reversed_kernel_formula_stride1(oracle_mod):
         if min(oracle.out_shape(p)) <= 0:
             continue
         count += 1
-        N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _ = (int(v) for v in p)
+        N, H, W, C, kH, kW, sh, sw, dh, dw, pt, pb, pl, pr, _, _ = (int(v) for v in p)
         w = rng.standard_normal((C, kH, kW))
         dy = rng.standard_normal(oracle.out_shape(p))
         dyc = to_nchw(p, dy)
@@ -488,7 +488,7 @@ def test_golden_weight_gradient(oracle_mod):
 
 def test_weight_gradient_equals_torch_autograd(oracle_mod):
     for p, layout, rng in valid_cases(141, 50):
-        N, H, W, C, kH, kW, sh, sw, dh, dw_, pt, pb, pl, pr, _ = (int(v) for v in p)
+        N, H, W, C, kH, kW, sh, sw, dh, dw_, pt, pb, pl, pr, _, _ = (int(v) for v in p)
         x = rng.standard_normal(oracle.in_shape(p))
         dy = rng.standard_normal(oracle.out_shape(p))
         wt = torch.from_numpy(rng.standard_normal((C, 1, kH, kW))).requires_grad_(True)
@@ -602,3 +602,110 @@ def test_bn_act_constant_input_closed_form(oracle_mod, layout):
             want = {"none": u, "relu": max(u, 0.0), "relu6": min(max(u, 0.0), 6.0),
                     "silu": u / (1.0 + np.exp(-u))}[act]
             assert abs(y[c, 2, 2] - want) <= 1e-12 * max(1.0, abs(want)), (act, c)
+
+
+# ---------------------------------------------------- channel multiplier ---
+
+def mult_cases(seed, count, **kw):
+    """Random valid problems with a channel multiplier M in 2..4."""
+    out = []
+    for p, layout, rng in valid_cases(seed, count, **kw):
+        p = p.copy()
+        p[15] = int(rng.integers(2, 5))
+        out.append((p, layout, rng))
+    return out
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+def test_golden_multiplier(oracle_mod, layout):
+    g = load_golden("multiplier_2x.json")
+    shape = (1, g["H"], g["W"], g["C"]) if layout == "nhwc" else (1, g["C"], g["H"], g["W"])
+    p = oracle.problem(shape, g["kH"], g["kW"], 1, 1, tuple(g["pads"]), layout,
+                       multiplier=g["M"])
+    x = chw_to(layout, [g["x"]])
+    y = oracle.fwd(p, x, g["w"], g["b"])
+    assert np.array_equal(to_chw(layout, y), np.array(g["y"]))
+    dx = oracle.bwd_input(p, chw_to(layout, g["bwd"]["dy"]), g["w"])
+    assert np.array_equal(to_chw(layout, dx)[0], np.array(g["bwd"]["dx"]))
+    idx = np.arange(dx.size)
+    assert np.array_equal(oracle.bwd_input_at(p, chw_to(layout, g["bwd"]["dy"]), g["w"], idx),
+                          dx.reshape(-1))
+    dw, db = oracle.bwd_weight(p, x, chw_to(layout, g["wgrad"]["dy"]))
+    assert np.array_equal(dw, np.array(g["wgrad"]["dw"]))
+    assert np.array_equal(db, np.array(g["wgrad"]["db"]))
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_multiplier_equals_torch_grouped_conv(oracle_mod, dense):
+    # the library's grouped conv (groups = C, C*M output channels), float64
+    for p, layout, rng in mult_cases(171, 30):
+        Co = oracle.out_channels(p)
+        x = rng.standard_normal(oracle.in_shape(p))
+        w = rng.standard_normal((Co, int(p[4]), int(p[5])))
+        b = rng.standard_normal(Co)
+        np.testing.assert_allclose(oracle.fwd(p, x, w, b), torch_fwd(p, x, w, b, dense),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_multiplier_gradients_equal_torch_autograd(oracle_mod):
+    for p, layout, rng in mult_cases(181, 30):
+        N, H, W, C, kH, kW, sh, sw, dh, dw_, pt, pb, pl, pr, _, M = (int(v) for v in p)
+        x = rng.standard_normal(oracle.in_shape(p))
+        dy = rng.standard_normal(oracle.out_shape(p))
+        xt = torch.from_numpy(np.ascontiguousarray(to_nchw(p, x))).requires_grad_(True)
+        wt = torch.from_numpy(rng.standard_normal((C * M, 1, kH, kW))).requires_grad_(True)
+        bt = torch.from_numpy(rng.standard_normal(C * M)).requires_grad_(True)
+        y = F.conv2d(F.pad(xt, (pl, pr, pt, pb)), wt, bt, (sh, sw), 0, (dh, dw_), groups=C)
+        gx, gw, gb = torch.autograd.grad(y, (xt, wt, bt),
+                                         torch.from_numpy(np.ascontiguousarray(to_nchw(p, dy))))
+        w = wt.detach().numpy()[:, 0]
+        np.testing.assert_allclose(to_nchw(p, oracle.bwd_input(p, dy, w)), gx.numpy(),
+                                   rtol=1e-12, atol=1e-12)
+        dw, db = oracle.bwd_weight(p, x, dy)
+        np.testing.assert_allclose(dw, gw.numpy()[:, 0], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(db, gb.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_multiplier_is_depthwise_of_repeated_channels(oracle_mod):
+    """With M output channels per input channel, the forward equals the plain
+    depthwise forward of x with every channel repeated M times, and the input
+    gradient is that forward's input gradient summed over each channel's M
+    copies."""
+    for p, layout, rng in mult_cases(191, 30):
+        M = int(p[15])
+        x = rng.standard_normal(oracle.in_shape(p))
+        Co = oracle.out_channels(p)
+        w = rng.standard_normal((Co, int(p[4]), int(p[5])))
+        b = rng.standard_normal(Co)
+        dy = rng.standard_normal(oracle.out_shape(p))
+        axis = 3 if layout == "nhwc" else 1
+        x_rep = np.repeat(x, M, axis=axis)
+        p1 = oracle.problem(x_rep.shape, int(p[4]), int(p[5]), (int(p[6]), int(p[7])),
+                            (int(p[8]), int(p[9])), tuple(int(v) for v in p[10:14]), layout)
+        assert np.array_equal(oracle.fwd(p, x, w, b), oracle.fwd(p1, x_rep, w, b))
+        dx1 = oracle.bwd_input(p1, dy, w)
+        shape = list(dx1.shape)
+        shape[axis:axis + 1] = [shape[axis] // M, M]
+        np.testing.assert_allclose(oracle.bwd_input(p, dy, w),
+                                   dx1.reshape(shape).sum(axis=axis + 1), rtol=1e-13, atol=1e-13)
+        dw, db = oracle.bwd_weight(p, x, dy)
+        dw1, db1 = oracle.bwd_weight(p1, x_rep, dy)
+        np.testing.assert_allclose(dw, dw1, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(db, db1, rtol=1e-13, atol=1e-13)
+
+
+def test_multiplier_adjoint_identity(oracle_mod):
+    for p, layout, rng in mult_cases(201, 40, max_hw=10, max_k=4, max_c=3):
+        x = rng.standard_normal(oracle.in_shape(p))
+        w = rng.standard_normal((oracle.out_channels(p), int(p[4]), int(p[5])))
+        dy = rng.standard_normal(oracle.out_shape(p))
+        lhs = float(np.sum(dy * oracle.fwd(p, x, w)))
+        rhs = float(np.sum(oracle.bwd_input(p, dy, w) * x))
+        assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs)), (lhs, rhs)
+        idx = rng.integers(0, x.size, size=50)
+        np.testing.assert_allclose(oracle.bwd_input_at(p, dy, w, idx),
+                                   oracle.bwd_input(p, dy, w).reshape(-1)[idx],
+                                   rtol=1e-12, atol=1e-12)
+        oidx = rng.integers(0, dy.size, size=50)
+        np.testing.assert_allclose(oracle.fwd_at(p, x, w, None, oidx),
+                                   oracle.fwd(p, x, w).reshape(-1)[oidx], rtol=1e-12, atol=1e-12)
