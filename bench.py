@@ -65,21 +65,25 @@ def workload_cases(name):
             "Conformer-style 1-D: 16x1x512x512 1x31 SAME, NHWC and NCHW f32"
     if name == "tiny":
         return wl.tiny(), "Tiny: 1x8x8x4 3x3 SAME NHWC f32"
+    if name == "multiplier":
+        return [c for c in wl.multiplier() if c.H == 512], \
+            "Channel multiplier 2: 1x512x512x128 -> 256 channels 3x3 SAME, NHWC and NCHW f32"
     raise ValueError(name)
 
 
 def algorithmic_bytes(case, Ho, Wo, op):
     """Bytes one call must move at minimum: read the input once, write the
     output once, read the filters (and the bias for the forward)."""
+    Co = case.C * case.multiplier  # output channels
     n_in = case.N * case.C * case.H * case.W
-    n_out = case.N * case.C * Ho * Wo
-    wbytes = case.C * case.kH * case.kW * (2 if case.wtype == "f16" else 4)
+    n_out = case.N * Co * Ho * Wo
+    wbytes = Co * case.kH * case.kW * (2 if case.wtype == "f16" else 4)
     if op == "fwd":
-        return 4 * n_in + 4 * n_out + wbytes + (4 * case.C if case.bias else 0)
-    if op == "fused":  # forward + four [C] batch-norm statistics
-        return 4 * n_in + 4 * n_out + wbytes + (4 * case.C if case.bias else 0) + 16 * case.C
-    if op == "wgrad":  # read x and dy, write dW [C,kH,kW] and db [C] (f32)
-        return 4 * n_in + 4 * n_out + 4 * case.C * case.kH * case.kW + 4 * case.C
+        return 4 * n_in + 4 * n_out + wbytes + (4 * Co if case.bias else 0)
+    if op == "fused":  # forward + four [Co] batch-norm statistics
+        return 4 * n_in + 4 * n_out + wbytes + (4 * Co if case.bias else 0) + 16 * Co
+    if op == "wgrad":  # read x and dy, write dW [Co,kH,kW] and db [Co] (f32)
+        return 4 * n_in + 4 * n_out + 4 * Co * case.kH * case.kW + 4 * Co
     return 4 * n_out + 4 * n_in + wbytes
 
 
@@ -188,7 +192,7 @@ class Shape:
         self.case = case
         desc = dw.make_desc(case.N, case.H, case.W, case.C, case.kH, case.kW,
                             stride=case.stride, dilation=case.dilation, padding=case.padding,
-                            layout=case.layout, wtype=case.wtype)
+                            layout=case.layout, wtype=case.wtype, multiplier=case.multiplier)
         self.desc = desc
         self.Ho, self.Wo = dw.dwconv2d_out_shape(desc)
         self.host = make_inputs(case, (self.Ho, self.Wo))
@@ -210,11 +214,11 @@ class Shape:
         from depthwise_convolution_fwd_b200.workloads import make_bn
         c = self.case
         self.act = act
-        self.bn = [t.to(device) for t in make_bn(c.C, c.seed + 500)[:4]]
+        self.bn = [t.to(device) for t in make_bn(c.Co, c.seed + 500)[:4]]
         self.ws_bytes = dw.dwconv2d_bwd_weight_workspace_size(self.desc)
         self.ws = torch.empty(max(1, self.ws_bytes), dtype=torch.uint8, device=device)
-        self.dW = torch.empty(c.C * c.kH * c.kW, device=device)
-        self.db = torch.empty(c.C, device=device)
+        self.dW = torch.empty(c.Co * c.kH * c.kW, device=device)
+        self.db = torch.empty(c.Co, device=device)
         for op in ("fused", "wgrad"):
             self.bytes[op] = algorithmic_bytes(c, self.Ho, self.Wo, op)
 
@@ -432,7 +436,8 @@ def run_e2e(args, torch, dw, shapes, device, stream, world):
             y = dw.dwconv2d_fwd(x, w, b, stride=c.stride, dilation=c.dilation,
                                 padding=c.padding, layout=c.layout)
             dx = dw.dwconv2d_bwd_input(dy, w, (c.H, c.W), stride=c.stride, dilation=c.dilation,
-                                       padding=c.padding, layout=c.layout)
+                                       padding=c.padding, layout=c.layout,
+                                       multiplier=c.multiplier)
             outs["y"].copy_(y, non_blocking=True)
             outs["dx"].copy_(dx, non_blocking=True)
 
@@ -583,7 +588,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["mobilenet", "large", "conformer", "tiny"],
+    ap.add_argument("--workload", choices=["mobilenet", "large", "conformer", "tiny", "multiplier"],
                     default="mobilenet")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=8.0)

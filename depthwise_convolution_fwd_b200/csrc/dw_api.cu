@@ -128,6 +128,7 @@ static constexpr int64_t kMaxExtent = int64_t(1) << 30;
 static constexpr int kMaxKernel = 1 << 12;
 static constexpr int kMaxStrideDil = 1 << 12;
 static constexpr int kMaxPad = 1 << 20;
+static constexpr int kMaxMultiplier = 1 << 12;
 
 static dw_status_t resolve(const dw_desc_t* d, Problem* p) {
     if (!d) return DW_ERR_INVALID_ARG;
@@ -144,7 +145,11 @@ static dw_status_t resolve(const dw_desc_t* d, Problem* p) {
     if (d->layout != DW_NHWC && d->layout != DW_NCHW) return DW_ERR_INVALID_ARG;
     if (d->wtype != DW_F32 && d->wtype != DW_F16) return DW_ERR_INVALID_ARG;
     if (d->algo < DW_ALGO_AUTO || d->algo > DW_ALGO_TILED) return DW_ERR_INVALID_ARG;
+    if (d->multiplier < 0 || d->multiplier > kMaxMultiplier) return DW_ERR_INVALID_ARG;
     p->N = d->N; p->H = d->H; p->W = d->W; p->C = d->C;
+    p->M = d->multiplier == 0 ? 1 : d->multiplier;
+    p->Co = p->C * p->M;
+    if (p->Co > kMaxExtent) return DW_ERR_INVALID_ARG;
     p->kH = d->kH; p->kW = d->kW;
     p->sh = d->stride_h; p->sw = d->stride_w;
     p->dh = d->dil_h; p->dw = d->dil_w;
@@ -166,7 +171,7 @@ static dw_status_t resolve(const dw_desc_t* d, Problem* p) {
     p->Wo = out_extent(p->W, p->kW, p->sw, p->dw, p->pl, p->pr);
     if (p->Ho < 1 || p->Wo < 1) return DW_ERR_INVALID_ARG;
     // element counts must stay well inside int64
-    const double elems = double(p->N) * double(p->C) *
+    const double elems = double(p->N) * double(p->Co) *
                          double(p->H > p->Ho ? p->H : p->Ho) *
                          double(p->W > p->Wo ? p->W : p->Wo);
     if (elems > 9.0e15) return DW_ERR_INVALID_ARG;
@@ -188,15 +193,15 @@ struct Buffers {
 
 static dw_status_t check_buffers(const Problem& p, Op op, const Buffers& bf) {
     if (!bf.in || !bf.w || !bf.out) return DW_ERR_INVALID_ARG;
-    const size_t in_elems = size_t(p.N) * size_t(p.C) *
-                            (op == OP_FWD ? size_t(p.H) * size_t(p.W) : size_t(p.Ho) * size_t(p.Wo));
-    const size_t out_elems = size_t(p.N) * size_t(p.C) *
-                             (op == OP_FWD ? size_t(p.Ho) * size_t(p.Wo) : size_t(p.H) * size_t(p.W));
-    const size_t w_bytes = size_t(p.C) * size_t(p.kH) * size_t(p.kW) * (p.wtype == DW_F16 ? 2 : 4);
+    const size_t x_elems = size_t(p.N) * size_t(p.C) * size_t(p.H) * size_t(p.W);
+    const size_t y_elems = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo);
+    const size_t in_elems = op == OP_FWD ? x_elems : y_elems;
+    const size_t out_elems = op == OP_FWD ? y_elems : x_elems;
+    const size_t w_bytes = size_t(p.Co) * size_t(p.kH) * size_t(p.kW) * (p.wtype == DW_F16 ? 2 : 4);
     const size_t out_bytes = out_elems * 4;
     if (overlaps(bf.out, out_bytes, bf.in, in_elems * 4)) return DW_ERR_ALIAS;
     if (overlaps(bf.out, out_bytes, bf.w, w_bytes)) return DW_ERR_ALIAS;
-    if (op == OP_FWD && overlaps(bf.out, out_bytes, bf.b, size_t(p.C) * 4)) return DW_ERR_ALIAS;
+    if (op == OP_FWD && overlaps(bf.out, out_bytes, bf.b, size_t(p.Co) * 4)) return DW_ERR_ALIAS;
     return DW_OK;
 }
 
@@ -209,10 +214,10 @@ static dw_status_t run(const dw_desc_t* desc, Op op, const Buffers& bf, cudaStre
     if (st != DW_OK) return st;
     if (epi) {
         // every statistics array must stay clear of y
-        const size_t yb = size_t(p.N) * size_t(p.C) * size_t(p.Ho) * size_t(p.Wo) * 4;
+        const size_t yb = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo) * 4;
         const float* stats[4] = {epi->gamma, epi->beta, epi->mean, epi->var};
         for (const float* v : stats)
-            if (overlaps(bf.out, yb, v, size_t(p.C) * 4)) return DW_ERR_ALIAS;
+            if (overlaps(bf.out, yb, v, size_t(p.Co) * 4)) return DW_ERR_ALIAS;
         p.epi = *epi;
     }
     const int algo = desc->algo;
@@ -309,9 +314,9 @@ static dw_status_t run_bwd_weight(const dw_desc_t* desc, const float* x, const f
     if (!x || !dy || !dw || !ws) return DW_ERR_INVALID_ARG;
     if (ws_bytes < bwd_weight_workspace_bytes(p)) return DW_ERR_INVALID_ARG;
     const size_t xb = size_t(p.N) * size_t(p.C) * size_t(p.H) * size_t(p.W) * 4;
-    const size_t gb = size_t(p.N) * size_t(p.C) * size_t(p.Ho) * size_t(p.Wo) * 4;
-    const size_t wb = size_t(p.C) * size_t(p.kH) * size_t(p.kW) * 4;
-    const size_t bb = size_t(p.C) * 4;
+    const size_t gb = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo) * 4;
+    const size_t wb = size_t(p.Co) * size_t(p.kH) * size_t(p.kW) * 4;
+    const size_t bb = size_t(p.Co) * 4;
     const void* ins[2] = {x, dy};
     const size_t inb[2] = {xb, gb};
     void* outs[3] = {dw, db, ws};

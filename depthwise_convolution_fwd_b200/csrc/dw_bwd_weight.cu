@@ -40,6 +40,7 @@ constexpr int kFold = 16;           // direct kernels: float32 terms per float64
 
 struct DArgs {
     int64_t N, C, H, W, Ho, Wo;
+    int64_t M, Co;   // output channels per input channel, output channels
     int kH, kW, sh, sw, dh, dw, pt, pl;
     int T;           // taps + 1 (the last slot is the bias)
     int64_t P;       // output positions per channel = N*Ho*Wo
@@ -57,8 +58,9 @@ __global__ void __launch_bounds__(256) partial_direct_nhwc(const float* __restri
     allow_dependents();
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.items; i += stride) {
-        const int64_t c = i % a.C;
-        const int64_t r = i / a.C;
+        const int64_t o = i % a.Co;  // output channel; it reads input channel o / M
+        const int64_t c = o / a.M;
+        const int64_t r = i / a.Co;
         const int t = int(r % a.T);
         const int64_t j = r / a.T;
         const bool bias = t == a.T - 1;
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(256) partial_direct_nhwc(const float* __restri
         float part32 = 0.f;
         int cnt = 0;
         for (int64_t pp = p0; pp < p1; ++pp) {
-            const float g = __ldg(dy + ((n * a.Ho + ho) * a.Wo + wo) * a.C + c);
+            const float g = __ldg(dy + ((n * a.Ho + ho) * a.Wo + wo) * a.Co + o);
             if (bias) {
                 part32 += g;
             } else {
@@ -108,8 +110,9 @@ __global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restri
     const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < a.items;
          i += warps) {
-        const int64_t c = i % a.C;
-        const int64_t r = i / a.C;
+        const int64_t o = i % a.Co;  // output channel; it reads input channel o / M
+        const int64_t c = o / a.M;
+        const int64_t r = i / a.Co;
         const int t = int(r % a.T);
         const int64_t j = r / a.T;
         const bool bias = t == a.T - 1;
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restri
         for (int64_t pp = p0 + lane; pp < p1; pp += 32) {
             const int64_t wo = pp % a.Wo, q = pp / a.Wo;
             const int64_t ho = q % a.Ho, n = q / a.Ho;
-            const float g = __ldg(dy + ((n * a.C + c) * a.Ho + ho) * a.Wo + wo);
+            const float g = __ldg(dy + ((n * a.Co + o) * a.Ho + ho) * a.Wo + wo);
             if (bias) {
                 part32 += g;
             } else {
@@ -144,7 +147,6 @@ __global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restri
     }
 }
 
-// part[(j*T + t)*C + c] summed over j in order.
 // Fixed-order sum of `count` float64 terms by one warp: lane l adds terms
 // l, l+32, ... in order, then a fixed butterfly combines the lanes; lane 0's
 // value is the result (the same bits on every run).  32 independent load
@@ -180,6 +182,7 @@ int64_t finalize_blocks(int64_t items, int sms) {
     return fb < 1 ? 1 : fb;
 }
 
+// part[(j*T + t)*C + c] summed over j (C: the output channels).
 __global__ void __launch_bounds__(256) finalize_direct(const double* __restrict__ part,
                                                        float* __restrict__ dw,
                                                        float* __restrict__ db, int64_t C, int T,
@@ -425,10 +428,11 @@ int64_t direct_chunks(const Problem& p, int64_t& chunk) {
 size_t direct_workspace(const Problem& p) {
     int64_t chunk;
     const int64_t chunks = direct_chunks(p, chunk);
-    return size_t(chunks) * size_t(p.kH * p.kW + 1) * size_t(p.C) * sizeof(double);
+    return size_t(chunks) * size_t(p.kH * p.kW + 1) * size_t(p.Co) * sizeof(double);
 }
 
 size_t tiled_workspace(const Problem& p) {
+    if (p.M != 1) return 0;
     const int64_t tc = (p.C + kLanes - 1) / kLanes;
     const int64_t g = tc >= kMaxTiledCtas ? tc : (kMaxTiledCtas / tc) * tc;
     return size_t(g) * size_t(p.kH * p.kW + 1) * kLanes * sizeof(double);
@@ -438,12 +442,13 @@ dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, flo
                           void* ws, cudaStream_t stream) {
     DArgs a;
     a.N = p.N; a.C = p.C; a.H = p.H; a.W = p.W; a.Ho = p.Ho; a.Wo = p.Wo;
+    a.M = p.M; a.Co = p.Co;
     a.kH = p.kH; a.kW = p.kW; a.sh = p.sh; a.sw = p.sw; a.dh = p.dh; a.dw = p.dw;
     a.pt = p.pt; a.pl = p.pl;
     a.T = p.kH * p.kW + 1;
     a.P = p.N * p.Ho * p.Wo;
     a.chunks = direct_chunks(p, a.chunk);
-    a.items = a.chunks * a.T * p.C;
+    a.items = a.chunks * a.T * p.Co;
     double* part = static_cast<double*>(ws);
     const int dev = current_device();
     const int64_t cap = int64_t(sm_count(dev)) * 8;
@@ -457,9 +462,9 @@ dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, flo
                         : launch_pdl(partial_direct_nchw, dim3(unsigned(blocks)), dim3(256), 0,
                                      stream, x, dy, part, a);
     if (e != cudaSuccess) return DW_ERR_CUDA;
-    const int64_t fb = finalize_blocks(p.C * a.T, sm_count(dev));
+    const int64_t fb = finalize_blocks(p.Co * a.T, sm_count(dev));
     e = launch_pdl(finalize_direct, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
-                   static_cast<const double*>(part), dw, db, int64_t(p.C), a.T, a.chunks);
+                   static_cast<const double*>(part), dw, db, int64_t(p.Co), a.T, a.chunks);
     if (e != cudaSuccess) return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
@@ -907,7 +912,7 @@ int rows_nblocks(const Problem& p, int& nper) {
 }
 
 size_t rows_nchw_workspace(const Problem& p) {
-    if (p.layout != DW_NCHW || p.kH != 1) return 0;
+    if (p.layout != DW_NCHW || p.kH != 1 || p.M != 1) return 0;
     int nper;
     const int nb = rows_nblocks(p, nper);
     return size_t(nb) * size_t(p.kW + 1) * size_t(p.C) * sizeof(double);
@@ -991,7 +996,7 @@ int nchw_bands_cap(const Problem& p) {
 }
 
 size_t tiled_nchw_workspace(const Problem& p) {
-    if (p.layout != DW_NCHW) return 0;
+    if (p.layout != DW_NCHW || p.M != 1) return 0;
     return size_t(p.N) * size_t(p.C) * size_t(nchw_bands_cap(p)) * size_t(p.kH * p.kW + 1) *
            sizeof(double);
 }
@@ -1101,6 +1106,7 @@ using W1x31 = WCfg<1, 31, 1, 1, 1, 8, 8, 1, 4>;
 
 dw_status_t tiled_pick(const Problem& p, const float* x, const float* dy, float* dw, float* db,
                        void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
     if (p.layout == DW_NCHW) return tiled_pick_nchw(p, x, dy, dw, db, ws, stream, err, dry_run);
     if (p.layout != DW_NHWC || p.C % 4 != 0) return DW_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)

@@ -28,9 +28,11 @@ struct Epilogue {
 
 // A resolved problem: everything the kernels need, pads already resolved.
 // H, W, C, N are the extents of x (forward input) / dx (gradient output);
-// Ho, Wo the extents of y / dy.
+// Ho, Wo the extents of y / dy, which have Co = C*M channels (M output
+// channels per input channel; output channel o reads input channel o / M).
 struct Problem {
     int64_t N, H, W, C, Ho, Wo;
+    int64_t M = 1, Co = 0;
     int kH, kW, sh, sw, dh, dw;
     int pt, pb, pl, pr;
     int layout;  // DW_NHWC / DW_NCHW

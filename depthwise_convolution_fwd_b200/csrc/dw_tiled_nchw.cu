@@ -654,6 +654,7 @@ dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const vo
                               bool dry_run) {
     using namespace nchw;
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
+    if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
     if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
     const int64_t Win = op == OP_FWD ? p.W : p.Wo;
     if (Win % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row stride: 16-byte multiple

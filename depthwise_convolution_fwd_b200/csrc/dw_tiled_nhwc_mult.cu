@@ -1,0 +1,41 @@
+// NHWC tiled kernels: forward with a channel multiplier M (page "Incorrect
+// stableHLO for grouped convolution gradient": a conv from C to C*M channels
+// with groups = C).  A tile holds 32 output channels and the 32/M input
+// channels they read; each lane's 4 output channels take their input values
+// from one (M >= 4) or two (M = 2) input channels of the staged window (the
+// kernel in dw_tiled_nhwc.cuh).  Other multipliers use the direct kernel.
+#include "dw_tiled_nhwc.cuh"
+
+namespace dw {
+namespace nhwc {
+
+// (KH KW S D TR | THT TWT WX WY NS | VEC NO MINB CB MULT)
+template <int M>
+using M33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4, 4, 0, 2, 32, M>;
+template <int M>
+using M33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4, 4, 0, 2, 32, M>;
+template <int M>
+using M55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 2, 4, 2, 1, 32, M>;
+
+template <int M>
+dw_status_t mult_pick(const Problem& p, const float* in, const void* w, const float* b,
+                      float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    const Op op = OP_FWD;
+    if (p.kH == 3 && p.kW == 3 && p.sh == 1 && p.dh == 1)
+        return launch<M33s1<M>>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && p.sh == 2 && p.dh == 1)
+        return launch<M33s2<M>>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 5 && p.kW == 5 && p.sh == 1 && p.dh == 1)
+        return launch<M55s1<M>>(p, op, in, w, b, out, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
+dw_status_t mult_launch(const Problem& p, const float* in, const void* w, const float* b,
+                        float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.M == 2) return mult_pick<2>(p, in, w, b, out, stream, err, dry_run);
+    if (p.M == 4) return mult_pick<4>(p, in, w, b, out, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
+}  // namespace nhwc
+}  // namespace dw

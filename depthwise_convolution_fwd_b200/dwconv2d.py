@@ -46,7 +46,8 @@ class DwDesc(ctypes.Structure):
                 ("pad_mode", ctypes.c_int32), ("pad_top", ctypes.c_int32),
                 ("pad_bottom", ctypes.c_int32), ("pad_left", ctypes.c_int32),
                 ("pad_right", ctypes.c_int32), ("layout", ctypes.c_int32),
-                ("wtype", ctypes.c_int32), ("algo", ctypes.c_int32)]
+                ("wtype", ctypes.c_int32), ("algo", ctypes.c_int32),
+                ("multiplier", ctypes.c_int32)]
 
 
 class DwError(RuntimeError):
@@ -112,9 +113,10 @@ def _pair(v) -> Tuple[int, int]:
 
 def make_desc(N: int, H: int, W: int, C: int, kH: int, kW: int, *, stride=1, dilation=1,
               padding: Union[str, int, Sequence[int]] = "same", layout: str = "nhwc",
-              wtype: str = "f32", algo: str = "auto") -> DwDesc:
+              wtype: str = "f32", algo: str = "auto", multiplier: int = 1) -> DwDesc:
     """Descriptor for input extents N,H,W,C.  padding: "same" (XLA rule), an
-    int, a (vertical, horizontal) pair or (top, bottom, left, right)."""
+    int, a (vertical, horizontal) pair or (top, bottom, left, right);
+    multiplier: output channels per input channel (C*multiplier in all)."""
     d = DwDesc()
     d.N, d.H, d.W, d.C = int(N), int(H), int(W), int(C)
     d.kH, d.kW = int(kH), int(kW)
@@ -136,6 +138,7 @@ def make_desc(N: int, H: int, W: int, C: int, kH: int, kW: int, *, stride=1, dil
     d.layout = _LAYOUTS[layout.lower()]
     d.wtype = {"f32": DW_F32, "f16": DW_F16}[wtype]
     d.algo = _ALGOS[algo]
+    d.multiplier = int(multiplier)
     return d
 
 
@@ -233,6 +236,7 @@ def _check_act(t: torch.Tensor, name: str):
 
 
 def _weights(w: torch.Tensor, C: int, device) -> Tuple[torch.Tensor, int, int, str]:
+    """w: [C,kH,kW] or [C,1,kH,kW] where C counts the OUTPUT channels."""
     if not isinstance(w, torch.Tensor) or w.device != device:
         raise TypeError("w must be a CUDA tensor on the activations' device")
     if w.dim() == 4:
@@ -256,6 +260,16 @@ def _weights(w: torch.Tensor, C: int, device) -> Tuple[torch.Tensor, int, int, s
     return w, kH, kW, wt
 
 
+def _out_channels(w: torch.Tensor, C: int) -> Tuple[int, int]:
+    """(C*M, M) from the filter's leading extent: M filters per input channel."""
+    if not isinstance(w, torch.Tensor) or w.dim() < 1:
+        raise TypeError("w must be a tensor")
+    Co = int(w.shape[0])
+    if Co < C or Co % C != 0:
+        raise ValueError(f"w must have C*multiplier rows for C={C}, got {Co}")
+    return Co, Co // C
+
+
 def _stream_ptr(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
@@ -270,14 +284,15 @@ def dwconv2d_fwd(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tensor] = N
         N, H, W, C = x.shape
     else:
         N, C, H, W = x.shape
-    w, kH, kW, wt = _weights(w, C, x.device)
+    Co, M = _out_channels(w, C)
+    w, kH, kW, wt = _weights(w, Co, x.device)
     if b is not None:
-        if b.device != x.device or b.dtype != torch.float32 or b.numel() != C or not b.is_contiguous():
-            raise ValueError("b must be a contiguous float32 CUDA tensor of C elements")
+        if b.device != x.device or b.dtype != torch.float32 or b.numel() != Co or not b.is_contiguous():
+            raise ValueError("b must be a contiguous float32 CUDA tensor of C*multiplier elements")
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, wtype=wt, algo=algo)
+                     layout=layout, wtype=wt, algo=algo, multiplier=M)
     Ho, Wo = dwconv2d_out_shape(desc)
-    shape = (N, Ho, Wo, C) if desc.layout == DW_NHWC else (N, C, Ho, Wo)
+    shape = (N, Ho, Wo, Co) if desc.layout == DW_NHWC else (N, Co, Ho, Wo)
     if out is None:
         out = torch.empty(shape, device=x.device, dtype=torch.float32)
     else:
@@ -308,26 +323,28 @@ def dwconv2d_fwd_bn_act(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tens
         N, H, W, C = x.shape
     else:
         N, C, H, W = x.shape
-    w, kH, kW, wt = _weights(w, C, x.device)
+    Co, M = _out_channels(w, C)
+    w, kH, kW, wt = _weights(w, Co, x.device)
     if b is not None:
-        if b.device != x.device or b.dtype != torch.float32 or b.numel() != C or not b.is_contiguous():
-            raise ValueError("b must be a contiguous float32 CUDA tensor of C elements")
+        if b.device != x.device or b.dtype != torch.float32 or b.numel() != Co or not b.is_contiguous():
+            raise ValueError("b must be a contiguous float32 CUDA tensor of C*multiplier elements")
     ptrs, eps = None, 0.0
     if bn is not None:
         if len(bn) != 5:
             raise ValueError("bn must be (gamma, beta, running_mean, running_var, eps)")
         for t in bn[:4]:
             if (not isinstance(t, torch.Tensor) or t.device != x.device or t.dtype != torch.float32
-                    or t.numel() != C or not t.is_contiguous()):
-                raise ValueError("batch-norm statistics must be contiguous float32 CUDA tensors of C elements")
+                    or t.numel() != Co or not t.is_contiguous()):
+                raise ValueError("batch-norm statistics must be contiguous float32 CUDA tensors of "
+                                 "C*multiplier elements")
         ptrs = [t.data_ptr() for t in bn[:4]]
         eps = float(bn[4])
     if act not in _ACTS:
         raise ValueError(f"act must be one of {sorted(_ACTS)}")
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, wtype=wt, algo=algo)
+                     layout=layout, wtype=wt, algo=algo, multiplier=M)
     Ho, Wo = dwconv2d_out_shape(desc)
-    shape = (N, Ho, Wo, C) if desc.layout == DW_NHWC else (N, C, Ho, Wo)
+    shape = (N, Ho, Wo, Co) if desc.layout == DW_NHWC else (N, Co, Ho, Wo)
     if out is None:
         out = torch.empty(shape, device=x.device, dtype=torch.float32)
     else:
@@ -344,18 +361,23 @@ def dwconv2d_fwd_bn_act(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tens
 
 def dwconv2d_bwd_input(dy: torch.Tensor, w: torch.Tensor, input_hw: Tuple[int, int], *,
                        stride=1, dilation=1, padding="same", layout: str = "nhwc",
-                       algo: str = "auto", out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                       algo: str = "auto", out: Optional[torch.Tensor] = None,
+                       multiplier: int = 1) -> torch.Tensor:
     """dx = input gradient of the forward whose input had spatial extents
-    input_hw = (H, W), given the output cotangent dy."""
+    input_hw = (H, W), given the output cotangent dy (C*multiplier channels)."""
     _check_act(dy, "dy")
     H, W = (int(v) for v in input_hw)
     if layout.lower() == "nhwc":
-        N, Ho, Wo, C = dy.shape
+        N, Ho, Wo, Co = dy.shape
     else:
-        N, C, Ho, Wo = dy.shape
-    w, kH, kW, wt = _weights(w, C, dy.device)
+        N, Co, Ho, Wo = dy.shape
+    M = int(multiplier)
+    if M < 1 or Co % M != 0:
+        raise ValueError(f"dy's {Co} channels are not a multiple of multiplier {M}")
+    C = Co // M
+    w, kH, kW, wt = _weights(w, Co, dy.device)
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, wtype=wt, algo=algo)
+                     layout=layout, wtype=wt, algo=algo, multiplier=M)
     if dwconv2d_out_shape(desc) != (Ho, Wo):
         raise ValueError(f"dy spatial extents {(Ho, Wo)} do not match the forward's "
                          f"{dwconv2d_out_shape(desc)}")
@@ -379,8 +401,9 @@ def dwconv2d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel_hw: Tuple[int,
                         algo: str = "auto", bias: bool = True,
                         dw: Optional[torch.Tensor] = None, db: Optional[torch.Tensor] = None,
                         workspace: Optional[torch.Tensor] = None):
-    """(dW [C,kH,kW], db [C] or None): weight and bias gradients of the
-    forward with input x and output cotangent dy.  `workspace` (a CUDA byte
+    """(dW [C*M,kH,kW], db [C*M] or None): weight and bias gradients of the
+    forward with input x (C channels) and output cotangent dy (C*M channels;
+    M, the channel multiplier, is read off dy).  `workspace` (a CUDA byte
     tensor of at least dwconv2d_bwd_weight_workspace_size bytes) is allocated
     when not given."""
     _check_act(x, "x")
@@ -392,18 +415,21 @@ def dwconv2d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel_hw: Tuple[int,
         N, H, W, C = x.shape
     else:
         N, C, H, W = x.shape
+    Co = int(dy.shape[3] if layout.lower() == "nhwc" else dy.shape[1])
+    if Co < C or Co % C != 0:
+        raise ValueError(f"dy must have C*multiplier channels for C={C}, got {Co}")
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, algo=algo)
+                     layout=layout, algo=algo, multiplier=Co // C)
     Ho, Wo = dwconv2d_out_shape(desc)
-    want = (N, Ho, Wo, C) if desc.layout == DW_NHWC else (N, C, Ho, Wo)
+    want = (N, Ho, Wo, Co) if desc.layout == DW_NHWC else (N, Co, Ho, Wo)
     if tuple(dy.shape) != want:
         raise ValueError(f"dy must have shape {want}, got {tuple(dy.shape)}")
     if dw is None:
-        dw = torch.empty((C, kH, kW), device=x.device, dtype=torch.float32)
-    elif dw.dtype != torch.float32 or dw.numel() != C * kH * kW or not dw.is_contiguous():
-        raise ValueError("dw must be a contiguous float32 tensor of C*kH*kW elements")
+        dw = torch.empty((Co, kH, kW), device=x.device, dtype=torch.float32)
+    elif dw.dtype != torch.float32 or dw.numel() != Co * kH * kW or not dw.is_contiguous():
+        raise ValueError("dw must be a contiguous float32 tensor of C*multiplier*kH*kW elements")
     if bias and db is None:
-        db = torch.empty((C,), device=x.device, dtype=torch.float32)
+        db = torch.empty((Co,), device=x.device, dtype=torch.float32)
     need = dwconv2d_bwd_weight_workspace_size(desc)
     if workspace is None:
         workspace = torch.empty((max(need, 1),), device=x.device, dtype=torch.uint8)

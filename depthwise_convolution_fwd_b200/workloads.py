@@ -35,16 +35,21 @@ class Case:
     act: str = "uniform"      # x and dy: "uniform" U(-1,1) or "normal" N(0,1)
     bias: bool = True         # b ~ U(-0.1, 0.1)
     seed: int = 0
+    multiplier: int = 1       # output channels per input channel (C*multiplier outputs)
 
     def in_shape(self) -> Tuple[int, int, int, int]:
         if self.layout == "nhwc":
             return (self.N, self.H, self.W, self.C)
         return (self.N, self.C, self.H, self.W)
 
+    @property
+    def Co(self) -> int:
+        return self.C * self.multiplier
+
     def out_shape(self, Ho: int, Wo: int) -> Tuple[int, int, int, int]:
         if self.layout == "nhwc":
-            return (self.N, Ho, Wo, self.C)
-        return (self.N, self.C, Ho, Wo)
+            return (self.N, Ho, Wo, self.Co)
+        return (self.N, self.Co, Ho, Wo)
 
     def with_(self, **kw) -> "Case":
         return dataclasses.replace(self, **kw)
@@ -59,7 +64,7 @@ def _act(gen: torch.Generator, shape, kind: str) -> torch.Tensor:
 
 
 def make_inputs(case: Case, out_hw: Tuple[int, int]) -> Dict[str, Optional[torch.Tensor]]:
-    """CPU float32 tensors x, w ([C,kH,kW], float32 or float16), b, dy.
+    """CPU float32 tensors x, w ([C*M,kH,kW], float32 or float16), b [C*M], dy.
 
     W ~ N(0, 1/(kH*kW)) (variance 1/(kH*kW)); with wtype "f16" the draw is
     rounded to float16 (round to nearest even), so `w` holds float16-exact
@@ -67,9 +72,9 @@ def make_inputs(case: Case, out_hw: Tuple[int, int]) -> Dict[str, Optional[torch
     """
     gen = torch.Generator().manual_seed(case.seed)
     x = _act(gen, case.in_shape(), case.act)
-    w = torch.randn((case.C, case.kH, case.kW), generator=gen, dtype=torch.float32)
+    w = torch.randn((case.Co, case.kH, case.kW), generator=gen, dtype=torch.float32)
     w = w * (1.0 / (case.kH * case.kW)) ** 0.5
-    b = (torch.rand((case.C,), generator=gen, dtype=torch.float32) * 0.2 - 0.1) if case.bias else None
+    b = (torch.rand((case.Co,), generator=gen, dtype=torch.float32) * 0.2 - 0.1) if case.bias else None
     dy = _act(gen, case.out_shape(*out_hw), case.act)
     if case.wtype == "f16":
         w16 = w.to(torch.float16)
@@ -132,6 +137,19 @@ def large() -> List[Case]:
         out.append(Case(f"large_30x19x128_7x7_{layout}", 1, 30, 19, 128, 7, 7,
                         layout=layout, seed=seed))
         seed += 1
+    return out
+
+
+def multiplier() -> List[Case]:
+    """Channel multiplier: the grouped-gradient page's case (a 3x3 conv from 4
+    to 8 channels, groups = 4, on a 4x4 input; W,H,C,N = 4,4,4,1) and a
+    bandwidth-sized one, 1x512x512x128 -> 256 channels 3x3 SAME (the same
+    output bytes as the large case), NHWC and NCHW."""
+    out = [Case("mult_page_1x4x4x4_m2", 1, 4, 4, 4, 3, 3, padding=0, multiplier=2,
+                act="uniform", seed=1500)]
+    for i, layout in enumerate(("nhwc", "nchw")):
+        out.append(Case(f"mult_512x512x128_m2_{layout}", 1, 512, 512, 128, 3, 3, layout=layout,
+                        multiplier=2, seed=1501 + i))
     return out
 
 

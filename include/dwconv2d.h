@@ -99,6 +99,14 @@ enum { DW_ACT_NONE = 0, DW_ACT_RELU = 1, DW_ACT_RELU6 = 2, DW_ACT_SILU = 3 };
  * DW_ALGO_DIRECT forces the one-thread-per-output kernel (any shape);
  * DW_ALGO_TILED forces the TMA-tiled kernels (DW_ERR_UNSUPPORTED if they do
  * not cover the shape).
+ * multiplier: M output channels per input channel (0 and 1 both mean the
+ * plain depthwise convolution, M = 1; at most 4096).  With M > 1 the
+ * forward maps C input channels to C*M output channels: output channel
+ * o = c*M + j reads only input channel c = o / M, through filter w[o] and
+ * bias b[o] (a grouped convolution with groups = C, as in the page
+ * "Incorrect stableHLO for grouped convolution gradient", a conv from 4 to
+ * 8 channels with groups = 4).  Then w is [C*M,kH,kW], b [C*M], y and dy
+ * have C*M channels, x and dx have C; every entry point applies it.
  */
 typedef struct dw_desc {
     int64_t N, H, W, C;
@@ -110,6 +118,7 @@ typedef struct dw_desc {
     int32_t layout;
     int32_t wtype;
     int32_t algo;
+    int32_t multiplier;
 } dw_desc_t;
 
 /* Output extents Ho, Wo of the forward for `desc` (host only, no CUDA call).

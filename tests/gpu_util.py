@@ -22,7 +22,7 @@ TOL = 1e-5
 
 def problem(case: Case):
     return oracle.problem(case.in_shape(), case.kH, case.kW, case.stride, case.dilation,
-                          case.padding, case.layout)
+                          case.padding, case.layout, multiplier=case.multiplier)
 
 
 def out_hw(case: Case):
@@ -96,13 +96,14 @@ def gpu_bwd(case, inp, algo="auto", w_key="w", out=None, device="cuda"):
     w = inp[w_key].to(device)
     return dw.dwconv2d_bwd_input(dy, w, (case.H, case.W), stride=case.stride,
                                  dilation=case.dilation, padding=case.padding,
-                                 layout=case.layout, algo=algo, out=out)
+                                 layout=case.layout, algo=algo, out=out,
+                                 multiplier=case.multiplier)
 
 
 def desc_of(case, algo="auto"):
     return dw.make_desc(case.N, case.H, case.W, case.C, case.kH, case.kW, stride=case.stride,
                         dilation=case.dilation, padding=case.padding, layout=case.layout,
-                        wtype=case.wtype, algo=algo)
+                        wtype=case.wtype, algo=algo, multiplier=case.multiplier)
 
 
 def chosen_algo(case, op, t_in, t_w, t_out, algo="auto"):

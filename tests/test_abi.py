@@ -219,3 +219,31 @@ def test_fused_epilogue_host_checks(lib):
     bad = dw.make_desc(1, 8, 8, 4, 3, 3)
     bad.kH = 0
     assert R(bad, x, w, None, st, 1e-5, dw.DW_ACT_NONE, y, 0) == dw.DW_ERR_INVALID_ARG
+
+
+def test_channel_multiplier_host_checks(lib):
+    # 0 and 1 both mean the plain depthwise convolution; negative or huge: invalid
+    fake = 1 << 40
+    for m, ok in ((0, True), (1, True), (3, True), (-1, False), (5000, False)):
+        d = dw.make_desc(1, 8, 8, 4, 3, 3, multiplier=m)
+        if ok:
+            assert dw.dwconv2d_out_shape(d) == (8, 8)
+        else:
+            with pytest.raises(dw.DwError):
+                dw.dwconv2d_out_shape(d)
+            assert dw.fwd_raw(d, fake, fake + (1 << 20), None, fake + (2 << 20), 0) == dw.DW_ERR_INVALID_ARG
+    # sizes use C*M output channels: x 1 KiB, y 2 KiB (M = 2)
+    d = dw.make_desc(1, 8, 8, 4, 3, 3, multiplier=2)
+    base = 1 << 40
+    w = base + (1 << 20)
+    assert dw.dwconv2d_query_algo(d, 0, base, w, base + 1024) > 0          # adjacent: fine
+    assert dw.fwd_raw(d, base, w, None, w - 2047, 0) == dw.DW_ERR_ALIAS      # y (2 KiB) over w
+    assert dw.fwd_raw(d, base, w, w + 4096, w + 4096 - 2040, 0) == dw.DW_ERR_ALIAS  # y over b
+    assert dw.bwd_input_raw(d, base, w, base + 2040, 0) == dw.DW_ERR_ALIAS   # dx over dy (2 KiB)
+    # filter of C*M rows: a y placed right after a 4*9*4-byte filter would overlap an 8-row one
+    assert dw.fwd_raw(d, base, w, None, w + 4 * 9 * 4, 0) == dw.DW_ERR_ALIAS
+    # the weight gradient sizes dW and db by C*M as well
+    need = dw.dwconv2d_bwd_weight_workspace_size(d)
+    x, dy, dwp, db, ws = base, base + (1 << 24), base + (2 << 24), base + (3 << 24), base + (4 << 24)
+    assert dw.bwd_weight_raw(d, x, dy, dwp, dwp + 8 * 9 * 4 - 4, ws, need, 0) == dw.DW_ERR_ALIAS
+    assert dw.dwconv2d_query_algo(d, 2, x, dy, dwp) == dw.DW_ALGO_DIRECT

@@ -42,7 +42,7 @@ def cuda_ready():
 
 
 def bn_of(case):
-    return wl.make_bn(case.C, case.seed + 500)
+    return wl.make_bn(case.Co, case.seed + 500)
 
 
 def bound(case, inp, bn, act, idx=None):
