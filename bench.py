@@ -71,20 +71,21 @@ def workload_cases(name):
     raise ValueError(name)
 
 
-def algorithmic_bytes(case, Ho, Wo, op):
+def algorithmic_bytes(case, Ho, Wo, op, esz=4):
     """Bytes one call must move at minimum: read the input once, write the
-    output once, read the filters (and the bias for the forward)."""
+    output once, read the filters (and the bias for the forward); esz is the
+    activation element size (4 for float32, 2 for float16 / bfloat16)."""
     Co = case.C * case.multiplier  # output channels
     n_in = case.N * case.C * case.H * case.W
     n_out = case.N * Co * Ho * Wo
     wbytes = Co * case.kH * case.kW * (2 if case.wtype == "f16" else 4)
     if op == "fwd":
-        return 4 * n_in + 4 * n_out + wbytes + (4 * Co if case.bias else 0)
+        return esz * (n_in + n_out) + wbytes + (4 * Co if case.bias else 0)
     if op == "fused":  # forward + four [Co] batch-norm statistics
-        return 4 * n_in + 4 * n_out + wbytes + (4 * Co if case.bias else 0) + 16 * Co
+        return esz * (n_in + n_out) + wbytes + (4 * Co if case.bias else 0) + 16 * Co
     if op == "wgrad":  # read x and dy, write dW [Co,kH,kW] and db [Co] (f32)
-        return 4 * n_in + 4 * n_out + 4 * Co * case.kH * case.kW + 4 * Co
-    return 4 * n_out + 4 * n_in + wbytes
+        return esz * (n_in + n_out) + 4 * Co * case.kH * case.kW + 4 * Co
+    return esz * (n_out + n_in) + wbytes
 
 
 def src_digest():
@@ -187,16 +188,22 @@ class ClockSampler:
 class Shape:
     """One workload shape with its buffer sets and prepared C-ABI calls."""
 
-    def __init__(self, case, dw, torch, device, sets):
+    def __init__(self, case, dw, torch, device, sets, atype="f32"):
         from depthwise_convolution_fwd_b200.workloads import make_inputs
         self.case = case
         desc = dw.make_desc(case.N, case.H, case.W, case.C, case.kH, case.kW,
                             stride=case.stride, dilation=case.dilation, padding=case.padding,
-                            layout=case.layout, wtype=case.wtype, multiplier=case.multiplier)
+                            layout=case.layout, wtype=case.wtype, multiplier=case.multiplier,
+                            atype=atype)
         self.desc = desc
         self.Ho, self.Wo = dw.dwconv2d_out_shape(desc)
-        self.host = make_inputs(case, (self.Ho, self.Wo))
-        self.bytes = {op: algorithmic_bytes(case, self.Ho, self.Wo, op) for op in ("fwd", "bwd")}
+        dt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[atype]
+        self.esz = 4 if atype == "f32" else 2
+        host = make_inputs(case, (self.Ho, self.Wo))
+        host["x"], host["dy"] = host["x"].to(dt), host["dy"].to(dt)
+        self.host = host
+        self.bytes = {op: algorithmic_bytes(case, self.Ho, self.Wo, op, self.esz)
+                      for op in ("fwd", "bwd")}
         self.w = self.host["w"].to(device)
         self.b = None if self.host["b"] is None else self.host["b"].to(device)
         out_shape = case.out_shape(self.Ho, self.Wo)
@@ -204,9 +211,9 @@ class Shape:
         for _ in range(sets):
             self.sets.append({
                 "x": self.host["x"].to(device), "dy": self.host["dy"].to(device),
-                "y": torch.empty(out_shape, device=device),
-                "dx": torch.empty(case.in_shape(), device=device)})
-        self.set_bytes = sum(t.numel() * 4 for t in self.sets[0].values())
+                "y": torch.empty(out_shape, device=device, dtype=dt),
+                "dx": torch.empty(case.in_shape(), device=device, dtype=dt)})
+        self.set_bytes = sum(t.numel() * t.element_size() for t in self.sets[0].values())
 
     def prepare_next_rows(self, dw, torch, device, act):
         """Buffers of the calls measured beside the step: the weight gradient
@@ -220,7 +227,7 @@ class Shape:
         self.dW = torch.empty(c.Co * c.kH * c.kW, device=device)
         self.db = torch.empty(c.Co, device=device)
         for op in ("fused", "wgrad"):
-            self.bytes[op] = algorithmic_bytes(c, self.Ho, self.Wo, op)
+            self.bytes[op] = algorithmic_bytes(c, self.Ho, self.Wo, op, self.esz)
 
     def call(self, dw, op, r, stream):
         s = self.sets[r % len(self.sets)]
@@ -350,6 +357,19 @@ def run_ours(args, rank, world, local_rank):
                 if op == "fused":
                     k["epilogue"] = f"inference batch norm + {act}"
                 next_rows[f"{sh.case.name}:{op}"] = k
+        # 16-bit activations: the same calls moving half the bytes
+        for c in cases:
+            for at in ("f16", "bf16"):
+                sh16 = Shape(c, dw, torch, device, 1, atype=at)
+                with torch.cuda.stream(stream):
+                    for op in ("fwd", "bwd"):
+                        sh16.call(dw, op, 0, sptr)
+                torch.cuda.synchronize()
+                for op in ("fwd", "bwd"):
+                    k = time_kernel(torch, dw, sh16, op, l2, stream)
+                    k["frac"] = k["gbs"] / peak
+                    next_rows[f"{c.name}:{op}_{at}"] = k
+                del sh16
 
     # end to end through the public tensor API: pinned host inputs -> device,
     # forward + input gradient, outputs -> pinned host, every step

@@ -144,6 +144,7 @@ static dw_status_t resolve(const dw_desc_t* d, Problem* p) {
         return DW_ERR_INVALID_ARG;
     if (d->layout != DW_NHWC && d->layout != DW_NCHW) return DW_ERR_INVALID_ARG;
     if (d->wtype != DW_F32 && d->wtype != DW_F16) return DW_ERR_INVALID_ARG;
+    if (d->atype != DW_F32 && d->atype != DW_F16 && d->atype != DW_BF16) return DW_ERR_INVALID_ARG;
     if (d->algo < DW_ALGO_AUTO || d->algo > DW_ALGO_TILED) return DW_ERR_INVALID_ARG;
     if (d->multiplier < 0 || d->multiplier > kMaxMultiplier) return DW_ERR_INVALID_ARG;
     p->N = d->N; p->H = d->H; p->W = d->W; p->C = d->C;
@@ -153,7 +154,7 @@ static dw_status_t resolve(const dw_desc_t* d, Problem* p) {
     p->kH = d->kH; p->kW = d->kW;
     p->sh = d->stride_h; p->sw = d->stride_w;
     p->dh = d->dil_h; p->dw = d->dil_w;
-    p->layout = d->layout; p->wtype = d->wtype;
+    p->layout = d->layout; p->wtype = d->wtype; p->atype = d->atype;
     if (d->pad_mode == DW_PAD_SAME) {
         same_pads(d->H, d->kH, d->stride_h, d->dil_h, &p->pt, &p->pb);
         same_pads(d->W, d->kW, d->stride_w, d->dil_w, &p->pl, &p->pr);
@@ -185,10 +186,10 @@ static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 struct Buffers {
-    const float* in;
+    const void* in;  // activations of type p.atype
     const void* w;
     const float* b;
-    float* out;
+    void* out;       // activations of type p.atype
 };
 
 static dw_status_t check_buffers(const Problem& p, Op op, const Buffers& bf) {
@@ -198,8 +199,9 @@ static dw_status_t check_buffers(const Problem& p, Op op, const Buffers& bf) {
     const size_t in_elems = op == OP_FWD ? x_elems : y_elems;
     const size_t out_elems = op == OP_FWD ? y_elems : x_elems;
     const size_t w_bytes = size_t(p.Co) * size_t(p.kH) * size_t(p.kW) * (p.wtype == DW_F16 ? 2 : 4);
-    const size_t out_bytes = out_elems * 4;
-    if (overlaps(bf.out, out_bytes, bf.in, in_elems * 4)) return DW_ERR_ALIAS;
+    const size_t eb = size_t(act_bytes(p.atype));
+    const size_t out_bytes = out_elems * eb;
+    if (overlaps(bf.out, out_bytes, bf.in, in_elems * eb)) return DW_ERR_ALIAS;
     if (overlaps(bf.out, out_bytes, bf.w, w_bytes)) return DW_ERR_ALIAS;
     if (op == OP_FWD && overlaps(bf.out, out_bytes, bf.b, size_t(p.Co) * 4)) return DW_ERR_ALIAS;
     return DW_OK;
@@ -214,7 +216,8 @@ static dw_status_t run(const dw_desc_t* desc, Op op, const Buffers& bf, cudaStre
     if (st != DW_OK) return st;
     if (epi) {
         // every statistics array must stay clear of y
-        const size_t yb = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo) * 4;
+        const size_t yb = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo) *
+                          size_t(act_bytes(p.atype));
         const float* stats[4] = {epi->gamma, epi->beta, epi->mean, epi->var};
         for (const float* v : stats)
             if (overlaps(bf.out, yb, v, size_t(p.Co) * 4)) return DW_ERR_ALIAS;
@@ -265,16 +268,16 @@ dw_status_t dwconv2d_resolved_pads(const dw_desc_t* desc, int32_t pads[4]) {
     return DW_OK;
 }
 
-dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const float* x, const void* w, const float* b,
-                         float* y, void* stream) {
+dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const void* x, const void* w, const float* b,
+                         void* y, void* stream) {
     return run(desc, OP_FWD, Buffers{x, w, b, y}, static_cast<cudaStream_t>(stream), false,
                nullptr);
 }
 
-dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const float* x, const void* w,
+dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const void* x, const void* w,
                                 const float* b, const float* gamma, const float* beta,
                                 const float* mean, const float* var, float eps, int32_t act,
-                                float* y, void* stream) {
+                                void* y, void* stream) {
     const int given = (gamma != nullptr) + (beta != nullptr) + (mean != nullptr) + (var != nullptr);
     if (given != 0 && given != 4) return DW_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || !(eps <= 3.402823466e38f)) return DW_ERR_INVALID_ARG;  // NaN, inf, < 0
@@ -290,7 +293,7 @@ dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const float* x, const voi
                nullptr, &e);
 }
 
-dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy, const void* w, float* dx,
+dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const void* dy, const void* w, void* dx,
                                void* stream) {
     return run(desc, OP_BWD_INPUT, Buffers{dy, w, nullptr, dx}, static_cast<cudaStream_t>(stream),
                false, nullptr);
@@ -305,7 +308,7 @@ dw_status_t dwconv2d_bwd_weight_workspace_size(const dw_desc_t* desc, uint64_t* 
     return DW_OK;
 }
 
-static dw_status_t run_bwd_weight(const dw_desc_t* desc, const float* x, const float* dy,
+static dw_status_t run_bwd_weight(const dw_desc_t* desc, const void* x, const void* dy,
                                   float* dw, float* db, void* ws, uint64_t ws_bytes,
                                   cudaStream_t stream, bool dry_run, int32_t* chosen) {
     Problem p;
@@ -313,8 +316,9 @@ static dw_status_t run_bwd_weight(const dw_desc_t* desc, const float* x, const f
     if (st != DW_OK) return st;
     if (!x || !dy || !dw || !ws) return DW_ERR_INVALID_ARG;
     if (ws_bytes < bwd_weight_workspace_bytes(p)) return DW_ERR_INVALID_ARG;
-    const size_t xb = size_t(p.N) * size_t(p.C) * size_t(p.H) * size_t(p.W) * 4;
-    const size_t gb = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo) * 4;
+    const size_t eb = size_t(act_bytes(p.atype));
+    const size_t xb = size_t(p.N) * size_t(p.C) * size_t(p.H) * size_t(p.W) * eb;
+    const size_t gb = size_t(p.N) * size_t(p.Co) * size_t(p.Ho) * size_t(p.Wo) * eb;
     const size_t wb = size_t(p.Co) * size_t(p.kH) * size_t(p.kW) * 4;
     const size_t bb = size_t(p.Co) * 4;
     const void* ins[2] = {x, dy};
@@ -335,14 +339,14 @@ static dw_status_t run_bwd_weight(const dw_desc_t* desc, const float* x, const f
     return bwd_weight_launch(p, desc->algo, x, dy, dw, db, ws, stream, err, dry_run, chosen);
 }
 
-dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const float* x, const float* dy, float* dw,
+dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const void* x, const void* dy, float* dw,
                                 float* db, void* workspace, uint64_t workspace_bytes,
                                 void* stream) {
     return run_bwd_weight(desc, x, dy, dw, db, workspace, workspace_bytes,
                           static_cast<cudaStream_t>(stream), false, nullptr);
 }
 
-dw_status_t dwconv2d_bwd_weight_noalloc(const dw_desc_t* desc, const float* x, const float* dy,
+dw_status_t dwconv2d_bwd_weight_noalloc(const dw_desc_t* desc, const void* x, const void* dy,
                                         float* dw, float* db, void* stream) {
     Problem p;
     const dw_status_t st = resolve(desc, &p);
@@ -363,7 +367,7 @@ int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void* in, c
         if (st != DW_OK) return -st;
         const uint64_t need = bwd_weight_workspace_bytes(p);
         // a workspace address far from the tensors, only used for the checks
-        st = run_bwd_weight(desc, static_cast<const float*>(in), static_cast<const float*>(w),
+        st = run_bwd_weight(desc, in, w,
                             static_cast<float*>(const_cast<void*>(out)), nullptr,
                             reinterpret_cast<void*>(uintptr_t(1) << 62), need, nullptr, true,
                             &chosen);
@@ -373,8 +377,7 @@ int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void* in, c
     int32_t chosen = 0;
     const dw_status_t st =
         run(desc, static_cast<Op>(op),
-            Buffers{static_cast<const float*>(in), w, nullptr,
-                    static_cast<float*>(const_cast<void*>(out))},
+            Buffers{in, w, nullptr, const_cast<void*>(out)},
             nullptr, true, &chosen);
     return st == DW_OK ? chosen : -st;
 }

@@ -51,8 +51,9 @@ struct DArgs {
 
 // NHWC: one thread per (chunk, tap, channel), channel fastest, so a warp reads
 // 32 consecutive channels of one pixel.
-__global__ void __launch_bounds__(256) partial_direct_nhwc(const float* __restrict__ x,
-                                                           const float* __restrict__ dy,
+template <class TA>
+__global__ void __launch_bounds__(256) partial_direct_nhwc(const TA* __restrict__ x,
+                                                           const TA* __restrict__ dy,
                                                            double* __restrict__ part, DArgs a) {
     grid_dependency_wait();
     allow_dependents();
@@ -73,14 +74,15 @@ __global__ void __launch_bounds__(256) partial_direct_nhwc(const float* __restri
         float part32 = 0.f;
         int cnt = 0;
         for (int64_t pp = p0; pp < p1; ++pp) {
-            const float g = __ldg(dy + ((n * a.Ho + ho) * a.Wo + wo) * a.Co + o);
+            const float g = ActIO<TA>::load1(dy + ((n * a.Ho + ho) * a.Wo + wo) * a.Co + o);
             if (bias) {
                 part32 += g;
             } else {
                 const int64_t hi = ho * a.sh + int64_t(kh) * a.dh - a.pt;
                 const int64_t wi = wo * a.sw + int64_t(kw) * a.dw - a.pl;
                 if (hi >= 0 && hi < a.H && wi >= 0 && wi < a.W)
-                    part32 = fmaf(g, __ldg(x + ((n * a.H + hi) * a.W + wi) * a.C + c), part32);
+                    part32 = fmaf(g, ActIO<TA>::load1(x + ((n * a.H + hi) * a.W + wi) * a.C + c),
+                                  part32);
             }
             if (++cnt == kFold) {
                 acc += double(part32);
@@ -101,8 +103,9 @@ __global__ void __launch_bounds__(256) partial_direct_nhwc(const float* __restri
 
 // NCHW: one warp per (chunk, tap, channel); lanes walk consecutive output
 // positions (W innermost), then the warp sums its lanes.
-__global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restrict__ x,
-                                                           const float* __restrict__ dy,
+template <class TA>
+__global__ void __launch_bounds__(256) partial_direct_nchw(const TA* __restrict__ x,
+                                                           const TA* __restrict__ dy,
                                                            double* __restrict__ part, DArgs a) {
     grid_dependency_wait();
     allow_dependents();
@@ -125,14 +128,15 @@ __global__ void __launch_bounds__(256) partial_direct_nchw(const float* __restri
         for (int64_t pp = p0 + lane; pp < p1; pp += 32) {
             const int64_t wo = pp % a.Wo, q = pp / a.Wo;
             const int64_t ho = q % a.Ho, n = q / a.Ho;
-            const float g = __ldg(dy + ((n * a.Co + o) * a.Ho + ho) * a.Wo + wo);
+            const float g = ActIO<TA>::load1(dy + ((n * a.Co + o) * a.Ho + ho) * a.Wo + wo);
             if (bias) {
                 part32 += g;
             } else {
                 const int64_t hi = ho * a.sh + int64_t(kh) * a.dh - a.pt;
                 const int64_t wi = wo * a.sw + int64_t(kw) * a.dw - a.pl;
                 if (hi >= 0 && hi < a.H && wi >= 0 && wi < a.W)
-                    part32 = fmaf(g, __ldg(x + ((n * a.C + c) * a.H + hi) * a.W + wi), part32);
+                    part32 = fmaf(g, ActIO<TA>::load1(x + ((n * a.C + c) * a.H + hi) * a.W + wi),
+                                  part32);
             }
             if (++cnt == kFold) {
                 acc += double(part32);
@@ -211,8 +215,11 @@ struct TArgs {
     int ntiles;
 };
 
-template <int KH_, int KW_, int S_, int D_, int THT_, int TWT_, int WX_, int WY_, int NS_>
+template <int KH_, int KW_, int S_, int D_, int THT_, int TWT_, int WX_, int WY_, int NS_,
+          class TA_ = float>
 struct WCfg {
+    using TA = TA_;  // activation element type of x and dy
+    static constexpr int ESZ = sizeof(TA);
     static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
     static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
     static constexpr int T = KH * KW + 1;
@@ -224,13 +231,15 @@ struct WCfg {
     static constexpr int IW = (TW - 1) * S + (KW - 1) * D + 1;
     static constexpr int RH = (THT - 1) * S + (KH - 1) * D + 1;
     static constexpr int RW = (TWT - 1) * S + (KW - 1) * D + 1;
-    static constexpr int XBYTES = IH * IW * kLanes * 4;
-    static constexpr int GBYTES = TH * TW * kLanes * 4;
-    static constexpr int STAGE_BYTES = XBYTES + GBYTES;
+    static constexpr int XBYTES = IH * IW * kLanes * ESZ;
+    static constexpr int GBYTES = TH * TW * kLanes * ESZ;
+    static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;  // dy box on a 128-byte boundary
+    static constexpr int STAGE_TX = XBYTES + GBYTES;           // bytes the two loads bring
+    static constexpr int STAGE_BYTES = (XPITCH + GBYTES + 127) / 128 * 128;
     static constexpr int RED_BYTES = NCW * T * kLanes * 8;
     static constexpr int AREA = NS * STAGE_BYTES > RED_BYTES ? NS * STAGE_BYTES : RED_BYTES;
     static constexpr size_t SMEM = size_t(AREA) + size_t(2 * NS) * 8 + 16;
-    static_assert(XBYTES % 128 == 0 && GBYTES % 128 == 0, "TMA shared-memory alignment");
+    static_assert(ESZ == 4 || (XBYTES % 128 == 0 || XPITCH > XBYTES), "stage layout");
     static_assert(IH <= 256 && IW <= 256 && TW <= 256 && TH <= 256, "TMA box limit");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -301,9 +310,9 @@ __global__ void __launch_bounds__(K::NT, 1)
                 }
                 const WTile T = decode<K>(t, a);
                 unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+                mbar_arrive_expect_tx(&full[s], K::STAGE_TX);
                 tma_load_4d(st, &xmap, &full[s], T.cb * kLanes, T.ix0, T.iy0, T.n);
-                tma_load_4d(st + K::XBYTES, &gmap, &full[s], T.cb * kLanes, T.ox0, T.oy0, T.n);
+                tma_load_4d(st + K::XPITCH, &gmap, &full[s], T.cb * kLanes, T.ox0, T.oy0, T.n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -331,24 +340,26 @@ __global__ void __launch_bounds__(K::NT, 1)
             }
             break;
         }
-        const float* xb = reinterpret_cast<const float*>(smem + size_t(s) * K::STAGE_BYTES);
-        const float* gb = xb + K::XBYTES / 4;
+        using TA = typename K::TA;
+        const TA* xb = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_BYTES);
+        const TA* gb = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_BYTES + K::XPITCH);
         float g[K::THT][K::TWT];
 #pragma unroll
         for (int j = 0; j < K::THT; ++j)
 #pragma unroll
-            for (int i = 0; i < K::TWT; ++i) g[j][i] = gb[((j0 + j) * K::TW + i0 + i) * kLanes + lane];
+            for (int i = 0; i < K::TWT; ++i)
+                g[j][i] = ActIO<TA>::load1(gb + ((j0 + j) * K::TW + i0 + i) * kLanes + lane);
         float acc[K::KH][K::KW];
 #pragma unroll
         for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
             for (int kw = 0; kw < K::KW; ++kw) acc[kh][kw] = 0.f;
-        const float* win = xb + ((j0 * K::S) * K::IW + i0 * K::S) * kLanes + lane;
+        const TA* win = xb + ((j0 * K::S) * K::IW + i0 * K::S) * kLanes + lane;
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             static_for<0, K::RW>([&](auto q_) {
                 constexpr int q = decltype(q_)::value;
-                const float v = win[(r * K::IW + q) * kLanes];
+                const float v = ActIO<TA>::load1(win + (r * K::IW + q) * kLanes);
                 static_for<0, K::THT>([&](auto j_) {
                     constexpr int j = decltype(j_)::value;
                     constexpr int kh = tap_of<K>(r, j);
@@ -438,7 +449,18 @@ size_t tiled_workspace(const Problem& p) {
     return size_t(g) * size_t(p.kH * p.kW + 1) * kLanes * sizeof(double);
 }
 
-dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, float* dw, float* db,
+template <class TA>
+cudaError_t launch_direct_partial(const Problem& p, const void* x, const void* dy, double* part,
+                                  const DArgs& a, int64_t blocks, cudaStream_t stream) {
+    const TA* xt = static_cast<const TA*>(x);
+    const TA* gt = static_cast<const TA*>(dy);
+    return p.layout == DW_NHWC ? launch_pdl(partial_direct_nhwc<TA>, dim3(unsigned(blocks)),
+                                            dim3(256), 0, stream, xt, gt, part, a)
+                               : launch_pdl(partial_direct_nchw<TA>, dim3(unsigned(blocks)),
+                                            dim3(256), 0, stream, xt, gt, part, a);
+}
+
+dw_status_t launch_direct(const Problem& p, const void* x, const void* dy, float* dw, float* db,
                           void* ws, cudaStream_t stream) {
     DArgs a;
     a.N = p.N; a.C = p.C; a.H = p.H; a.W = p.W; a.Ho = p.Ho; a.Wo = p.Wo;
@@ -456,11 +478,10 @@ dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, flo
     int64_t blocks = (threads_needed + 255) / 256;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    cudaError_t e = p.layout == DW_NHWC
-                        ? launch_pdl(partial_direct_nhwc, dim3(unsigned(blocks)), dim3(256), 0,
-                                     stream, x, dy, part, a)
-                        : launch_pdl(partial_direct_nchw, dim3(unsigned(blocks)), dim3(256), 0,
-                                     stream, x, dy, part, a);
+    cudaError_t e =
+        p.atype == DW_F16    ? launch_direct_partial<__half>(p, x, dy, part, a, blocks, stream)
+        : p.atype == DW_BF16 ? launch_direct_partial<__nv_bfloat16>(p, x, dy, part, a, blocks, stream)
+                             : launch_direct_partial<float>(p, x, dy, part, a, blocks, stream);
     if (e != cudaSuccess) return DW_ERR_CUDA;
     const int64_t fb = finalize_blocks(p.Co * a.T, sm_count(dev));
     e = launch_pdl(finalize_direct, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
@@ -470,7 +491,7 @@ dw_status_t launch_direct(const Problem& p, const float* x, const float* dy, flo
 }
 
 template <class K>
-dw_status_t launch_tiled(const Problem& p, const float* x, const float* dy, float* dw, float* db,
+dw_status_t launch_tiled(const Problem& p, const void* x, const void* dy, float* dw, float* db,
                          void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
     TArgs a;
     a.part = static_cast<double*>(ws);
@@ -506,18 +527,18 @@ dw_status_t launch_tiled(const Problem& p, const float* x, const float* dy, floa
 
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMap xmap, gmap;
+    constexpr cuuint64_t E = K::ESZ;
     const cuuint64_t xd[4] = {cuuint64_t(p.C), cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.N)};
-    const cuuint64_t xs[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * p.W) * 4,
-                              cuuint64_t(p.C * p.W * p.H) * 4};
+    const cuuint64_t xs[3] = {cuuint64_t(p.C) * E, cuuint64_t(p.C * p.W) * E,
+                              cuuint64_t(p.C * p.W * p.H) * E};
     const cuuint32_t xbox[4] = {kLanes, K::IW, K::IH, 1};
     const cuuint64_t gd[4] = {cuuint64_t(p.C), cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.N)};
-    const cuuint64_t gs[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * p.Wo) * 4,
-                              cuuint64_t(p.C * p.Wo * p.Ho) * 4};
+    const cuuint64_t gs[3] = {cuuint64_t(p.C) * E, cuuint64_t(p.C * p.Wo) * E,
+                              cuuint64_t(p.C * p.Wo * p.Ho) * E};
     const cuuint32_t gbox[4] = {kLanes, K::TW, K::TH, 1};
-    if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
-                          xbox, estr) != CUDA_SUCCESS ||
-        encode_tensor_map(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(dy), gd, gs,
-                          gbox, estr) != CUDA_SUCCESS)
+    constexpr CUtensorMapDataType dt = ActIO<typename K::TA>::kTma;
+    if (encode_tensor_map(&xmap, dt, 4, const_cast<void*>(x), xd, xs, xbox, estr) != CUDA_SUCCESS ||
+        encode_tensor_map(&gmap, dt, 4, const_cast<void*>(dy), gd, gs, gbox, estr) != CUDA_SUCCESS)
         return DW_ERR_CUDA;
     if (launch_pdl(partial_tiled<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap, gmap,
                    a) != cudaSuccess)
@@ -1097,30 +1118,47 @@ dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, f
 }
 
 //                         KH KW  S  D THT TWT WX WY NS
-using W33s1 = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4>;
-using W33s2 = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4>;
-using W55s1 = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3>;
-using W77s1 = WCfg<7, 7, 1, 1, 1, 4, 4, 2, 3>;
-using W1x15 = WCfg<1, 15, 1, 1, 1, 8, 8, 1, 4>;
-using W1x31 = WCfg<1, 31, 1, 1, 1, 8, 8, 1, 4>;
+template <class TA> using W33s1 = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4, TA>;
+template <class TA> using W33s2 = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4, TA>;
+template <class TA> using W55s1 = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3, TA>;
+template <class TA> using W77s1 = WCfg<7, 7, 1, 1, 1, 4, 4, 2, 3, TA>;
+template <class TA> using W1x15 = WCfg<1, 15, 1, 1, 1, 8, 8, 1, 4, TA>;
+template <class TA> using W1x31 = WCfg<1, 31, 1, 1, 1, 8, 8, 1, 4, TA>;
 
-dw_status_t tiled_pick(const Problem& p, const float* x, const float* dy, float* dw, float* db,
+template <class TA>
+dw_status_t tiled_pick_nhwc(const Problem& p, const void* x, const void* dy, float* dw, float* db,
+                            void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    // TMA row strides: C elements a multiple of 16 bytes
+    if ((p.C * int64_t(sizeof(TA))) % 16 != 0) return DW_ERR_UNSUPPORTED;
+    const int S = p.sh;
+#define DW_W(CFG) return launch_tiled<CFG<TA>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && S == 1) DW_W(W33s1)
+    if (p.kH == 3 && p.kW == 3 && S == 2) DW_W(W33s2)
+    if (p.kH == 5 && p.kW == 5 && S == 1) DW_W(W55s1)
+    if (p.kH == 7 && p.kW == 7 && S == 1) DW_W(W77s1)
+    if (p.kH == 1 && p.kW == 15 && S == 1) DW_W(W1x15)
+    if (p.kH == 1 && p.kW == 31 && S == 1) DW_W(W1x31)
+#undef DW_W
+    return DW_ERR_UNSUPPORTED;
+}
+
+dw_status_t tiled_pick(const Problem& p, const void* x, const void* dy, float* dw, float* db,
                        void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
     if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
-    if (p.layout == DW_NCHW) return tiled_pick_nchw(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.layout != DW_NHWC || p.C % 4 != 0) return DW_ERR_UNSUPPORTED;
+    if (p.layout == DW_NCHW) {
+        if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;  // 16-bit NCHW: direct kernels
+        return tiled_pick_nchw(p, static_cast<const float*>(x), static_cast<const float*>(dy), dw,
+                               db, ws, stream, err, dry_run);
+    }
+    if (p.layout != DW_NHWC) return DW_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
         return DW_ERR_UNSUPPORTED;
     if (p.sh != p.sw || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
     if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.C >= INT_MAX) return DW_ERR_UNSUPPORTED;
-    const int S = p.sh;
-    if (p.kH == 3 && p.kW == 3 && S == 1) return launch_tiled<W33s1>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 3 && p.kW == 3 && S == 2) return launch_tiled<W33s2>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 5 && p.kW == 5 && S == 1) return launch_tiled<W55s1>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 7 && p.kW == 7 && S == 1) return launch_tiled<W77s1>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 1 && p.kW == 15 && S == 1) return launch_tiled<W1x15>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 1 && p.kW == 31 && S == 1) return launch_tiled<W1x31>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    return DW_ERR_UNSUPPORTED;
+    if (p.atype == DW_F16) return tiled_pick_nhwc<__half>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.atype == DW_BF16)
+        return tiled_pick_nhwc<__nv_bfloat16>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    return tiled_pick_nhwc<float>(p, x, dy, dw, db, ws, stream, err, dry_run);
 }
 
 }  // namespace wgrad
@@ -1135,7 +1173,7 @@ size_t bwd_weight_workspace_bytes(const Problem& p) {
     return m;
 }
 
-dw_status_t bwd_weight_launch(const Problem& p, int algo, const float* x, const float* dy,
+dw_status_t bwd_weight_launch(const Problem& p, int algo, const void* x, const void* dy,
                               float* dw, float* db, void* ws, cudaStream_t stream, int32_t* err,
                               bool dry_run, int32_t* chosen) {
     if (algo == DW_ALGO_AUTO || algo == DW_ALGO_TILED) {

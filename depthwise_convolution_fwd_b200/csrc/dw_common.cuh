@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -37,6 +38,7 @@ struct Problem {
     int pt, pb, pl, pr;
     int layout;  // DW_NHWC / DW_NCHW
     int wtype;   // DW_F32 / DW_F16
+    int atype = DW_F32;  // activations (x, y, dy, dx): DW_F32 / DW_F16 / DW_BF16
     Epilogue epi;  // forward only; off for every other call
 };
 
@@ -44,20 +46,20 @@ enum Op { OP_FWD = 0, OP_BWD_INPUT = 1 };
 
 // Launch entry points of each kernel family.  `dry_run` only answers whether
 // the family covers the problem (DW_OK / DW_ERR_UNSUPPORTED) without touching
-// the device.
-dw_status_t direct_launch(const Problem& p, Op op, const float* in, const void* w,
-                          const float* b, float* out, cudaStream_t stream);
-dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const float* in, const void* w,
-                              const float* b, float* out, cudaStream_t stream,
+// the device.  `in` and `out` hold activations of type p.atype.
+dw_status_t direct_launch(const Problem& p, Op op, const void* in, const void* w,
+                          const float* b, void* out, cudaStream_t stream);
+dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const void* in, const void* w,
+                              const float* b, void* out, cudaStream_t stream,
                               int32_t* dev_err, bool dry_run);
-dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const void* w,
-                              const float* b, float* out, cudaStream_t stream,
+dw_status_t tiled_nchw_launch(const Problem& p, Op op, const void* in, const void* w,
+                              const float* b, void* out, cudaStream_t stream,
                               int32_t* dev_err, bool dry_run);
 
 // Weight / bias gradient (dw_bwd_weight.cu): workspace bytes the call needs,
 // and the launch (partials into `ws`, then the fixed-order finalize).
 size_t bwd_weight_workspace_bytes(const Problem& p);
-dw_status_t bwd_weight_launch(const Problem& p, int algo, const float* x, const float* dy,
+dw_status_t bwd_weight_launch(const Problem& p, int algo, const void* x, const void* dy,
                               float* dw, float* db, void* ws, cudaStream_t stream,
                               int32_t* dev_err, bool dry_run, int32_t* chosen);
 
@@ -343,5 +345,79 @@ __device__ __forceinline__ void fma4(float4& acc, const float4& v, const float4&
 __device__ __forceinline__ void store4(float* p, const float4& v) {
     *reinterpret_cast<float4*>(p) = v;
 }
+
+// Activation element types: float32, float16, bfloat16.  Loads widen to
+// float32 exactly; stores round to nearest even.  load4/store4 move 4
+// consecutive elements (16 or 8 bytes, aligned to that size).
+template <class TA>
+struct ActIO;
+
+template <>
+struct ActIO<float> {
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    static __device__ __forceinline__ float load1(const float* p) { return *p; }
+    static __device__ __forceinline__ float2 load2(const float* p) {
+        return *reinterpret_cast<const float2*>(p);
+    }
+    static __device__ __forceinline__ float4 load4(const float* p) {
+        return *reinterpret_cast<const float4*>(p);
+    }
+    static __device__ __forceinline__ void store1(float* p, float v) { *p = v; }
+    static __device__ __forceinline__ void store4(float* p, const float4& v) { dw::store4(p, v); }
+};
+
+template <>
+struct ActIO<__half> {
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    static __device__ __forceinline__ float load1(const __half* p) { return __half2float(*p); }
+    static __device__ __forceinline__ float2 load2(const __half* p) {
+        return __half22float2(*reinterpret_cast<const __half2*>(p));
+    }
+    static __device__ __forceinline__ float4 load4(const __half* p) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+    static __device__ __forceinline__ void store1(__half* p, float v) { *p = __float2half_rn(v); }
+    static __device__ __forceinline__ void store4(__half* p, const float4& v) {
+        const __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+        uint2 raw;
+        raw.x = *reinterpret_cast<const uint32_t*>(&a);
+        raw.y = *reinterpret_cast<const uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(p) = raw;
+    }
+};
+
+template <>
+struct ActIO<__nv_bfloat16> {
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    static __device__ __forceinline__ float load1(const __nv_bfloat16* p) {
+        return __bfloat162float(*p);
+    }
+    static __device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    }
+    static __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+    static __device__ __forceinline__ void store1(__nv_bfloat16* p, float v) {
+        *p = __float2bfloat16_rn(v);
+    }
+    static __device__ __forceinline__ void store4(__nv_bfloat16* p, const float4& v) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+        uint2 raw;
+        raw.x = *reinterpret_cast<const uint32_t*>(&a);
+        raw.y = *reinterpret_cast<const uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(p) = raw;
+    }
+};
+
+// Bytes of one activation element of type `atype` (DW_F32 / DW_F16 / DW_BF16).
+inline int act_bytes(int atype) { return atype == DW_F32 ? 4 : 2; }
 
 }  // namespace dw

@@ -27,9 +27,10 @@ struct DirectArgs {
     Epilogue epi;  // forward only
 };
 
-template <int LAYOUT>
-__device__ __forceinline__ void decode(int64_t i, int64_t C, int64_t Hx, int64_t Wx, int64_t& n,
-                                       int64_t& c, int64_t& h, int64_t& w) {
+// I: index type (int32_t when every flat index fits, else int64_t; 64-bit
+// division is several times the cost of 32-bit division).
+template <int LAYOUT, class I>
+__device__ __forceinline__ void decode(I i, I C, I Hx, I Wx, I& n, I& c, I& h, I& w) {
     if (LAYOUT == DW_NHWC) {
         c = i % C; i /= C;
         w = i % Wx; i /= Wx;
@@ -41,33 +42,34 @@ __device__ __forceinline__ void decode(int64_t i, int64_t C, int64_t Hx, int64_t
     }
 }
 
-template <int LAYOUT>
-__device__ __forceinline__ int64_t offset(int64_t n, int64_t c, int64_t h, int64_t w,
-                                          int64_t C, int64_t Hx, int64_t Wx) {
+template <int LAYOUT, class I>
+__device__ __forceinline__ I offset(I n, I c, I h, I w, I C, I Hx, I Wx) {
     return LAYOUT == DW_NHWC ? ((n * Hx + h) * Wx + w) * C + c : ((n * C + c) * Hx + h) * Wx + w;
 }
 
-template <int LAYOUT>
-__global__ void __launch_bounds__(256) direct_fwd_kernel(const float* __restrict__ x,
+template <int LAYOUT, class TA, class I>
+__global__ void __launch_bounds__(256) direct_fwd_kernel(const TA* __restrict__ x,
                                                          const void* __restrict__ w,
                                                          const float* __restrict__ b,
-                                                         float* __restrict__ y, DirectArgs a) {
+                                                         TA* __restrict__ y, DirectArgs a) {
     grid_dependency_wait();
     allow_dependents();
+    const I C = I(a.C), Co = I(a.Co), M = I(a.M), H = I(a.H), W = I(a.W), Ho = I(a.Ho),
+            Wo = I(a.Wo);
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.total; i += stride) {
-        int64_t n, o, ho, wo;
-        decode<LAYOUT>(i, a.Co, a.Ho, a.Wo, n, o, ho, wo);
-        const int64_t c = o / a.M;  // the input channel output o reads
+        I n, o, ho, wo;
+        decode<LAYOUT, I>(I(i), Co, Ho, Wo, n, o, ho, wo);
+        const I c = o / M;  // the input channel output o reads
         float acc = 0.f;
-        const int64_t wbase = o * a.kH * a.kW;
+        const int64_t wbase = int64_t(o) * a.kH * a.kW;
         for (int kh = 0; kh < a.kH; ++kh) {
-            const int64_t hi = ho * a.sh + int64_t(kh) * a.dh - a.pt;
-            if (hi < 0 || hi >= a.H) continue;
+            const I hi = ho * I(a.sh) + I(kh) * I(a.dh) - I(a.pt);
+            if (hi < 0 || hi >= H) continue;
             for (int kw = 0; kw < a.kW; ++kw) {
-                const int64_t wi = wo * a.sw + int64_t(kw) * a.dw - a.pl;
-                if (wi < 0 || wi >= a.W) continue;
-                acc = fmaf(__ldg(x + offset<LAYOUT>(n, c, hi, wi, a.C, a.H, a.W)),
+                const I wi = wo * I(a.sw) + I(kw) * I(a.dw) - I(a.pl);
+                if (wi < 0 || wi >= W) continue;
+                acc = fmaf(ActIO<TA>::load1(x + offset<LAYOUT, I>(n, c, hi, wi, C, H, W)),
                            load_weight(w, a.wtype, wbase + kh * a.kW + kw), acc);
             }
         }
@@ -77,47 +79,83 @@ __global__ void __launch_bounds__(256) direct_fwd_kernel(const float* __restrict
             bn_scale_shift(a.epi, int(o), scale, shift);
             acc = epilogue_apply(acc, scale, shift, a.epi.act);
         }
-        y[i] = acc;
+        ActIO<TA>::store1(y + i, acc);
     }
 }
 
-template <int LAYOUT>
-__global__ void __launch_bounds__(256) direct_bwd_kernel(const float* __restrict__ dy,
+template <int LAYOUT, class TA, class I>
+__global__ void __launch_bounds__(256) direct_bwd_kernel(const TA* __restrict__ dy,
                                                          const void* __restrict__ w,
-                                                         float* __restrict__ dx, DirectArgs a) {
+                                                         TA* __restrict__ dx, DirectArgs a) {
     grid_dependency_wait();
     allow_dependents();
+    const I C = I(a.C), Co = I(a.Co), M = I(a.M), H = I(a.H), W = I(a.W), Ho = I(a.Ho),
+            Wo = I(a.Wo), sh = I(a.sh), sw = I(a.sw);
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.total; i += stride) {
-        int64_t n, c, hi, wi;
-        decode<LAYOUT>(i, a.C, a.H, a.W, n, c, hi, wi);
+        I n, c, hi, wi;
+        decode<LAYOUT, I>(I(i), C, H, W, n, c, hi, wi);
         float acc = 0.f;
         // every output channel of input channel c: o = c*M .. c*M + M-1
-        for (int64_t o = c * a.M; o < (c + 1) * a.M; ++o) {
-            const int64_t wbase = o * a.kH * a.kW;
+        for (I o = c * M; o < (c + 1) * M; ++o) {
+            const int64_t wbase = int64_t(o) * a.kH * a.kW;
             for (int kh = 0; kh < a.kH; ++kh) {
-                const int64_t th = hi + a.pt - int64_t(kh) * a.dh;  // = ho * sh
-                if (th < 0 || th % a.sh != 0) continue;
-                const int64_t ho = th / a.sh;
-                if (ho >= a.Ho) continue;
+                const I th = hi + I(a.pt) - I(kh) * I(a.dh);  // = ho * sh
+                if (th < 0 || th % sh != 0) continue;
+                const I ho = th / sh;
+                if (ho >= Ho) continue;
                 for (int kw = 0; kw < a.kW; ++kw) {
-                    const int64_t tw = wi + a.pl - int64_t(kw) * a.dw;  // = wo * sw
-                    if (tw < 0 || tw % a.sw != 0) continue;
-                    const int64_t wo = tw / a.sw;
-                    if (wo >= a.Wo) continue;
+                    const I tw = wi + I(a.pl) - I(kw) * I(a.dw);  // = wo * sw
+                    if (tw < 0 || tw % sw != 0) continue;
+                    const I wo = tw / sw;
+                    if (wo >= Wo) continue;
                     acc = fmaf(load_weight(w, a.wtype, wbase + kh * a.kW + kw),
-                               __ldg(dy + offset<LAYOUT>(n, o, ho, wo, a.Co, a.Ho, a.Wo)), acc);
+                               ActIO<TA>::load1(dy + offset<LAYOUT, I>(n, o, ho, wo, Co, Ho, Wo)),
+                               acc);
                 }
             }
         }
-        dx[i] = acc;
+        ActIO<TA>::store1(dx + i, acc);
     }
+}
+
+template <class TA, class I>
+cudaError_t launch_typed(const Problem& p, Op op, const void* in, const void* w, const float* b,
+                         void* out, cudaStream_t stream, dim3 grid, dim3 block,
+                         const DirectArgs& a) {
+    const TA* src = static_cast<const TA*>(in);
+    TA* dst = static_cast<TA*>(out);
+    if (op == OP_FWD)
+        return p.layout == DW_NHWC
+                   ? launch_pdl(direct_fwd_kernel<DW_NHWC, TA, I>, grid, block, 0, stream, src, w,
+                                b, dst, a)
+                   : launch_pdl(direct_fwd_kernel<DW_NCHW, TA, I>, grid, block, 0, stream, src, w,
+                                b, dst, a);
+    return p.layout == DW_NHWC
+               ? launch_pdl(direct_bwd_kernel<DW_NHWC, TA, I>, grid, block, 0, stream, src, w,
+                            dst, a)
+               : launch_pdl(direct_bwd_kernel<DW_NCHW, TA, I>, grid, block, 0, stream, src, w,
+                            dst, a);
+}
+
+template <class TA>
+cudaError_t launch_index(const Problem& p, Op op, const void* in, const void* w, const float* b,
+                         void* out, cudaStream_t stream, dim3 grid, dim3 block,
+                         const DirectArgs& a) {
+    // every flat index and intermediate (with pads and taps) inside int32?
+    const int64_t big = p.N * (p.Co > p.C ? p.Co : p.C) * (p.H > p.Ho ? p.H : p.Ho) *
+                        (p.W > p.Wo ? p.W : p.Wo);
+    const int64_t span = int64_t(p.kH) * p.dh + int64_t(p.kW) * p.dw + p.pt + p.pl +
+                         (p.H + p.W) * (p.sh + p.sw);
+    if (big < (int64_t(1) << 30) && span < (int64_t(1) << 30))
+        return launch_typed<TA, int32_t>(p, op, in, w, b, out, stream, grid, block, a);
+    return launch_typed<TA, int64_t>(p, op, in, w, b, out, stream, grid, block, a);
 }
 
 }  // namespace
 
-dw_status_t direct_launch(const Problem& p, Op op, const float* in, const void* w, const float* b,
-                          float* out, cudaStream_t stream) {
+dw_status_t direct_launch(const Problem& p, Op op, const void* in, const void* w, const float* b,
+                          void* out, cudaStream_t stream) {
     DirectArgs a;
     a.N = p.N; a.C = p.C; a.H = p.H; a.W = p.W; a.Ho = p.Ho; a.Wo = p.Wo;
     a.M = p.M; a.Co = p.Co;
@@ -131,18 +169,14 @@ dw_status_t direct_launch(const Problem& p, Op op, const float* in, const void* 
     int64_t blocks = (a.total + threads - 1) / threads;
     if (blocks > max_blocks) blocks = max_blocks;
     if (blocks < 1) blocks = 1;
-    const dim3 grid(static_cast<unsigned>(blocks));
+    const dim3 grid(static_cast<unsigned>(blocks)), block(threads);
     cudaError_t e;
-    const dim3 block(threads);
-    if (op == OP_FWD) {
-        e = p.layout == DW_NHWC
-                ? launch_pdl(direct_fwd_kernel<DW_NHWC>, grid, block, 0, stream, in, w, b, out, a)
-                : launch_pdl(direct_fwd_kernel<DW_NCHW>, grid, block, 0, stream, in, w, b, out, a);
-    } else {
-        e = p.layout == DW_NHWC
-                ? launch_pdl(direct_bwd_kernel<DW_NHWC>, grid, block, 0, stream, in, w, out, a)
-                : launch_pdl(direct_bwd_kernel<DW_NCHW>, grid, block, 0, stream, in, w, out, a);
-    }
+    if (p.atype == DW_F16)
+        e = launch_index<__half>(p, op, in, w, b, out, stream, grid, block, a);
+    else if (p.atype == DW_BF16)
+        e = launch_index<__nv_bfloat16>(p, op, in, w, b, out, stream, grid, block, a);
+    else
+        e = launch_index<float>(p, op, in, w, b, out, stream, grid, block, a);
     if (e != cudaSuccess) return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }

@@ -649,12 +649,15 @@ dw_status_t launch_op(const Problem& p, Op op, const float* in, const void* w, c
 
 }  // namespace nchw
 
-dw_status_t tiled_nchw_launch(const Problem& p, Op op, const float* in, const void* w,
-                              const float* b, float* out, cudaStream_t stream, int32_t* err,
+dw_status_t tiled_nchw_launch(const Problem& p, Op op, const void* in_v, const void* w,
+                              const float* b, void* out_v, cudaStream_t stream, int32_t* err,
                               bool dry_run) {
     using namespace nchw;
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
     if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
+    if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;  // 16-bit activations: direct kernels
+    const float* in = static_cast<const float*>(in_v);
+    float* out = static_cast<float*>(out_v);
     if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
     const int64_t Win = op == OP_FWD ? p.W : p.Wo;
     if (Win % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row stride: 16-byte multiple

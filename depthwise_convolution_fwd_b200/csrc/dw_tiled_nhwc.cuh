@@ -54,7 +54,8 @@ struct VecOps<4> {
     static __device__ __forceinline__ T add(const T& a, const T& b) {
         return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
     }
-    static __device__ __forceinline__ void store(float* p, const T& v) { store4(p, v); }
+    template <class TA>
+    static __device__ __forceinline__ void store(TA* p, const T& v) { ActIO<TA>::store4(p, v); }
     template <class WT>
     static __device__ __forceinline__ T load_w(const WT* w, int64_t o, int step) {
         return make_float4(float(w[o]), float(w[o + step]), float(w[o + 2 * step]),
@@ -91,7 +92,8 @@ struct VecOps<1> {
         acc = fmaf(v, w, acc);
     }
     static __device__ __forceinline__ T add(const T& a, const T& b) { return a + b; }
-    static __device__ __forceinline__ void store(float* p, const T& v) { *p = v; }
+    template <class TA>
+    static __device__ __forceinline__ void store(TA* p, const T& v) { ActIO<TA>::store1(p, v); }
     template <class WT>
     static __device__ __forceinline__ T load_w(const WT* w, int64_t o, int) {
         return float(w[o]);
@@ -113,7 +115,7 @@ struct VecOps<1> {
 struct Args {
     const void* w;
     const float* b;
-    float* out;
+    void* out;  // elements of the configuration's activation type
     int32_t* err;
     int wtype;
     int C;
@@ -129,8 +131,11 @@ struct Args {
 // stored straight from registers).  MINB: CTAs per SM the register budget is
 // sized for.
 template <int KH_, int KW_, int S_, int D_, bool TR_, int THT_, int TWT_, int WX_, int WY_, int NS_,
-          int VEC_ = 4, int NO_ = 2, int MINB_ = 1, int CB_ = 32, int MULT_ = 1>
+          int VEC_ = 4, int NO_ = 2, int MINB_ = 1, int CB_ = 32, int MULT_ = 1,
+          class TA_ = float>
 struct Cfg {
+    using TA = TA_;  // activation element type (float, __half, __nv_bfloat16)
+    static constexpr int ESZ = sizeof(TA);
     static constexpr int CB = CB_;  // (output) channels per tile
     // channel multiplier: a tile's CB output channels read CBI = CB / MULT
     // input channels (output channel o reads input channel o / MULT)
@@ -156,18 +161,20 @@ struct Cfg {
     // rows / columns of the input window one thread reads
     static constexpr int RH = TR ? AH + (THT - 1) / S + 1 : (THT - 1) * S + (KH - 1) * D + 1;
     static constexpr int RW = TR ? AW + (TWT - 1) / S + 1 : (TWT - 1) * S + (KW - 1) * D + 1;
-    static constexpr int STAGE_BYTES = IH * IW * CBI * 4;  // one TMA load
+    static constexpr int STAGE_BYTES = IH * IW * CBI * ESZ;  // one TMA load
     static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
-    static constexpr int OUT_V = TH * TW * CV;  // output staging buffer in lane vectors
-    static constexpr int OUT_BYTES = TH * TW * CB * 4;
+    static constexpr int OUT_ELEMS = TH * TW * CB;  // output staging buffer
+    static constexpr int OUT_BYTES = OUT_ELEMS * ESZ;
     static constexpr size_t SMEM =
         size_t(NS) * STAGE_PITCH + size_t(NO) * OUT_BYTES + size_t(2 * NS) * 8 + 16;
     static_assert((WX * WY * CV) % 32 == 0, "whole consumer warps");
     static_assert(IH <= 256 && IW <= 256, "TMA box dimension limit");
     // every stage starts on a 128-byte boundary (tensor-copy destination rule)
-    static_assert(MULT > 1 || STAGE_BYTES % 128 == 0, "TMA shared-memory alignment");
-    static_assert(MULT == 1 || (!TR && VEC == 4 && CB % MULT == 0 && CBI % 4 == 0),
-                  "multiplier tiles: forward, 4-channel lanes, 16-byte input rows");
+    static_assert(MULT > 1 || ESZ < 4 || STAGE_BYTES % 128 == 0, "TMA shared-memory alignment");
+    static_assert(NO == 0 || OUT_BYTES % 128 == 0, "staging buffers on 128-byte boundaries");
+    static_assert((CBI * ESZ) % 16 == 0, "16-byte rows in the input box");
+    static_assert(MULT == 1 || (!TR && VEC == 4 && CB % MULT == 0),
+                  "multiplier tiles: forward, 4-channel lanes");
     static_assert(!TR || (THT % S == 0 && TWT % S == 0), "transposed blocks are phase aligned");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -224,14 +231,16 @@ __device__ __forceinline__ Tile decode_tile(int t, const Args& a) {
 // for a channel multiplier the input channels its 4 output channels read,
 // each repeated MULT times (MULT = 2: two channels, MULT >= 4: one).
 template <class K>
-__device__ __forceinline__ typename VecOps<K::VEC>::T load_cell(const float* p) {
+__device__ __forceinline__ typename VecOps<K::VEC>::T load_cell(const typename K::TA* p) {
+    using IO = ActIO<typename K::TA>;
     if constexpr (K::MULT == 1) {
-        return *reinterpret_cast<const typename VecOps<K::VEC>::T*>(p);
+        if constexpr (K::VEC == 4) return IO::load4(p);
+        else return IO::load1(p);
     } else if constexpr (K::MULT == 2) {
-        const float2 f = *reinterpret_cast<const float2*>(p);
+        const float2 f = IO::load2(p);
         return make_float4(f.x, f.x, f.y, f.y);
     } else {
-        const float f = *p;
+        const float f = IO::load1(p);
         return make_float4(f, f, f, f);
     }
 }
@@ -247,7 +256,8 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     using V = typename VO::T;
     constexpr int CV = K::CV;
     extern __shared__ __align__(128) unsigned char smem[];
-    V* outbuf = reinterpret_cast<V*>(smem + size_t(K::NS) * K::STAGE_PITCH);
+    using TA = typename K::TA;
+    TA* outbuf = reinterpret_cast<TA*>(smem + size_t(K::NS) * K::STAGE_PITCH);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH +
                                                  size_t(K::NO) * K::OUT_BYTES);
     uint64_t* empty = full + K::NS;
@@ -391,8 +401,8 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 
         // this thread's window: cell (r, q) holds CBI input channels; the
         // lane's 4 output channels cv*4.. read input channels (cv*4)/MULT..
-        const float* win = reinterpret_cast<const float*>(smem + size_t(s) * K::STAGE_PITCH) +
-                           (r0 * K::IW + q0) * K::CBI + (cv * K::VEC) / K::MULT;
+        const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
+                        (r0 * K::IW + q0) * K::CBI + (cv * K::VEC) / K::MULT;
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             static_for<0, K::RW>([&](auto q_) {
@@ -434,12 +444,12 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 if (tid == 0) bulk_wait_group_read<K::NO - 1>();
                 named_barrier_sync(1, K::NCT);
             }
-            V* o = outbuf + size_t(ob) * K::OUT_V + (j0 * K::TW + i0) * CV + cv;
+            TA* o = outbuf + size_t(ob) * K::OUT_ELEMS + (j0 * K::TW + i0) * K::CB + cv * K::VEC;
 #pragma unroll
             for (int j = 0; j < K::THT; ++j)
 #pragma unroll
                 for (int i = 0; i < K::TWT; ++i)
-                    o[(j * K::TW + i) * CV] = finish(acc[j][i]);
+                    VO::store(o + (j * K::TW + i) * K::CB, finish(acc[j][i]));
             fence_proxy_async_smem();
             if (named_barrier_or(1, K::NCT, !ok)) {
                 if (tid == 0) {
@@ -449,12 +459,14 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 break;
             }
             if (tid == 0) {
-                tma_store_4d(&omap, outbuf + size_t(ob) * K::OUT_V, T.cb * K::CB, T.ox0, T.oy0, T.n);
+                tma_store_4d(&omap, outbuf + size_t(ob) * K::OUT_ELEMS, T.cb * K::CB, T.ox0, T.oy0,
+                             T.n);
                 bulk_commit_group();
             }
         } else if (c < a.C) {
             const int ho0 = T.oy0 + j0, wo0 = T.ox0 + i0;
-            float* base = a.out + (int64_t(T.n) * a.Hout + ho0) * row_pitch + int64_t(wo0) * a.C + c;
+            TA* base = static_cast<TA*>(a.out) + (int64_t(T.n) * a.Hout + ho0) * row_pitch +
+                       int64_t(wo0) * a.C + c;
 #pragma unroll
             for (int j = 0; j < K::THT; ++j) {
                 const int ho = ho0 + j;
@@ -476,8 +488,8 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 
 // Launch attributes and the tensor map; `grid_cap` caps resident CTAs.
 template <class K>
-dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, const float* b,
-                   float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+dw_status_t launch(const Problem& p, Op op, const void* in, const void* w, const float* b,
+                   void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     const bool tr = op == OP_BWD_INPUT;
     if (tr != K::TR) return DW_ERR_UNSUPPORTED;
     Args a;
@@ -523,24 +535,25 @@ dw_status_t launch(const Problem& p, Op op, const float* in, const void* w, cons
 
     const int64_t Hin = tr ? p.Ho : p.H, Win = tr ? p.Wo : p.W;
     CUtensorMap map;
+    constexpr cuuint64_t E = K::ESZ;
+    constexpr CUtensorMapDataType dt = ActIO<typename K::TA>::kTma;
     const cuuint64_t dims[4] = {cuuint64_t(p.C), cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.N)};
-    const cuuint64_t strides[3] = {cuuint64_t(p.C) * 4, cuuint64_t(p.C * Win) * 4,
-                                   cuuint64_t(p.C * Win * Hin) * 4};
+    const cuuint64_t strides[3] = {cuuint64_t(p.C) * E, cuuint64_t(p.C * Win) * E,
+                                   cuuint64_t(p.C * Win * Hin) * E};
     const cuuint32_t box[4] = {K::CBI, K::IW, K::IH, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
-                          strides, box, estr) != CUDA_SUCCESS)
+    if (encode_tensor_map(&map, dt, 4, const_cast<void*>(in), dims, strides, box, estr) !=
+        CUDA_SUCCESS)
         return DW_ERR_CUDA;
     // output map: the staging buffer is a [TH][TW][32] box of the output
     CUtensorMap omap = map;
     if constexpr (K::NO > 0) {
         const cuuint64_t odims[4] = {cuuint64_t(a.C), cuuint64_t(a.Wout), cuuint64_t(a.Hout),
                                      cuuint64_t(p.N)};
-        const cuuint64_t ostrides[3] = {cuuint64_t(a.C) * 4, cuuint64_t(a.C) * a.Wout * 4,
-                                        cuuint64_t(a.C) * a.Wout * a.Hout * 4};
+        const cuuint64_t ostrides[3] = {cuuint64_t(a.C) * E, cuuint64_t(a.C) * a.Wout * E,
+                                        cuuint64_t(a.C) * a.Wout * a.Hout * E};
         const cuuint32_t obox[4] = {K::CB, K::TW, K::TH, 1};
-        if (encode_tensor_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out, odims, ostrides,
-                              obox, estr) != CUDA_SUCCESS)
+        if (encode_tensor_map(&omap, dt, 4, out, odims, ostrides, obox, estr) != CUDA_SUCCESS)
             return DW_ERR_CUDA;
     }
 
@@ -568,24 +581,117 @@ int64_t tile_count(const Problem& p, Op op) {
 // Big tiles for large problems; small tiles when the big ones would leave
 // most SMs idle.
 template <class Big, class Small>
-dw_status_t launch_pick(const Problem& p, Op op, const float* in, const void* w, const float* b,
-                        float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+dw_status_t launch_pick(const Problem& p, Op op, const void* in, const void* w, const float* b,
+                        void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     const int sms = dry_run ? 148 : sm_count(current_device());
     if (tile_count<Big>(p, op) >= 2 * int64_t(sms))
         return launch<Big>(p, op, in, w, b, out, stream, err, dry_run);
     return launch<Small>(p, op, in, w, b, out, stream, err, dry_run);
 }
 
-// Instantiation units: forward (dw_tiled_nhwc.cu), input gradient
-// (dw_tiled_nhwc_bwd.cu) and forward with a channel multiplier
-// (dw_tiled_nhwc_mult.cu).  Each returns DW_ERR_UNSUPPORTED for a shape it
-// has no configuration for.
-dw_status_t fwd_launch(const Problem& p, const float* in, const void* w, const float* b,
-                       float* out, cudaStream_t stream, int32_t* err, bool dry_run);
-dw_status_t bwd_launch(const Problem& p, const float* in, const void* w, float* out,
-                       cudaStream_t stream, int32_t* err, bool dry_run);
-dw_status_t mult_launch(const Problem& p, const float* in, const void* w, const float* b,
-                        float* out, cudaStream_t stream, int32_t* err, bool dry_run);
+// Instantiated configurations, per activation type TA
+// (KH KW S D TR | THT TWT WX WY NS [VEC NO MINB CB MULT TA]);
+// shared memory = NS input stages + NO output staging buffers <= 227 KB.
+template <class TA> using F33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4, 4, 0, 2, 32, 1, TA>;
+template <class TA> using F33s1s = Cfg<3, 3, 1, 1, false, 2, 4, 4, 2, 4, 1, 2, 2, 32, 1, TA>;
+template <class TA> using F33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4, 4, 0, 2, 32, 1, TA>;
+template <class TA> using F33d2 = Cfg<3, 3, 1, 2, false, 2, 4, 8, 4, 2, 4, 2, 1, 32, 1, TA>;
+template <class TA> using F33d3 = Cfg<3, 3, 1, 3, false, 2, 4, 8, 4, 2, 4, 2, 1, 32, 1, TA>;
+template <class TA> using F55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 2, 4, 2, 1, 32, 1, TA>;
+template <class TA> using F55s1s = Cfg<5, 5, 1, 1, false, 2, 4, 4, 2, 4, 1, 2, 2, 32, 1, TA>;
+template <class TA> using F1x3 = Cfg<1, 3, 1, 1, false, 1, 8, 16, 1, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using F1x5 = Cfg<1, 5, 1, 1, false, 1, 8, 16, 1, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using F1x7 = Cfg<1, 7, 1, 1, false, 1, 8, 16, 1, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using F1x15 = Cfg<1, 15, 1, 1, false, 1, 16, 8, 1, 4, 1, 2, 1, 32, 1, TA>;
+template <class TA> using F1x31 = Cfg<1, 31, 1, 1, false, 1, 16, 2, 1, 4, 1, 2, 1, 128, 1, TA>;
+template <class TA> using F77s1 = Cfg<7, 7, 1, 1, false, 2, 4, 4, 2, 3, 1, 2, 1, 32, 1, TA>;
+template <class TA> using B33s1 = Cfg<3, 3, 1, 1, true, 2, 4, 8, 4, 4, 4, 0, 2, 32, 1, TA>;
+template <class TA> using B33s1s = Cfg<3, 3, 1, 1, true, 2, 4, 4, 2, 4, 1, 2, 2, 32, 1, TA>;
+template <class TA> using B33s2 = Cfg<3, 3, 2, 1, true, 4, 4, 8, 4, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B33s2s = Cfg<3, 3, 2, 1, true, 2, 2, 8, 4, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B33d2 = Cfg<3, 3, 1, 2, true, 2, 4, 8, 4, 2, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B33d3 = Cfg<3, 3, 1, 3, true, 2, 4, 8, 4, 2, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B55s1 = Cfg<5, 5, 1, 1, true, 2, 4, 8, 4, 2, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B55s1s = Cfg<5, 5, 1, 1, true, 2, 4, 4, 2, 4, 1, 2, 2, 32, 1, TA>;
+template <class TA> using B1x3 = Cfg<1, 3, 1, 1, true, 1, 8, 16, 1, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B1x5 = Cfg<1, 5, 1, 1, true, 1, 8, 16, 1, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B1x7 = Cfg<1, 7, 1, 1, true, 1, 8, 16, 1, 4, 4, 2, 1, 32, 1, TA>;
+template <class TA> using B1x15 = Cfg<1, 15, 1, 1, true, 1, 16, 8, 1, 4, 1, 2, 1, 32, 1, TA>;
+template <class TA> using B1x31 = Cfg<1, 31, 1, 1, true, 1, 16, 2, 1, 4, 1, 2, 1, 128, 1, TA>;
+template <class TA> using B77s1 = Cfg<7, 7, 1, 1, true, 2, 4, 4, 2, 3, 1, 2, 1, 32, 1, TA>;
+
+template <class TA>
+dw_status_t fwd_launch_t(const Problem& p, const void* in, const void* w, const float* b,
+                         void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    const int S = p.sh, D = p.dh;
+    const Op op = OP_FWD;
+#define DW_ONE(FC) return launch<FC<TA>>(p, op, in, w, b, out, stream, err, dry_run);
+#define DW_TWO(FC, FCS) \
+    return launch_pick<FC<TA>, FCS<TA>>(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 1) DW_TWO(F33s1, F33s1s)
+    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1) DW_ONE(F33s2)
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 2) DW_ONE(F33d2)
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 3) DW_ONE(F33d3)
+    if (p.kH == 5 && p.kW == 5 && S == 1 && D == 1) DW_TWO(F55s1, F55s1s)
+    if (p.kH == 7 && p.kW == 7 && S == 1 && D == 1) DW_ONE(F77s1)
+    if (p.kH == 1 && S == 1 && D == 1) {
+        if (p.kW == 3) DW_ONE(F1x3)
+        if (p.kW == 5) DW_ONE(F1x5)
+        if (p.kW == 7) DW_ONE(F1x7)
+        if (p.kW == 15) DW_ONE(F1x15)
+        if (p.kW == 31) DW_ONE(F1x31)
+    }
+#undef DW_ONE
+#undef DW_TWO
+    return DW_ERR_UNSUPPORTED;
+}
+
+template <class TA>
+dw_status_t bwd_launch_t(const Problem& p, const void* in, const void* w, void* out,
+                         cudaStream_t stream, int32_t* err, bool dry_run) {
+    const int S = p.sh, D = p.dh;
+    const Op op = OP_BWD_INPUT;
+#define DW_ONE(BC) return launch<BC<TA>>(p, op, in, w, nullptr, out, stream, err, dry_run);
+#define DW_TWO(BC, BCS) \
+    return launch_pick<BC<TA>, BCS<TA>>(p, op, in, w, nullptr, out, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 1) DW_TWO(B33s1, B33s1s)
+    if (p.kH == 3 && p.kW == 3 && S == 2 && D == 1) DW_TWO(B33s2, B33s2s)
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 2) DW_ONE(B33d2)
+    if (p.kH == 3 && p.kW == 3 && S == 1 && D == 3) DW_ONE(B33d3)
+    if (p.kH == 5 && p.kW == 5 && S == 1 && D == 1) DW_TWO(B55s1, B55s1s)
+    if (p.kH == 7 && p.kW == 7 && S == 1 && D == 1) DW_ONE(B77s1)
+    if (p.kH == 1 && S == 1 && D == 1) {
+        if (p.kW == 3) DW_ONE(B1x3)
+        if (p.kW == 5) DW_ONE(B1x5)
+        if (p.kW == 7) DW_ONE(B1x7)
+        if (p.kW == 15) DW_ONE(B1x15)
+        if (p.kW == 31) DW_ONE(B1x31)
+    }
+#undef DW_ONE
+#undef DW_TWO
+    return DW_ERR_UNSUPPORTED;
+}
+
+// Instantiation units, each compiled on its own: the forward for float32
+// (dw_tiled_nhwc.cu, also the family's dispatcher), the input gradient for
+// float32 (dw_tiled_nhwc_bwd.cu), both calls for float16 and bfloat16
+// activations (dw_tiled_nhwc_f16.cu, dw_tiled_nhwc_bf16.cu) and the forward
+// with a channel multiplier (dw_tiled_nhwc_mult.cu).  Each returns
+// DW_ERR_UNSUPPORTED for a shape it has no configuration for.
+dw_status_t fwd_launch_f32(const Problem& p, const void* in, const void* w, const float* b,
+                           void* out, cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t bwd_launch_f32(const Problem& p, const void* in, const void* w, void* out,
+                           cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t fwd_launch_f16(const Problem& p, const void* in, const void* w, const float* b,
+                           void* out, cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t bwd_launch_f16(const Problem& p, const void* in, const void* w, void* out,
+                           cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t fwd_launch_bf16(const Problem& p, const void* in, const void* w, const float* b,
+                            void* out, cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t bwd_launch_bf16(const Problem& p, const void* in, const void* w, void* out,
+                            cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t mult_launch(const Problem& p, const void* in, const void* w, const float* b,
+                        void* out, cudaStream_t stream, int32_t* err, bool dry_run);
 
 }  // namespace nhwc
 }  // namespace dw

@@ -18,8 +18,8 @@ template <int M>
 using M55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 2, 4, 2, 1, 32, M>;
 
 template <int M>
-dw_status_t mult_pick(const Problem& p, const float* in, const void* w, const float* b,
-                      float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+dw_status_t mult_pick(const Problem& p, const void* in, const void* w, const float* b,
+                      void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     const Op op = OP_FWD;
     if (p.kH == 3 && p.kW == 3 && p.sh == 1 && p.dh == 1)
         return launch<M33s1<M>>(p, op, in, w, b, out, stream, err, dry_run);
@@ -30,8 +30,8 @@ dw_status_t mult_pick(const Problem& p, const float* in, const void* w, const fl
     return DW_ERR_UNSUPPORTED;
 }
 
-dw_status_t mult_launch(const Problem& p, const float* in, const void* w, const float* b,
-                        float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+dw_status_t mult_launch(const Problem& p, const void* in, const void* w, const float* b,
+                        void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     if (p.M == 2) return mult_pick<2>(p, in, w, b, out, stream, err, dry_run);
     if (p.M == 4) return mult_pick<4>(p, in, w, b, out, stream, err, dry_run);
     return DW_ERR_UNSUPPORTED;

@@ -20,7 +20,7 @@ _lib = None
  DW_ERR_DEVICE_TIMEOUT, DW_ERR_TOO_LARGE) = range(7)
 DW_NOALLOC_SCRATCH_BYTES = 16 << 20
 DW_NHWC, DW_NCHW = 0, 1
-DW_F32, DW_F16 = 0, 1
+DW_F32, DW_F16, DW_BF16 = 0, 1, 2
 DW_PAD_EXPLICIT, DW_PAD_SAME = 0, 1
 DW_ALGO_AUTO, DW_ALGO_DIRECT, DW_ALGO_TILED = 0, 1, 2
 DW_ACT_NONE, DW_ACT_RELU, DW_ACT_RELU6, DW_ACT_SILU = 0, 1, 2, 3
@@ -47,7 +47,7 @@ class DwDesc(ctypes.Structure):
                 ("pad_bottom", ctypes.c_int32), ("pad_left", ctypes.c_int32),
                 ("pad_right", ctypes.c_int32), ("layout", ctypes.c_int32),
                 ("wtype", ctypes.c_int32), ("algo", ctypes.c_int32),
-                ("multiplier", ctypes.c_int32)]
+                ("multiplier", ctypes.c_int32), ("atype", ctypes.c_int32)]
 
 
 class DwError(RuntimeError):
@@ -113,10 +113,12 @@ def _pair(v) -> Tuple[int, int]:
 
 def make_desc(N: int, H: int, W: int, C: int, kH: int, kW: int, *, stride=1, dilation=1,
               padding: Union[str, int, Sequence[int]] = "same", layout: str = "nhwc",
-              wtype: str = "f32", algo: str = "auto", multiplier: int = 1) -> DwDesc:
+              wtype: str = "f32", algo: str = "auto", multiplier: int = 1,
+              atype: str = "f32") -> DwDesc:
     """Descriptor for input extents N,H,W,C.  padding: "same" (XLA rule), an
     int, a (vertical, horizontal) pair or (top, bottom, left, right);
-    multiplier: output channels per input channel (C*multiplier in all)."""
+    multiplier: output channels per input channel (C*multiplier in all);
+    atype: activation element type "f32", "f16" or "bf16"."""
     d = DwDesc()
     d.N, d.H, d.W, d.C = int(N), int(H), int(W), int(C)
     d.kH, d.kW = int(kH), int(kW)
@@ -139,6 +141,7 @@ def make_desc(N: int, H: int, W: int, C: int, kH: int, kW: int, *, stride=1, dil
     d.wtype = {"f32": DW_F32, "f16": DW_F16}[wtype]
     d.algo = _ALGOS[algo]
     d.multiplier = int(multiplier)
+    d.atype = {"f32": DW_F32, "f16": DW_F16, "bf16": DW_BF16}[atype]
     return d
 
 
@@ -226,11 +229,16 @@ def dwconv2d_bwd_weight_workspace_size(desc: DwDesc) -> int:
 
 # ------------------------------------------------------------ tensor calls --
 
-def _check_act(t: torch.Tensor, name: str):
+_ATYPES = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}
+
+
+def _check_act(t: torch.Tensor, name: str, dtype: Optional[torch.dtype] = None):
     if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
         raise TypeError(f"{name} must be a CUDA tensor")
-    if t.dtype != torch.float32:
-        raise TypeError(f"{name} must be float32, got {t.dtype}")
+    if t.dtype not in _ATYPES:
+        raise TypeError(f"{name} must be float32, float16 or bfloat16, got {t.dtype}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} like the other activations, got {t.dtype}")
     if t.dim() != 4 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous 4-D tensor")
 
@@ -290,13 +298,13 @@ def dwconv2d_fwd(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tensor] = N
         if b.device != x.device or b.dtype != torch.float32 or b.numel() != Co or not b.is_contiguous():
             raise ValueError("b must be a contiguous float32 CUDA tensor of C*multiplier elements")
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, wtype=wt, algo=algo, multiplier=M)
+                     layout=layout, wtype=wt, algo=algo, multiplier=M, atype=_ATYPES[x.dtype])
     Ho, Wo = dwconv2d_out_shape(desc)
     shape = (N, Ho, Wo, Co) if desc.layout == DW_NHWC else (N, Co, Ho, Wo)
     if out is None:
-        out = torch.empty(shape, device=x.device, dtype=torch.float32)
+        out = torch.empty(shape, device=x.device, dtype=x.dtype)
     else:
-        _check_act(out, "out")
+        _check_act(out, "out", x.dtype)
         if tuple(out.shape) != shape or out.device != x.device:
             raise ValueError(f"out must have shape {shape} on {x.device}")
     with torch.cuda.device(x.device):
@@ -342,13 +350,13 @@ def dwconv2d_fwd_bn_act(x: torch.Tensor, w: torch.Tensor, b: Optional[torch.Tens
     if act not in _ACTS:
         raise ValueError(f"act must be one of {sorted(_ACTS)}")
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, wtype=wt, algo=algo, multiplier=M)
+                     layout=layout, wtype=wt, algo=algo, multiplier=M, atype=_ATYPES[x.dtype])
     Ho, Wo = dwconv2d_out_shape(desc)
     shape = (N, Ho, Wo, Co) if desc.layout == DW_NHWC else (N, Co, Ho, Wo)
     if out is None:
-        out = torch.empty(shape, device=x.device, dtype=torch.float32)
+        out = torch.empty(shape, device=x.device, dtype=x.dtype)
     else:
-        _check_act(out, "out")
+        _check_act(out, "out", x.dtype)
         if tuple(out.shape) != shape or out.device != x.device:
             raise ValueError(f"out must have shape {shape} on {x.device}")
     with torch.cuda.device(x.device):
@@ -377,15 +385,15 @@ def dwconv2d_bwd_input(dy: torch.Tensor, w: torch.Tensor, input_hw: Tuple[int, i
     C = Co // M
     w, kH, kW, wt = _weights(w, Co, dy.device)
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, wtype=wt, algo=algo, multiplier=M)
+                     layout=layout, wtype=wt, algo=algo, multiplier=M, atype=_ATYPES[dy.dtype])
     if dwconv2d_out_shape(desc) != (Ho, Wo):
         raise ValueError(f"dy spatial extents {(Ho, Wo)} do not match the forward's "
                          f"{dwconv2d_out_shape(desc)}")
     shape = (N, H, W, C) if desc.layout == DW_NHWC else (N, C, H, W)
     if out is None:
-        out = torch.empty(shape, device=dy.device, dtype=torch.float32)
+        out = torch.empty(shape, device=dy.device, dtype=dy.dtype)
     else:
-        _check_act(out, "out")
+        _check_act(out, "out", dy.dtype)
         if tuple(out.shape) != shape or out.device != dy.device:
             raise ValueError(f"out must have shape {shape} on {dy.device}")
     with torch.cuda.device(dy.device):
@@ -407,7 +415,7 @@ def dwconv2d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel_hw: Tuple[int,
     tensor of at least dwconv2d_bwd_weight_workspace_size bytes) is allocated
     when not given."""
     _check_act(x, "x")
-    _check_act(dy, "dy")
+    _check_act(dy, "dy", x.dtype)
     if dy.device != x.device:
         raise ValueError("x and dy must be on the same device")
     kH, kW = (int(v) for v in kernel_hw)
@@ -419,7 +427,7 @@ def dwconv2d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel_hw: Tuple[int,
     if Co < C or Co % C != 0:
         raise ValueError(f"dy must have C*multiplier channels for C={C}, got {Co}")
     desc = make_desc(N, H, W, C, kH, kW, stride=stride, dilation=dilation, padding=padding,
-                     layout=layout, algo=algo, multiplier=Co // C)
+                     layout=layout, algo=algo, multiplier=Co // C, atype=_ATYPES[x.dtype])
     Ho, Wo = dwconv2d_out_shape(desc)
     want = (N, Ho, Wo, Co) if desc.layout == DW_NHWC else (N, Co, Ho, Wo)
     if tuple(dy.shape) != want:

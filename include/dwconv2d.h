@@ -80,7 +80,7 @@ enum {
 };
 
 enum { DW_NHWC = 0, DW_NCHW = 1 };                 /* dw_desc_t.layout   */
-enum { DW_F32 = 0, DW_F16 = 1 };                   /* dw_desc_t.wtype    */
+enum { DW_F32 = 0, DW_F16 = 1, DW_BF16 = 2 };      /* .wtype (F32/F16), .atype */
 enum { DW_PAD_EXPLICIT = 0, DW_PAD_SAME = 1 };     /* dw_desc_t.pad_mode */
 enum { DW_ALGO_AUTO = 0, DW_ALGO_DIRECT = 1, DW_ALGO_TILED = 2 }; /* .algo */
 /* activation of dwconv2d_fwd_bn_act: identity, max(u,0), min(max(u,0),6),
@@ -107,6 +107,12 @@ enum { DW_ACT_NONE = 0, DW_ACT_RELU = 1, DW_ACT_RELU6 = 2, DW_ACT_SILU = 3 };
  * "Incorrect stableHLO for grouped convolution gradient", a conv from 4 to
  * 8 channels with groups = 4).  Then w is [C*M,kH,kW], b [C*M], y and dy
  * have C*M channels, x and dx have C; every entry point applies it.
+ * atype: element type of the activations x, y, dy and dx: DW_F32 (0, the
+ * default), DW_F16 or DW_BF16.  16-bit activations are widened to float32
+ * exactly, every sum is formed in float32 exactly as for DW_F32, and each
+ * result is rounded once (to nearest even) to atype; the weight gradient's
+ * dW and db, bias and batch-norm statistics stay float32.  Extends the
+ * pages' f16 weights to the activations.
  */
 typedef struct dw_desc {
     int64_t N, H, W, C;
@@ -119,6 +125,7 @@ typedef struct dw_desc {
     int32_t wtype;
     int32_t algo;
     int32_t multiplier;
+    int32_t atype;
 } dw_desc_t;
 
 /* Output extents Ho, Wo of the forward for `desc` (host only, no CUDA call).
@@ -130,17 +137,17 @@ DW_API dw_status_t dwconv2d_resolved_pads(const dw_desc_t* desc, int32_t pads[4]
 
 /*
  * Forward: y = depthwise(x; w) + b.
- *   x: [N,H,W,C] or [N,C,H,W] float32, read only.
+ *   x: [N,H,W,C] or [N,C,H,W] of desc->atype (float32 by default), read only.
  *   w: [C,kH,kW] float32 or float16 (desc->wtype), read only.
  *   b: [C] float32 or NULL, read only.
- *   y: [N,Ho,Wo,C] or [N,C,Ho,Wo] float32, every element written.
+ *   y: [N,Ho,Wo,C] or [N,C,Ho,Wo] of desc->atype, every element written.
  * y must not overlap x, w or b (DW_ERR_ALIAS).
  * Page: LeanMlir Depthwise, "Depthwise conv2d forward"; strided forms
  * "Stride-2 SAME" / "Stride-2 XLA-SAME depthwise conv" (computed directly at
  * the sampled positions, never as a decimated stride-1 pass).
  */
-DW_API dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const float* x, const void* w,
-                         const float* b, float* y, void* stream);
+DW_API dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const void* x, const void* w,
+                                const float* b, void* y, void* stream);
 
 /*
  * Forward with a fused epilogue: y = act(BN(depthwise(x; w) + b)), where BN
@@ -166,34 +173,35 @@ DW_API dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const float* x, const voi
  * depthwise conv + batch-norm emitter; the pages do not spell the
  * normalisation out, and the inference-mode form above is the reading taken.
  */
-DW_API dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const float* x, const void* w,
+DW_API dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const void* x, const void* w,
                                        const float* b, const float* gamma, const float* beta,
                                        const float* mean, const float* var, float eps,
-                                       int32_t act, float* y, void* stream);
+                                       int32_t act, void* y, void* stream);
 
 /*
  * Input gradient: dx = J^T dy for the forward of `desc` (bias plays no part).
- *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] float32, read only.
+ *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] of desc->atype, read only.
  *   w:  [C,kH,kW] float32 or float16, read only.
- *   dx: [N,H,W,C] or [N,C,H,W] float32, every element written (positions no
+ *   dx: [N,H,W,C] or [N,C,H,W] of desc->atype, every element written (positions no
  *       output reads get 0; nothing is accumulated into previous contents).
  * dx must not overlap dy or w (DW_ERR_ALIAS).
  * Page: LeanMlir Depthwise, "Closed-form input gradient ... direct formula",
  * its reversed-kernel form, and the stride-2 / XLA-SAME input-VJP sections
  * (the forward's actual low pad is used, never a symmetric one).
  */
-DW_API dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy,
-                               const void* w, float* dx, void* stream);
+DW_API dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const void* dy, const void* w,
+                                      void* dx, void* stream);
 
 /*
  * Weight and bias gradients of the forward of `desc`:
  *   dW[c,kh,kw] = sum_{n,ho,wo} dy[n,ho,wo,c] * X(n, ho*sh + kh*dh - pt,
  *                                                 wo*sw + kw*dw - pl, c)
  *   db[c]       = sum_{n,ho,wo} dy[n,ho,wo,c]
- *   x:  [N,H,W,C] or [N,C,H,W] float32, read only.
- *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] float32, read only.
+ *   x:  [N,H,W,C] or [N,C,H,W] of desc->atype, read only.
+ *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] of desc->atype, read only.
  *   dw: [C,kH,kW] float32, every element written (also when desc->wtype is
- *       DW_F16: gradients are produced in float32).
+ *       DW_F16 or the activations are 16-bit: gradients are produced in
+ *       float32).
  *   db: [C] float32 or NULL (then the bias gradient is not produced).
  *   workspace: device memory of at least dwconv2d_bwd_weight_workspace_size()
  *       bytes, caller-owned; its contents on entry do not matter and are
@@ -207,7 +215,7 @@ DW_API dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const float* dy,
  * - closed-form formula" and the stride-2 / XLA-SAME weight and bias VJP
  * sections.
  */
-DW_API dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const float* x, const float* dy,
+DW_API dw_status_t dwconv2d_bwd_weight(const dw_desc_t* desc, const void* x, const void* dy,
                                        float* dw, float* db, void* workspace,
                                        uint64_t workspace_bytes, void* stream);
 
@@ -240,8 +248,8 @@ DW_API dw_status_t dwconv2d_bwd_weight_workspace_size(const dw_desc_t* desc, uin
  *     example on two streams) race on the array: the caller must order them.
  */
 #define DW_NOALLOC_SCRATCH_BYTES (16u << 20)
-DW_API dw_status_t dwconv2d_bwd_weight_noalloc(const dw_desc_t* desc, const float* x,
-                                               const float* dy, float* dw, float* db,
+DW_API dw_status_t dwconv2d_bwd_weight_noalloc(const dw_desc_t* desc, const void* x,
+                                               const void* dy, float* dw, float* db,
                                                void* stream);
 
 /*

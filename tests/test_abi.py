@@ -81,7 +81,8 @@ BAD = [
     dict(N=0), dict(H=0), dict(W=-1), dict(C=0), dict(kH=0), dict(kW=-2),
     dict(stride_h=0), dict(stride_w=-1), dict(dil_h=0), dict(dil_w=0),
     dict(pad_mode=2), dict(pad_mode=0, pad_top=-1), dict(pad_mode=0, pad_right=-3),
-    dict(layout=2), dict(wtype=5), dict(algo=3), dict(algo=-1),
+    dict(layout=2), dict(wtype=5), dict(wtype=2), dict(atype=3), dict(atype=-1),
+    dict(algo=3), dict(algo=-1),
     dict(kH=9, pad_mode=0),  # no output row left: Ho = 0
 ]
 
@@ -247,3 +248,23 @@ def test_channel_multiplier_host_checks(lib):
     x, dy, dwp, db, ws = base, base + (1 << 24), base + (2 << 24), base + (3 << 24), base + (4 << 24)
     assert dw.bwd_weight_raw(d, x, dy, dwp, dwp + 8 * 9 * 4 - 4, ws, need, 0) == dw.DW_ERR_ALIAS
     assert dw.dwconv2d_query_algo(d, 2, x, dy, dwp) == dw.DW_ALGO_DIRECT
+
+
+def test_half_activation_host_checks(lib):
+    # 16-bit activations: buffer sizes use 2-byte elements (x and y 512 B here)
+    base = 1 << 40
+    w = base + (1 << 20)
+    for at in (dw.DW_F16, dw.DW_BF16):
+        d = dw.make_desc(1, 8, 8, 4, 3, 3)
+        d.atype = at
+        assert dw.dwconv2d_query_algo(d, 0, base, w, base + 512) > 0        # adjacent: fine
+        assert dw.fwd_raw(d, base, w, None, base + 510, 0) == dw.DW_ERR_ALIAS
+        # C = 4 rows are 8 bytes: no 16-byte TMA rows, so the direct kernel
+        assert dw.dwconv2d_query_algo(d, 0, base, w, base + 512) == dw.DW_ALGO_DIRECT
+        d8 = dw.make_desc(1, 8, 8, 8, 3, 3)
+        d8.atype = at
+        assert dw.dwconv2d_query_algo(d8, 0, base, w, base + 1024) == dw.DW_ALGO_TILED
+        assert dw.dwconv2d_query_algo(d8, 2, base, base + 4096, w) == dw.DW_ALGO_TILED
+        dn = dw.make_desc(1, 8, 8, 8, 3, 3, layout="nchw")
+        dn.atype = at
+        assert dw.dwconv2d_query_algo(dn, 0, base, w, base + 1024) == dw.DW_ALGO_DIRECT
