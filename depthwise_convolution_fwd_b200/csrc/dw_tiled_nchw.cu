@@ -1,679 +1,36 @@
-// NCHW tiled kernels (stride 1): W innermost, TMA halo tiles, persistent CTAs.
-//
-// Each (n, c) plane is an independent image with its own filter (page
-// "LeanMlir Proofs/Architectures/Depthwise", comparison with regular conv2d:
-// no cross-channel mixing).  Lanes run along W: a thread owns 4 consecutive
-// outputs of a row (one float4) and THT rows, so a warp covers 128 columns
-// with 16-byte accesses on both the shared-memory reads and the global
-// stores.  For kH > 1 a CTA tile is TH x 128 outputs of one plane and its
-// input halo [TH + (kH-1)D][IWB] comes in one TMA load; for kH = 1 (the long
-// 1-D kernels) a tile is one row of 128 outputs in WY consecutive channels and
-// the TMA box spans those channels instead of rows.  TMA boxes must start on a
-// 16-byte boundary, so the box starts REM = (-pl) mod 4 columns left of the
-// first input column a tile needs; REM is a template parameter and every
-// thread's window is read as aligned float4s and indexed at compile time.
-// Taps sit in registers (per thread: the filter of its plane), streamed in
-// kh-major, kw-minor order per output.
-//
-// Modes: forward (y from x, pads pt/pl); reversed (input gradient at stride
-// 1: dx from dy with the reversed filter and the complementary pads
-// (kH-1)D - pt, (kW-1)D - pl; "Closed-form input gradient", reversed-kernel
-// form).
-#include <climits>
-#include <type_traits>
-
-#include "dw_common.cuh"
+// NCHW tiled kernels: the family's dispatcher and the float32 instantiations
+// (the kernels, configurations and launch code are in dw_tiled_nchw.cuh).
+#include "dw_tiled_nchw.cuh"
 
 namespace dw {
 namespace nchw {
 
-struct Args {
-    const void* w;
-    const float* b;
-    float* out;
-    int32_t* err;
-    int wtype;
-    int N, C, Hout, Wout;
-    int pt, pl;  // effective low pads of the correlation this kernel runs
-    FastDiv tiles_x, tiles_y, tiles_c;
-    int ntiles;
-    Epilogue epi;  // used by the EPI instantiations only
-};
-
-template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
-          int MINB_ = 1>
-struct Cfg {
-    static constexpr int MINB = MINB_;  // CTAs per SM the register budget is sized for
-    static constexpr int KH = KH_, KW = KW_, D = D_, REM = REM_;
-    static constexpr bool REV = REV_;
-    static constexpr bool ROWS = KH == 1;  // 1-D: thread rows are channels
-    static constexpr int THT = ROWS ? 1 : THT_, WX = WX_, WY = WY_, NS = NS_;
-    static constexpr int NCW = WX * WY / 32;  // consumer warps
-    static constexpr int NT = WX * WY + 32;   // + one producer warp
-    static constexpr int TW = 4 * WX;
-    static constexpr int TH = ROWS ? 1 : THT * WY;
-    static constexpr int IH = ROWS ? 1 : TH + (KH - 1) * D;
-    static constexpr int IWB = (REM + TW + (KW - 1) * D + 3) / 4 * 4;
-    static constexpr int BOXH = IH;
-    static constexpr int BOXC = ROWS ? WY : 1;
-    // bytes one TMA box delivers, and the stage pitch: every stage must start
-    // on a 128-byte boundary (shared-memory destination rule of tensor copies)
-    static constexpr int STAGE_BYTES = IWB * IH * BOXC * 4;
-    static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
-    static constexpr int STAGE_FLOATS = STAGE_PITCH / 4;
-    static constexpr int RH = THT + (KH - 1) * D;           // window rows
-    static constexpr int NV = (REM + 3 + (KW - 1) * D) / 4 + 1;  // float4 per window row
-    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NS) * 8 + 16;
-    static_assert((WX * WY) % 32 == 0, "whole consumer warps");
-    static_assert(IWB <= 256 && IH <= 256 && BOXC <= 256, "TMA box dimension limit");
-    static_assert(STAGE_PITCH % 128 == 0 && (IWB * 4) % 16 == 0, "TMA alignment");
-    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-};
-
-
-// tile t -> (tx, ty or output row h, plane or channel group, n)
-template <class K>
-__device__ __forceinline__ void decode_tile(int t, const Args& a, int& tx, int& ty, int& c,
-                                            int& n) {
-    int q = fast_div(t, a.tiles_x);
-    tx = t - q * a.tiles_x.d;
-    int r = fast_div(q, a.tiles_y);
-    ty = q - r * a.tiles_y.d;  // ROWS: output row h
-    n = fast_div(r, a.tiles_c);
-    c = r - n * a.tiles_c.d;   // ROWS: channel group; else channel
-}
-
-// EPI: kNoEpilogue, or the activation of the fused batch-norm / activation
-// epilogue of the forward.
-template <class K, int EPI>
-__global__ void __launch_bounds__(K::NT, K::MINB)
-    tiled_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
-    static_assert(EPI == kNoEpilogue || !K::REV, "the epilogue belongs to the forward");
-    extern __shared__ __align__(128) unsigned char smem[];
-    float* stages = reinterpret_cast<float*>(smem);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH);
-    uint64_t* empty = full + K::NS;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    // contiguous range of tiles for this CTA: neighbouring tiles share a
-    // plane (filter stays in registers) and their halos (L2 hits)
-    const int t_begin = int((int64_t(blockIdx.x) * a.ntiles) / gridDim.x);
-    const int t_end = int((int64_t(blockIdx.x + 1) * a.ntiles) / gridDim.x);
-
-    if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < K::NS; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], K::NCW);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-    grid_dependency_wait();
-    allow_dependents();
-
-    if (warp == K::NCW) {
-        // ---------------- producer warp: one lane issues every TMA load ----
-        if (lane == 0) {
-            prefetch_tensor_map(&tmap);
-            int k = 0;
-            bool ok = true;
-            for (int t = t_begin; t < t_end; ++t, ++k) {
-                const int s = k % K::NS;
-                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                int tx, ty, c, n;
-                decode_tile<K>(t, a, tx, ty, c, n);
-                const int ix0 = tx * K::TW - a.pl - K::REM;
-                float* dst = stages + size_t(s) * K::STAGE_FLOATS;
-                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
-                if constexpr (K::ROWS)
-                    tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
-                else
-                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH - a.pt, c, n);
-            }
-            if (!ok) {
-                *abort_flag = 1;
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
-                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
-                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
-            }
-        }
-        return;
-    }
-
-    // -------------------------- consumer warps --------------------------------
-    const int xi = tid % K::WX;
-    const int yi = tid / K::WX;
-    float wr[K::KH][K::KW];
-    float bias = 0.f;
-    int cur_key = -1;
-    bool live = false;
-    // the value stored for one output: acc + bias (-> epilogue)
-    auto finish = [&](float v) -> float {
-        if constexpr (EPI != kNoEpilogue) return activate<EPI>(v + bias);
-        else return v + bias;
-    };
-
-    int k = 0;
-    for (int t = t_begin; t < t_end; ++t, ++k) {
-        const int s = k % K::NS;
-        int tx, ty, cg, n;
-        decode_tile<K>(t, a, tx, ty, cg, n);
-        const int c = K::ROWS ? cg * K::WY + yi : cg;
-        const int key = cg + n * a.tiles_c.d;
-        if (key != cur_key) {
-            cur_key = key;
-            live = c < a.C;
-            const int64_t base = int64_t(live ? c : 0) * (K::KH * K::KW);
-#pragma unroll
-            for (int kh = 0; kh < K::KH; ++kh)
-#pragma unroll
-                for (int kw = 0; kw < K::KW; ++kw) {
-                    const int src = K::REV ? (K::KH - 1 - kh) * K::KW + (K::KW - 1 - kw)
-                                           : kh * K::KW + kw;
-                    wr[kh][kw] = live ? load_weight(a.w, a.wtype, base + src) : 0.f;
-                }
-            bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
-            if constexpr (EPI != kNoEpilogue) {
-                // fold the normalisation into the filter and the bias
-                if (live) {
-                    float sc, sh;
-                    bn_scale_shift(a.epi, c, sc, sh);
-#pragma unroll
-                    for (int kh = 0; kh < K::KH; ++kh)
-#pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] *= sc;
-                    bias = fmaf(bias, sc, sh);
-                }
-            }
-        }
-
-        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
-            if (lane == 0) {
-                *abort_flag = 1;
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
-            }
-            break;
-        }
-
-        float acc[K::THT][4];
-#pragma unroll
-        for (int j = 0; j < K::THT; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-
-        const int row0 = K::ROWS ? yi : yi * K::THT;
-        const float4* win = reinterpret_cast<const float4*>(stages + size_t(s) * K::STAGE_FLOATS +
-                                                            size_t(row0) * K::IWB) + xi;
-        static_for<0, K::RH>([&](auto r_) {
-            constexpr int r = decltype(r_)::value;
-            float v[4 * K::NV];
-#pragma unroll
-            for (int u = 0; u < K::NV; ++u) {
-                const float4 f = win[r * (K::IWB / 4) + u];
-                v[4 * u] = f.x;
-                v[4 * u + 1] = f.y;
-                v[4 * u + 2] = f.z;
-                v[4 * u + 3] = f.w;
-            }
-            static_for<0, K::THT>([&](auto j_) {
-                constexpr int j = decltype(j_)::value;
-                constexpr int khn = r - j;
-                if constexpr (khn >= 0 && khn % K::D == 0 && khn / K::D < K::KH) {
-                    constexpr int kh = khn / K::D;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw)
-                            acc[j][i] = fmaf(v[K::REM + i + kw * K::D], wr[kh][kw], acc[j][i]);
-                }
-            });
-        });
-
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-
-        if (live) {
-            const int wo0 = tx * K::TW + 4 * xi;
-#pragma unroll
-            for (int j = 0; j < K::THT; ++j) {
-                const int ho = K::ROWS ? ty : ty * K::TH + row0 + j;
-                if (ho >= a.Hout) continue;
-                float* dst = a.out + ((int64_t(n) * a.C + c) * a.Hout + ho) * a.Wout + wo0;
-                const float4 v = make_float4(finish(acc[j][0]), finish(acc[j][1]),
-                                             finish(acc[j][2]), finish(acc[j][3]));
-                if ((a.Wout & 3) == 0 && wo0 + 3 < a.Wout) {
-                    store4(dst, v);
-                } else {
-                    if (wo0 < a.Wout) dst[0] = v.x;
-                    if (wo0 + 1 < a.Wout) dst[1] = v.y;
-                    if (wo0 + 2 < a.Wout) dst[2] = v.z;
-                    if (wo0 + 3 < a.Wout) dst[3] = v.w;
-                }
-            }
-        }
-    }
-}
-
-template <class K>
-dw_status_t launch(const Problem& p, const float* in, const void* w, const float* b, float* out,
-                   cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff, int pl_eff) {
-    const int64_t Hin = K::REV ? p.Ho : p.H, Win = K::REV ? p.Wo : p.W;
-    Args a;
-    a.w = w;
-    a.b = K::REV ? nullptr : b;
-    a.out = out;
-    a.err = err;
-    a.wtype = p.wtype;
-    a.N = static_cast<int>(p.N);
-    a.C = static_cast<int>(p.C);
-    a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
-    a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
-    a.pt = pt_eff;
-    a.pl = pl_eff;
-    const int64_t tx = (a.Wout + K::TW - 1) / K::TW;
-    const int64_t ty = K::ROWS ? a.Hout : (a.Hout + K::TH - 1) / K::TH;
-    const int64_t tc = K::ROWS ? (p.C + K::WY - 1) / K::WY : p.C;
-    const int64_t nt = tx * ty * tc * p.N;
-    if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
-    a.tiles_x = make_fastdiv(static_cast<int>(tx));
-    a.tiles_y = make_fastdiv(static_cast<int>(ty));
-    a.tiles_c = make_fastdiv(static_cast<int>(tc));
-    a.ntiles = static_cast<int>(nt);
-    a.epi = K::REV ? Epilogue{} : p.epi;
-    if (dry_run) return DW_OK;
-
-    const int ev = epilogue_variant(a.epi);
-    void (*kern)(CUtensorMap, Args) = tiled_kernel<K, kNoEpilogue>;
-    if constexpr (!K::REV) {
-        if (ev == DW_ACT_NONE) kern = tiled_kernel<K, DW_ACT_NONE>;
-        if (ev == DW_ACT_RELU) kern = tiled_kernel<K, DW_ACT_RELU>;
-        if (ev == DW_ACT_RELU6) kern = tiled_kernel<K, DW_ACT_RELU6>;
-        if (ev == DW_ACT_SILU) kern = tiled_kernel<K, DW_ACT_SILU>;
-    }
-    static LaunchCache cache[5];
-    const int dev = current_device();
-    const int occ = prepare_kernel(reinterpret_cast<const void*>(kern), K::NT, K::SMEM,
-                                   cache[ev + 1], dev);
-    if (occ < 1) return DW_ERR_CUDA;
-
-    CUtensorMap map;
-    const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.C), cuuint64_t(p.N)};
-    const cuuint64_t strides[3] = {cuuint64_t(Win) * 4, cuuint64_t(Win * Hin) * 4,
-                                   cuuint64_t(Win * Hin * p.C) * 4};
-    const cuuint32_t box[4] = {K::IWB, K::BOXH, K::BOXC, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
-                          strides, box, estr) != CUDA_SUCCESS)
-        return DW_ERR_CUDA;
-    int64_t grid = int64_t(sm_count(dev)) * occ;
-    if (grid > a.ntiles) grid = a.ntiles;
-    if (launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream, map,
-                   a) != cudaSuccess)
-        return DW_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
-}
-
-// ---------------------------------------------------------------------------
-// Channel-lane kernel for 1 x kW filters (the long 1-D kernels): one TMA box
-// is 32 channel rows x the W halo of one output row; lane = channel row,
-// warp = W strip, each thread computes TWT consecutive outputs of its own
-// channel with its kW taps in registers, streaming its window from shared
-// memory once.  The stage row pitch IWB is chosen with IWB/4 odd, so the
-// 32 lanes' 16-byte reads (32 different rows, same column) fall in distinct
-// bank groups and never conflict.  Results leave through a per-warp TMA
-// store: each warp stages its 32-row x TWT-column block in its own
-// double-buffered slot and one lane issues the bulk store (the tensor engine
-// does the 32-row scatter); when the output row pitch is not a multiple of
-// 16 bytes they are stored from registers instead.
-template <int KW_, bool REV_, int REM_, int TWT_, int NCW_, int NS_>
-struct ClCfg {
-    static constexpr int KW = KW_, REM = REM_, TWT = TWT_, NCW = NCW_, NS = NS_;
-    static constexpr bool REV = REV_;
-    static constexpr int CH = 32;  // channel rows per tile (lanes)
-    static constexpr int NT = NCW * 32 + 32;
-    static constexpr int TW = TWT * NCW;
-    static constexpr int IWB0 = (REM + TW + (KW - 1) + 3) / 4 * 4;
-    static constexpr int IWB = (IWB0 / 4) % 2 == 1 ? IWB0 : IWB0 + 4;
-    static constexpr int STAGE_BYTES = IWB * CH * 4;
-    static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
-    static constexpr int STAGE_FLOATS = STAGE_PITCH / 4;
-    static constexpr int NV = (REM + TWT + KW - 1 + 3) / 4;  // float4 per thread window
-    static constexpr int OUT_FLOATS = CH * TWT;  // one warp's staging slot
-    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NCW) * OUT_FLOATS * 4 +
-                                   size_t(2 * NS) * 8 + 16;
-    static_assert(TWT % 4 == 0, "thread strips are whole float4s");
-    static_assert((OUT_FLOATS * 4) % 128 == 0, "staging slots on 128-byte boundaries");
-    static_assert(IWB <= 256, "TMA box dimension limit");
-    static_assert((IWB / 4) % 2 == 1, "conflict-free row pitch");
-    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-};
-
-template <class K, int EPI>
-__global__ void __launch_bounds__(K::NT, 1)
-    chl_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap omap,
-               const Args a, const int tma_store) {
-    static_assert(EPI == kNoEpilogue || !K::REV, "the epilogue belongs to the forward");
-    extern __shared__ __align__(128) unsigned char smem[];
-    float* stages = reinterpret_cast<float*>(smem);
-    float* outbuf = reinterpret_cast<float*>(smem + size_t(K::NS) * K::STAGE_PITCH);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH +
-                                                 size_t(2 * K::NCW) * K::OUT_FLOATS * 4);
-    uint64_t* empty = full + K::NS;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
-
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int t_begin = int((int64_t(blockIdx.x) * a.ntiles) / gridDim.x);
-    const int t_end = int((int64_t(blockIdx.x + 1) * a.ntiles) / gridDim.x);
-
-    if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < K::NS; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], K::NCW);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-    grid_dependency_wait();
-    allow_dependents();
-
-    if (warp == K::NCW) {
-        if (lane == 0) {
-            prefetch_tensor_map(&tmap);
-            int k = 0;
-            bool ok = true;
-            for (int t = t_begin; t < t_end; ++t, ++k) {
-                const int s = k % K::NS;
-                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                int tx, h, cg, n;
-                decode_tile<K>(t, a, tx, h, cg, n);
-                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
-                tma_load_4d(stages + size_t(s) * K::STAGE_FLOATS, &tmap, &full[s],
-                            tx * K::TW - a.pl - K::REM, h - a.pt, cg * K::CH, n);
-            }
-            if (!ok) {
-                *abort_flag = 1;
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
-                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
-                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
-            }
-        }
-        return;
-    }
-
-    float wr[K::KW];
-    float bias = 0.f;
-    int cur_key = -1;
-    bool live = false;
-    // the value stored for one output: acc + bias (-> epilogue)
-    auto finish = [&](float v) -> float {
-        if constexpr (EPI != kNoEpilogue) return activate<EPI>(v + bias);
-        else return v + bias;
-    };
-    int k = 0;
-    for (int t = t_begin; t < t_end; ++t, ++k) {
-        const int s = k % K::NS;
-        int tx, h, cg, n;
-        decode_tile<K>(t, a, tx, h, cg, n);
-        const int c = cg * K::CH + lane;
-        const int key = cg + n * a.tiles_c.d;
-        if (key != cur_key) {
-            cur_key = key;
-            live = c < a.C;
-            const int64_t base = int64_t(live ? c : 0) * K::KW;
-            if (a.wtype == DW_F16) {
-                const __half* wp = static_cast<const __half*>(a.w) + base;
-#pragma unroll
-                for (int kw = 0; kw < K::KW; ++kw)
-                    wr[kw] = __half2float(wp[K::REV ? K::KW - 1 - kw : kw]);
-            } else {
-                const float* wp = static_cast<const float*>(a.w) + base;
-#pragma unroll
-                for (int kw = 0; kw < K::KW; ++kw) wr[kw] = __ldg(wp + (K::REV ? K::KW - 1 - kw : kw));
-            }
-            bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
-            if constexpr (EPI != kNoEpilogue) {
-                // fold the normalisation into the filter and the bias
-                if (live) {
-                    float sc, sh;
-                    bn_scale_shift(a.epi, c, sc, sh);
-#pragma unroll
-                    for (int kw = 0; kw < K::KW; ++kw) wr[kw] *= sc;
-                    bias = fmaf(bias, sc, sh);
-                }
-            }
-        }
-
-        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
-            if (lane == 0) {
-                *abort_flag = 1;
-                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
-            }
-            break;
-        }
-
-        float acc[K::TWT];
-#pragma unroll
-        for (int i = 0; i < K::TWT; ++i) acc[i] = 0.f;
-        const float4* win = reinterpret_cast<const float4*>(stages + size_t(s) * K::STAGE_FLOATS) +
-                            lane * (K::IWB / 4) + warp * (K::TWT / 4);
-        static_for<0, K::NV>([&](auto u_) {
-            constexpr int u = decltype(u_)::value;
-            const float4 f = win[u];
-            const float e[4] = {f.x, f.y, f.z, f.w};
-            static_for<0, 4>([&](auto m_) {
-                constexpr int q = 4 * u + decltype(m_)::value - K::REM;  // window column
-                static_for<0, K::TWT>([&](auto i_) {
-                    constexpr int i = decltype(i_)::value;
-                    constexpr int kw = q - i;
-                    if constexpr (kw >= 0 && kw < K::KW)
-                        acc[i] = fmaf(e[decltype(m_)::value], wr[kw], acc[i]);
-                });
-            });
-        });
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-
-        if (tma_store) {
-            // warp-private staging slot ob: the store issued two tiles ago
-            // by this warp must have finished reading it
-            const int ob = k & 1;
-            if (k >= 2 && lane == 0) bulk_wait_group_read<1>();
-            __syncwarp();
-            float4* o = reinterpret_cast<float4*>(outbuf + size_t(2 * warp + ob) * K::OUT_FLOATS) +
-                        lane * (K::TWT / 4);
-#pragma unroll
-            for (int u = 0; u < K::TWT / 4; ++u)
-                o[u] = make_float4(finish(acc[4 * u]), finish(acc[4 * u + 1]),
-                                   finish(acc[4 * u + 2]), finish(acc[4 * u + 3]));
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_4d(&omap, outbuf + size_t(2 * warp + ob) * K::OUT_FLOATS,
-                             tx * K::TW + warp * K::TWT, h, cg * K::CH, n);
-                bulk_commit_group();
-            }
-        } else if (live && h < a.Hout) {
-            const int wo0 = tx * K::TW + warp * K::TWT;
-            float* dst = a.out + ((int64_t(n) * a.C + c) * a.Hout + h) * a.Wout + wo0;
-            const bool vec = (a.Wout & 3) == 0;
-#pragma unroll
-            for (int u = 0; u < K::TWT / 4; ++u) {
-                const float4 v = make_float4(finish(acc[4 * u]), finish(acc[4 * u + 1]),
-                                             finish(acc[4 * u + 2]), finish(acc[4 * u + 3]));
-                const int wo = wo0 + 4 * u;
-                if (vec && wo + 3 < a.Wout) {
-                    store4(dst + 4 * u, v);
-                } else {
-                    if (wo < a.Wout) dst[4 * u] = v.x;
-                    if (wo + 1 < a.Wout) dst[4 * u + 1] = v.y;
-                    if (wo + 2 < a.Wout) dst[4 * u + 2] = v.z;
-                    if (wo + 3 < a.Wout) dst[4 * u + 3] = v.w;
-                }
-            }
-        }
-    }
-    if (tma_store && lane == 0) bulk_wait_group<0>();
-}
-
-template <class K>
-dw_status_t launch_chl(const Problem& p, const float* in, const void* w, const float* b,
-                       float* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
-                       int pl_eff) {
-    const int64_t Hin = K::REV ? p.Ho : p.H, Win = K::REV ? p.Wo : p.W;
-    Args a;
-    a.w = w;
-    a.b = K::REV ? nullptr : b;
-    a.out = out;
-    a.err = err;
-    a.wtype = p.wtype;
-    a.N = static_cast<int>(p.N);
-    a.C = static_cast<int>(p.C);
-    a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
-    a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
-    a.pt = pt_eff;
-    a.pl = pl_eff;
-    const int64_t tx = (a.Wout + K::TW - 1) / K::TW;
-    const int64_t ty = a.Hout;
-    const int64_t tc = (p.C + K::CH - 1) / K::CH;
-    const int64_t nt = tx * ty * tc * p.N;
-    if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
-    a.tiles_x = make_fastdiv(static_cast<int>(tx));
-    a.tiles_y = make_fastdiv(static_cast<int>(ty));
-    a.tiles_c = make_fastdiv(static_cast<int>(tc));
-    a.ntiles = static_cast<int>(nt);
-    a.epi = K::REV ? Epilogue{} : p.epi;
-    if (dry_run) return DW_OK;
-
-    const int ev = epilogue_variant(a.epi);
-    void (*kern)(CUtensorMap, CUtensorMap, Args, int) = chl_kernel<K, kNoEpilogue>;
-    if constexpr (!K::REV) {
-        if (ev == DW_ACT_NONE) kern = chl_kernel<K, DW_ACT_NONE>;
-        if (ev == DW_ACT_RELU) kern = chl_kernel<K, DW_ACT_RELU>;
-        if (ev == DW_ACT_RELU6) kern = chl_kernel<K, DW_ACT_RELU6>;
-        if (ev == DW_ACT_SILU) kern = chl_kernel<K, DW_ACT_SILU>;
-    }
-    static LaunchCache cache[5];
-    const int dev = current_device();
-    const int occ = prepare_kernel(reinterpret_cast<const void*>(kern), K::NT, K::SMEM,
-                                   cache[ev + 1], dev);
-    if (occ < 1) return DW_ERR_CUDA;
-    CUtensorMap map;
-    const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.C), cuuint64_t(p.N)};
-    const cuuint64_t strides[3] = {cuuint64_t(Win) * 4, cuuint64_t(Win * Hin) * 4,
-                                   cuuint64_t(Win * Hin * p.C) * 4};
-    const cuuint32_t box[4] = {K::IWB, 1, K::CH, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (encode_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(in), dims,
-                          strides, box, estr) != CUDA_SUCCESS)
-        return DW_ERR_CUDA;
-    // output map for the per-warp bulk stores (row pitch must be a multiple
-    // of 16 bytes, as for every tensor map)
-    CUtensorMap omap = map;
-    int tma_store = 0;
-    if ((a.Wout & 3) == 0) {
-        const cuuint64_t odims[4] = {cuuint64_t(a.Wout), cuuint64_t(a.Hout), cuuint64_t(p.C),
-                                     cuuint64_t(p.N)};
-        const cuuint64_t ostrides[3] = {cuuint64_t(a.Wout) * 4, cuuint64_t(a.Wout) * a.Hout * 4,
-                                        cuuint64_t(a.Wout) * a.Hout * p.C * 4};
-        const cuuint32_t obox[4] = {K::TWT, 1, K::CH, 1};
-        if (encode_tensor_map(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out, odims, ostrides,
-                              obox, estr) != CUDA_SUCCESS)
-            return DW_ERR_CUDA;
-        tma_store = 1;
-    }
-    int64_t grid = int64_t(sm_count(dev)) * occ;
-    if (grid > a.ntiles) grid = a.ntiles;
-    if (launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(K::NT), K::SMEM, stream, map,
-                   omap, a, tma_store) != cudaSuccess)
-        return DW_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
-}
-
-template <int KW, bool REV, int TWT, int NCW, int NS>
-dw_status_t launch_chl_rem(const Problem& p, const float* in, const void* w, const float* b,
-                           float* out, cudaStream_t stream, int32_t* err, bool dry_run,
-                           int pt_eff, int pl_eff) {
-    switch (((-pl_eff) % 4 + 4) % 4) {
-        case 0: return launch_chl<ClCfg<KW, REV, 0, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        case 1: return launch_chl<ClCfg<KW, REV, 1, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        case 2: return launch_chl<ClCfg<KW, REV, 2, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        default: return launch_chl<ClCfg<KW, REV, 3, TWT, NCW, NS>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-    }
-}
-
-template <int KW, int TWT, int NCW, int NS>
-dw_status_t launch_chl_op(const Problem& p, Op op, const float* in, const void* w, const float* b,
-                          float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
-    if (op == OP_FWD)
-        return launch_chl_rem<KW, false, TWT, NCW, NS>(p, in, w, b, out, stream, err, dry_run,
-                                                       p.pt, p.pl);
-    return launch_chl_rem<KW, true, TWT, NCW, NS>(p, in, w, b, out, stream, err, dry_run, -p.pt,
-                                                  (KW - 1) - p.pl);
-}
-
-template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB>
-dw_status_t launch_rem(const Problem& p, const float* in, const void* w, const float* b,
-                       float* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
-                       int pl_eff) {
-    const int rem = ((-pl_eff) % 4 + 4) % 4;
-    switch (rem) {
-        case 0: return launch<Cfg<KH, KW, 1, REV, 0, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        case 1: return launch<Cfg<KH, KW, 1, REV, 1, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        case 2: return launch<Cfg<KH, KW, 1, REV, 2, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-        default: return launch<Cfg<KH, KW, 1, REV, 3, THT, WX, WY, NS, MINB>>(p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff);
-    }
-}
-
-template <int KH, int KW, int THT, int WX, int WY, int NS, int MINB = 1>
-dw_status_t launch_op(const Problem& p, Op op, const float* in, const void* w, const float* b,
-                      float* out, cudaStream_t stream, int32_t* err, bool dry_run) {
-    if (op == OP_FWD)
-        return launch_rem<KH, KW, false, THT, WX, WY, NS, MINB>(p, in, w, b, out, stream, err, dry_run,
-                                                          p.pt, p.pl);
-    return launch_rem<KH, KW, true, THT, WX, WY, NS, MINB>(p, in, w, b, out, stream, err, dry_run,
-                                                     (KH - 1) - p.pt, (KW - 1) - p.pl);
+dw_status_t nchw_launch_f32(const Problem& p, Op op, const void* in, const void* w,
+                            const float* b, void* out, cudaStream_t stream, int32_t* err,
+                            bool dry_run) {
+    return nchw_launch_t<float>(p, op, in, w, b, out, stream, err, dry_run);
 }
 
 }  // namespace nchw
 
-dw_status_t tiled_nchw_launch(const Problem& p, Op op, const void* in_v, const void* w,
-                              const float* b, void* out_v, cudaStream_t stream, int32_t* err,
+dw_status_t tiled_nchw_launch(const Problem& p, Op op, const void* in, const void* w,
+                              const float* b, void* out, cudaStream_t stream, int32_t* err,
                               bool dry_run) {
     using namespace nchw;
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
     if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
-    if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;  // 16-bit activations: direct kernels
-    const float* in = static_cast<const float*>(in_v);
-    float* out = static_cast<float*>(out_v);
     if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
     const int64_t Win = op == OP_FWD ? p.W : p.Wo;
-    if (Win % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row stride: 16-byte multiple
+    // TMA row stride: a multiple of 16 bytes
+    if ((Win * act_bytes(p.atype)) % 16 != 0) return DW_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15)
         return DW_ERR_UNSUPPORTED;
     if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.C >= INT_MAX ||
         p.Ho >= INT_MAX || p.Wo >= INT_MAX)
         return DW_ERR_UNSUPPORTED;
-    //                                                   KH  KW THT WX  WY NS
-    if (p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    if (p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 32, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    if (p.kH == 7 && p.kW == 7) return launch_op<7, 7, 4, 32, 4, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    //                                           KW TWT NCW NS
-    if (p.kH == 1 && p.kW == 15) return launch_chl_op<15, 16, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    if (p.kH == 1 && p.kW == 31) return launch_chl_op<31, 16, 8, 4>(p, op, in, w, b, out, stream, err, dry_run);
-    return DW_ERR_UNSUPPORTED;
+    if (p.atype == DW_F16) return nchw_launch_f16(p, op, in, w, b, out, stream, err, dry_run);
+    if (p.atype == DW_BF16) return nchw_launch_bf16(p, op, in, w, b, out, stream, err, dry_run);
+    return nchw_launch_f32(p, op, in, w, b, out, stream, err, dry_run);
 }
 
 }  // namespace dw

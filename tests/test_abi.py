@@ -265,6 +265,9 @@ def test_half_activation_host_checks(lib):
         d8.atype = at
         assert dw.dwconv2d_query_algo(d8, 0, base, w, base + 1024) == dw.DW_ALGO_TILED
         assert dw.dwconv2d_query_algo(d8, 2, base, base + 4096, w) == dw.DW_ALGO_TILED
-        dn = dw.make_desc(1, 8, 8, 8, 3, 3, layout="nchw")
+        dn = dw.make_desc(1, 8, 8, 8, 3, 3, layout="nchw")   # W = 8: 16-byte rows
         dn.atype = at
-        assert dw.dwconv2d_query_algo(dn, 0, base, w, base + 1024) == dw.DW_ALGO_DIRECT
+        assert dw.dwconv2d_query_algo(dn, 0, base, w, base + 1024) == dw.DW_ALGO_TILED
+        dn4 = dw.make_desc(1, 8, 12, 8, 3, 3, layout="nchw")  # W = 12: 24-byte rows
+        dn4.atype = at
+        assert dw.dwconv2d_query_algo(dn4, 0, base, w, base + 4096) == dw.DW_ALGO_DIRECT

@@ -97,7 +97,14 @@ def run_case(case, name, algo="auto"):
     torch.cuda.synchronize()
     gu.assert_close(gw.cpu().numpy(), dwr, dws, f"{case.name} {name} dW")
     gu.assert_close(gb.cpu().numpy(), dbr, dbs, f"{case.name} {name} db")
-    assert torch.equal(gw, gw32) and torch.equal(gb, gb32)
+    # same bits when both calls run the same kernel family (NCHW weight
+    # gradients of 16-bit activations use the direct kernel)
+    d16, d32 = gu.desc_of(case, kw["algo"]), gu.desc_of(case, kw["algo"])
+    d16.atype = {"f16": dw.DW_F16, "bf16": dw.DW_BF16}[name]
+    xp, gp = inp["x"].cuda(), inp["dy"].cuda()
+    if (dw.dwconv2d_query_algo(d16, 2, xp.data_ptr(), gp.data_ptr(), gw.data_ptr()) ==
+            dw.dwconv2d_query_algo(d32, 2, xp.data_ptr(), gp.data_ptr(), gw.data_ptr())):
+        assert torch.equal(gw, gw32) and torch.equal(gb, gb32)
 
 
 TILED = [
@@ -129,8 +136,43 @@ def test_tiled_half_activations(case, name):
     run_case(case, name, "tiled")
 
 
+# NCHW: every column phase of the 16-byte box start (REM 0..3, extra shift 0 or 4)
+NCHW = [
+    Case("hn_3x3_same", 2, 37, 48, 6, 3, 3, layout="nchw", seed=421),
+    Case("hn_3x3_pl0", 2, 29, 40, 5, 3, 3, padding=(0, 1, 0, 2), layout="nchw", seed=422),
+    Case("hn_3x3_pl2", 2, 31, 40, 4, 3, 3, padding=(2, 0, 2, 0), layout="nchw", seed=423),
+    Case("hn_3x3_pl3", 1, 26, 40, 6, 3, 3, padding=(1, 3, 3, 7), layout="nchw", seed=424),
+    Case("hn_3x3_pl5", 1, 21, 40, 5, 3, 3, padding=(1, 1, 5, 5), layout="nchw", seed=425),
+    Case("hn_5x5", 2, 35, 48, 5, 5, 5, layout="nchw", seed=426),
+    Case("hn_7x7", 2, 33, 32, 4, 7, 7, layout="nchw", seed=427),
+    Case("hn_1x31", 2, 2, 296, 40, 1, 31, act="normal", layout="nchw", seed=428),
+    Case("hn_1x15_pad", 2, 3, 64, 11, 1, 15, padding=(1, 0, 6, 8), act="normal",
+         layout="nchw", seed=429),
+    Case("hn_1x31_ragged", 1, 1, 296, 36, 1, 31, padding=(0, 0, 15, 14), act="normal",
+         layout="nchw", seed=430),
+]
+
+
+@pytest.mark.parametrize("name", ["f16", "bf16"])
+@pytest.mark.parametrize("case", NCHW, ids=lambda c: c.name)
+def test_nchw_tiled_half_activations(case, name):
+    dt, _ = DTYPES[name]
+    inp = inputs16(case, dt)
+    x = inp["x"].cuda()
+    Ho, Wo = gu.out_hw(case)
+    y = torch.empty(case.out_shape(Ho, Wo), device="cuda", dtype=dt)
+    desc = gu.desc_of(case)
+    desc.atype = {"f16": dw.DW_F16, "bf16": dw.DW_BF16}[name]
+    wp = inp["w"].cuda().data_ptr()
+    assert dw.dwconv2d_query_algo(desc, 0, x.data_ptr(), wp, y.data_ptr()) == dw.DW_ALGO_TILED
+    if Wo % 8 == 0:  # the input gradient reads dy rows of Wo elements
+        assert dw.dwconv2d_query_algo(desc, 1, y.data_ptr(), wp, x.data_ptr()) == dw.DW_ALGO_TILED
+    run_case(case, name, "auto")
+
+
 DIRECT = [
     Case("h_nchw_3x3", 2, 13, 16, 6, 3, 3, layout="nchw", seed=411),
+    Case("h_nchw_s2", 2, 13, 16, 6, 3, 3, stride=2, layout="nchw", seed=415),
     Case("h_c36", 2, 12, 14, 36, 3, 3, seed=412),   # C % 8 != 0: 16-bit rows not 16-byte
     Case("h_odd", 1, 9, 11, 7, 5, 5, stride=2, dilation=2, seed=413),
     Case("h_nchw_1x31", 2, 1, 70, 8, 1, 31, act="normal", layout="nchw", seed=414),
@@ -162,11 +204,12 @@ def test_fused_epilogue_half(name):
                 (case.name, act)
 
 
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
 @pytest.mark.parametrize("name", ["f16", "bf16"])
-def test_full_size_sampled(name):
+def test_full_size_sampled(name, layout):
     dt, u = DTYPES[name]
     rng = np.random.default_rng(31)
-    case = [c for c in wl.large() if c.H == 512 and c.layout == "nhwc"][0]
+    case = [c for c in wl.large() if c.H == 512 and c.layout == layout][0]
     inp = inputs16(case, dt)
     w32 = widened(inp)
     y = gu.gpu_fwd(case, inp)
