@@ -216,10 +216,15 @@ struct TArgs {
 };
 
 template <int KH_, int KW_, int S_, int D_, int THT_, int TWT_, int WX_, int WY_, int NS_,
-          class TA_ = float>
+          class TA_ = float, int MULT_ = 1>
 struct WCfg {
     using TA = TA_;  // activation element type of x and dy
     static constexpr int ESZ = sizeof(TA);
+    // channel multiplier: lane = output channel o of a 32-channel block, which
+    // reads input channel o / MULT; the x box holds the XC = 32 / MULT input
+    // channels of the block
+    static constexpr int MULT = MULT_;
+    static constexpr int XC = kLanes / MULT;
     static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
     static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
     static constexpr int T = KH * KW + 1;
@@ -231,7 +236,7 @@ struct WCfg {
     static constexpr int IW = (TW - 1) * S + (KW - 1) * D + 1;
     static constexpr int RH = (THT - 1) * S + (KH - 1) * D + 1;
     static constexpr int RW = (TWT - 1) * S + (KW - 1) * D + 1;
-    static constexpr int XBYTES = IH * IW * kLanes * ESZ;
+    static constexpr int XBYTES = IH * IW * XC * ESZ;
     static constexpr int GBYTES = TH * TW * kLanes * ESZ;
     static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;  // dy box on a 128-byte boundary
     static constexpr int STAGE_TX = XBYTES + GBYTES;           // bytes the two loads bring
@@ -239,7 +244,7 @@ struct WCfg {
     static constexpr int RED_BYTES = NCW * T * kLanes * 8;
     static constexpr int AREA = NS * STAGE_BYTES > RED_BYTES ? NS * STAGE_BYTES : RED_BYTES;
     static constexpr size_t SMEM = size_t(AREA) + size_t(2 * NS) * 8 + 16;
-    static_assert(ESZ == 4 || (XBYTES % 128 == 0 || XPITCH > XBYTES), "stage layout");
+    static_assert((XC * ESZ) % 16 == 0 && kLanes % MULT == 0, "16-byte rows in the x box");
     static_assert(IH <= 256 && IW <= 256 && TW <= 256 && TH <= 256, "TMA box limit");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                 const WTile T = decode<K>(t, a);
                 unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
                 mbar_arrive_expect_tx(&full[s], K::STAGE_TX);
-                tma_load_4d(st, &xmap, &full[s], T.cb * kLanes, T.ix0, T.iy0, T.n);
+                tma_load_4d(st, &xmap, &full[s], T.cb * K::XC, T.ix0, T.iy0, T.n);
                 tma_load_4d(st + K::XPITCH, &gmap, &full[s], T.cb * kLanes, T.ox0, T.oy0, T.n);
             }
             if (!ok) {
@@ -354,12 +359,12 @@ __global__ void __launch_bounds__(K::NT, 1)
         for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
             for (int kw = 0; kw < K::KW; ++kw) acc[kh][kw] = 0.f;
-        const TA* win = xb + ((j0 * K::S) * K::IW + i0 * K::S) * kLanes + lane;
+        const TA* win = xb + ((j0 * K::S) * K::IW + i0 * K::S) * K::XC + lane / K::MULT;
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             static_for<0, K::RW>([&](auto q_) {
                 constexpr int q = decltype(q_)::value;
-                const float v = ActIO<TA>::load1(win + (r * K::IW + q) * kLanes);
+                const float v = ActIO<TA>::load1(win + (r * K::IW + q) * K::XC);
                 static_for<0, K::THT>([&](auto j_) {
                     constexpr int j = decltype(j_)::value;
                     constexpr int kh = tap_of<K>(r, j);
@@ -443,8 +448,7 @@ size_t direct_workspace(const Problem& p) {
 }
 
 size_t tiled_workspace(const Problem& p) {
-    if (p.M != 1) return 0;
-    const int64_t tc = (p.C + kLanes - 1) / kLanes;
+    const int64_t tc = (p.Co + kLanes - 1) / kLanes;
     const int64_t g = tc >= kMaxTiledCtas ? tc : (kMaxTiledCtas / tc) * tc;
     return size_t(g) * size_t(p.kH * p.kW + 1) * kLanes * sizeof(double);
 }
@@ -496,12 +500,13 @@ dw_status_t launch_tiled(const Problem& p, const void* x, const void* dy, float*
     TArgs a;
     a.part = static_cast<double*>(ws);
     a.err = err;
-    a.C = static_cast<int>(p.C);
+    if (p.M != K::MULT) return DW_ERR_UNSUPPORTED;
+    a.C = static_cast<int>(p.Co);  // output channels: the lanes
     a.pt = p.pt;
     a.pl = p.pl;
     const int64_t ty = (p.Ho + K::TH - 1) / K::TH;
     const int64_t tx = (p.Wo + K::TW - 1) / K::TW;
-    const int64_t tc = (p.C + kLanes - 1) / kLanes;
+    const int64_t tc = (p.Co + kLanes - 1) / kLanes;
     const int64_t spatial = ty * tx * p.N;
     const int64_t nt = spatial * tc;
     if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
@@ -531,10 +536,10 @@ dw_status_t launch_tiled(const Problem& p, const void* x, const void* dy, float*
     const cuuint64_t xd[4] = {cuuint64_t(p.C), cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.N)};
     const cuuint64_t xs[3] = {cuuint64_t(p.C) * E, cuuint64_t(p.C * p.W) * E,
                               cuuint64_t(p.C * p.W * p.H) * E};
-    const cuuint32_t xbox[4] = {kLanes, K::IW, K::IH, 1};
-    const cuuint64_t gd[4] = {cuuint64_t(p.C), cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.N)};
-    const cuuint64_t gs[3] = {cuuint64_t(p.C) * E, cuuint64_t(p.C * p.Wo) * E,
-                              cuuint64_t(p.C * p.Wo * p.Ho) * E};
+    const cuuint32_t xbox[4] = {K::XC, K::IW, K::IH, 1};
+    const cuuint64_t gd[4] = {cuuint64_t(p.Co), cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.N)};
+    const cuuint64_t gs[3] = {cuuint64_t(p.Co) * E, cuuint64_t(p.Co * p.Wo) * E,
+                              cuuint64_t(p.Co * p.Wo * p.Ho) * E};
     const cuuint32_t gbox[4] = {kLanes, K::TW, K::TH, 1};
     constexpr CUtensorMapDataType dt = ActIO<typename K::TA>::kTma;
     if (encode_tensor_map(&xmap, dt, 4, const_cast<void*>(x), xd, xs, xbox, estr) != CUDA_SUCCESS ||
@@ -543,9 +548,9 @@ dw_status_t launch_tiled(const Problem& p, const void* x, const void* dy, float*
     if (launch_pdl(partial_tiled<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap, gmap,
                    a) != cudaSuccess)
         return DW_ERR_CUDA;
-    const int64_t fb = finalize_blocks(p.C * K::T, sm_count(dev));
+    const int64_t fb = finalize_blocks(p.Co * K::T, sm_count(dev));
     if (launch_pdl(finalize_tiled, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
-                   static_cast<const double*>(a.part), dw, db, int(p.C), K::T, int(tc),
+                   static_cast<const double*>(a.part), dw, db, int(p.Co), K::T, int(tc),
                    int(G)) != cudaSuccess)
         return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
@@ -1119,6 +1124,9 @@ dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, f
 
 //                         KH KW  S  D THT TWT WX WY NS
 template <class TA> using W33s1 = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4, TA>;
+template <int M> using W33s1m = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4, float, M>;
+template <int M> using W33s2m = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4, float, M>;
+template <int M> using W55s1m = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3, float, M>;
 template <class TA> using W33s2 = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4, TA>;
 template <class TA> using W55s1 = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3, TA>;
 template <class TA> using W77s1 = WCfg<7, 7, 1, 1, 1, 4, 4, 2, 3, TA>;
@@ -1142,9 +1150,32 @@ dw_status_t tiled_pick_nhwc(const Problem& p, const void* x, const void* dy, flo
     return DW_ERR_UNSUPPORTED;
 }
 
+// Channel multiplier (float32 NHWC, M = 2 or 4): 3x3, 3x3 stride 2, 5x5.
+template <int M>
+dw_status_t tiled_pick_mult(const Problem& p, const void* x, const void* dy, float* dw,
+                            float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    const int S = p.sh;
+#define DW_W(CFG) return launch_tiled<CFG<M>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 3 && p.kW == 3 && S == 1) DW_W(W33s1m)
+    if (p.kH == 3 && p.kW == 3 && S == 2) DW_W(W33s2m)
+    if (p.kH == 5 && p.kW == 5 && S == 1) DW_W(W55s1m)
+#undef DW_W
+    return DW_ERR_UNSUPPORTED;
+}
+
 dw_status_t tiled_pick(const Problem& p, const void* x, const void* dy, float* dw, float* db,
                        void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
-    if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
+    if (p.M != 1) {
+        // channel multiplier: float32 NHWC tiles for M = 2, 4; else the direct kernels
+        if (p.layout != DW_NHWC || p.atype != DW_F32 || (p.M != 2 && p.M != 4)) return DW_ERR_UNSUPPORTED;
+        if (p.C % 4 != 0 || ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15))
+            return DW_ERR_UNSUPPORTED;
+        if (p.sh != p.sw || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
+        if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.Co >= INT_MAX)
+            return DW_ERR_UNSUPPORTED;
+        return p.M == 2 ? tiled_pick_mult<2>(p, x, dy, dw, db, ws, stream, err, dry_run)
+                        : tiled_pick_mult<4>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    }
     if (p.layout == DW_NCHW) {
         if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;  // 16-bit NCHW: direct kernels
         return tiled_pick_nchw(p, static_cast<const float*>(x), static_cast<const float*>(dy), dw,

@@ -247,7 +247,9 @@ def test_channel_multiplier_host_checks(lib):
     need = dw.dwconv2d_bwd_weight_workspace_size(d)
     x, dy, dwp, db, ws = base, base + (1 << 24), base + (2 << 24), base + (3 << 24), base + (4 << 24)
     assert dw.bwd_weight_raw(d, x, dy, dwp, dwp + 8 * 9 * 4 - 4, ws, need, 0) == dw.DW_ERR_ALIAS
-    assert dw.dwconv2d_query_algo(d, 2, x, dy, dwp) == dw.DW_ALGO_DIRECT
+    assert dw.dwconv2d_query_algo(d, 2, x, dy, dwp) == dw.DW_ALGO_TILED
+    d3 = dw.make_desc(1, 8, 8, 4, 3, 3, multiplier=3)
+    assert dw.dwconv2d_query_algo(d3, 2, x, dy, dwp) == dw.DW_ALGO_DIRECT
 
 
 def test_half_activation_host_checks(lib):

@@ -72,7 +72,19 @@ def test_tiled_multiplier_forward(case):
     inp = gu.inputs(case)
     y = torch.empty(case.out_shape(*gu.out_hw(case)), device="cuda")
     assert gu.chosen_algo(case, 0, inp["x"].cuda(), inp["w"].cuda(), y) == dw.DW_ALGO_TILED
+    assert gu.chosen_algo(case, 2, inp["x"].cuda(), y, inp["w"].cuda()) == dw.DW_ALGO_TILED
     check_all(case, fwd_algos=("tiled", "direct"))
+    # the direct weight gradient agrees too
+    p = gu.problem(case)
+    x, dy = gu.f64(inp["x"]), gu.f64(inp["dy"])
+    dwr, dbr = oracle.bwd_weight(p, x, dy)
+    dws, dbs = oracle.bwd_weight(p, np.abs(x), np.abs(dy))
+    g_w, g_b = dw.dwconv2d_bwd_weight(inp["x"].cuda(), inp["dy"].cuda(), (case.kH, case.kW),
+                                      stride=case.stride, dilation=case.dilation,
+                                      padding=case.padding, layout=case.layout, algo="direct")
+    torch.cuda.synchronize()
+    gu.assert_close(g_w.cpu().numpy(), dwr, dws, f"{case.name} dW direct")
+    gu.assert_close(g_b.cpu().numpy(), dbr, dbs, f"{case.name} db direct")
 
 
 DIRECT = [
