@@ -136,11 +136,15 @@ template <int KH_, int KW_, int S_, int D_, bool TR_, int THT_, int TWT_, int WX
 struct Cfg {
     using TA = TA_;  // activation element type (float, __half, __nv_bfloat16)
     static constexpr int ESZ = sizeof(TA);
-    static constexpr int CB = CB_;  // (output) channels per tile
-    // channel multiplier: a tile's CB output channels read CBI = CB / MULT
-    // input channels (output channel o reads input channel o / MULT)
+    static constexpr int CB = CB_;  // channels per tile of the tensor written
+    // channel multiplier (output channel o reads input channel o / MULT).
+    // Forward: a tile's CB output channels read CB / MULT staged input
+    // channels.  Transposed mode: a tile's CB dx channels gather from
+    // CB * MULT staged dy channels, MT = MULT float4s per lane and cell.
     static constexpr int MULT = MULT_;
-    static constexpr int CBI = CB / MULT;
+    static constexpr bool TR0 = TR_;
+    static constexpr int SC = TR0 ? CB * MULT : CB / MULT;  // staged channels per pixel
+    static constexpr int MT = TR0 ? MULT : 1;
     static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
     static constexpr bool TR = TR_;
     static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
@@ -161,7 +165,7 @@ struct Cfg {
     // rows / columns of the input window one thread reads
     static constexpr int RH = TR ? AH + (THT - 1) / S + 1 : (THT - 1) * S + (KH - 1) * D + 1;
     static constexpr int RW = TR ? AW + (TWT - 1) / S + 1 : (TWT - 1) * S + (KW - 1) * D + 1;
-    static constexpr int STAGE_BYTES = IH * IW * CBI * ESZ;  // one TMA load
+    static constexpr int STAGE_BYTES = IH * IW * SC * ESZ;  // one TMA load
     static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
     static constexpr int OUT_ELEMS = TH * TW * CB;  // output staging buffer
     static constexpr int OUT_BYTES = OUT_ELEMS * ESZ;
@@ -172,9 +176,9 @@ struct Cfg {
     // every stage starts on a 128-byte boundary (tensor-copy destination rule)
     static_assert(MULT > 1 || ESZ < 4 || STAGE_BYTES % 128 == 0, "TMA shared-memory alignment");
     static_assert(NO == 0 || OUT_BYTES % 128 == 0, "staging buffers on 128-byte boundaries");
-    static_assert((CBI * ESZ) % 16 == 0, "16-byte rows in the input box");
-    static_assert(MULT == 1 || (!TR && VEC == 4 && CB % MULT == 0),
-                  "multiplier tiles: forward, 4-channel lanes");
+    static_assert((SC * ESZ) % 16 == 0 && SC <= 256, "16-byte rows in the input box");
+    static_assert(MULT == 1 || (VEC == 4 && (TR || CB % MULT == 0)),
+                  "multiplier tiles: 4-channel lanes");
     static_assert(!TR || (THT % S == 0 && TWT % S == 0), "transposed blocks are phase aligned");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 }
                 const Tile T = decode_tile<K>(t, a);
                 mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
-                tma_load_4d(smem + size_t(s) * K::STAGE_PITCH, &tmap, &full[s], T.cb * K::CBI, T.ix0,
+                tma_load_4d(smem + size_t(s) * K::STAGE_PITCH, &tmap, &full[s], T.cb * K::SC, T.ix0,
                             T.iy0, T.n);
             }
             if (!ok) {
@@ -318,19 +322,30 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     const int j0 = yi * K::THT, i0 = xi * K::TWT;
     const int64_t row_pitch = int64_t(a.Wout) * a.C;
 
-    V wr[K::KH][K::KW];
+    V wr[K::KH][K::KW][K::MT];
     V bias = VO::zero();
     int cur_cb = -1;
-    // the value stored for one output: acc (+ bias) (-> activation)
-    auto finish = [&](const V& acc) -> V {
-        if constexpr (K::TR) {
-            return acc;
+    // the value stored for one output: acc (+ bias) (-> activation); with a
+    // multiplier in transposed mode, dx channel c + e sums the MULT
+    // consecutive products of output channels (c + e) * MULT ..
+    auto finish = [&](const V (&acc)[K::MT]) -> V {
+        if constexpr (K::TR && K::MT == 2) {
+            return make_float4(acc[0].x + acc[0].y, acc[0].z + acc[0].w, acc[1].x + acc[1].y,
+                               acc[1].z + acc[1].w);
+        } else if constexpr (K::TR && K::MT == 4) {
+            return make_float4((acc[0].x + acc[0].y) + (acc[0].z + acc[0].w),
+                               (acc[1].x + acc[1].y) + (acc[1].z + acc[1].w),
+                               (acc[2].x + acc[2].y) + (acc[2].z + acc[2].w),
+                               (acc[3].x + acc[3].y) + (acc[3].z + acc[3].w));
+        } else if constexpr (K::TR) {
+            return acc[0];
         } else if constexpr (EPI != kNoEpilogue) {
-            return VO::template act<EPI>(VO::add(acc, bias));
+            return VO::template act<EPI>(VO::add(acc[0], bias));
         } else {
-            return VO::add(acc, bias);
+            return VO::add(acc[0], bias);
         }
     };
+    static_assert(K::MT == 1 || K::MT == 2 || K::MT == 4, "transposed multiplier 2 or 4");
 
     int k = 0;
     for (int t = blockIdx.x; t < a.ntiles; t += G, ++k) {
@@ -341,28 +356,36 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
             cur_cb = T.cb;
             const bool live = c < a.C;
             constexpr int step = K::KH * K::KW;
-            const int64_t o = int64_t(live ? c : 0) * step;
+            // filter rows: channel c (forward: the output channel), or in
+            // transposed mode with a multiplier output channels c*MULT + 4m..
+            const int64_t o = int64_t(live ? c : 0) * (K::TR ? K::MULT : 1) * step;
             // one branch on the weight type, then straight loads
             if (a.wtype == DW_F16) {
                 const __half* wp = static_cast<const __half*>(a.w);
 #pragma unroll
-                for (int kh = 0; kh < K::KH; ++kh)
+                for (int m = 0; m < K::MT; ++m)
 #pragma unroll
-                    for (int kw = 0; kw < K::KW; ++kw)
-                        wr[kh][kw] = VO::load_w(wp, o + kh * K::KW + kw, step);
+                    for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                        for (int kw = 0; kw < K::KW; ++kw)
+                            wr[kh][kw][m] = VO::load_w(wp, o + 4 * m * step + kh * K::KW + kw, step);
             } else {
                 const float* wp = static_cast<const float*>(a.w);
 #pragma unroll
-                for (int kh = 0; kh < K::KH; ++kh)
+                for (int m = 0; m < K::MT; ++m)
 #pragma unroll
-                    for (int kw = 0; kw < K::KW; ++kw)
-                        wr[kh][kw] = VO::load_w(wp, o + kh * K::KW + kw, step);
+                    for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                        for (int kw = 0; kw < K::KW; ++kw)
+                            wr[kh][kw][m] = VO::load_w(wp, o + 4 * m * step + kh * K::KW + kw, step);
             }
             if (!live) {
 #pragma unroll
-                for (int kh = 0; kh < K::KH; ++kh)
+                for (int m = 0; m < K::MT; ++m)
 #pragma unroll
-                    for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] = VO::zero();
+                    for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw][m] = VO::zero();
             }
             if (!K::TR && a.b != nullptr && live) bias = VO::load_b(a.b, c);
             if constexpr (EPI != kNoEpilogue) {
@@ -373,7 +396,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 #pragma unroll
                     for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] = VO::mul(wr[kh][kw], sc);
+                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw][0] = VO::mul(wr[kh][kw][0], sc);
                     bias = VO::fma(bias, sc, sh, 0);
                 }
             }
@@ -393,16 +416,20 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
         // consumer barrier below, so every consumer leaves together; the
         // shared-memory reads in between stay inside the stage)
 
-        V acc[K::THT][K::TWT];
+        V acc[K::THT][K::TWT][K::MT];
 #pragma unroll
         for (int j = 0; j < K::THT; ++j)
 #pragma unroll
-            for (int i = 0; i < K::TWT; ++i) acc[j][i] = VO::zero();
+            for (int i = 0; i < K::TWT; ++i)
+#pragma unroll
+                for (int m = 0; m < K::MT; ++m) acc[j][i][m] = VO::zero();
 
-        // this thread's window: cell (r, q) holds CBI input channels; the
-        // lane's 4 output channels cv*4.. read input channels (cv*4)/MULT..
+        // this thread's window: cell (r, q) holds SC staged channels.  The
+        // lane's 4 channels cv*4.. read, in the forward, input channels
+        // (cv*4)/MULT..; in transposed mode dy channels cv*4*MULT ..
         const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
-                        (r0 * K::IW + q0) * K::CBI + (cv * K::VEC) / K::MULT;
+                        (r0 * K::IW + q0) * K::SC +
+                        (K::TR ? cv * K::VEC * K::MULT : (cv * K::VEC) / K::MULT);
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             static_for<0, K::RW>([&](auto q_) {
@@ -416,7 +443,14 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     return false;
                 }();
                 if constexpr (used) {
-                    const V v = load_cell<K>(win + (r * K::IW + q) * K::CBI);
+                    V v[K::MT];
+                    if constexpr (K::MT == 1) {
+                        v[0] = load_cell<K>(win + (r * K::IW + q) * K::SC);
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < K::MT; ++m)
+                            v[m] = ActIO<TA>::load4(win + (r * K::IW + q) * K::SC + 4 * m);
+                    }
                     static_for<0, K::THT>([&](auto j_) {
                         constexpr int j = decltype(j_)::value;
                         constexpr int kh = tap_for<K, true>(r, j);
@@ -424,7 +458,11 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                             static_for<0, K::TWT>([&](auto i_) {
                                 constexpr int i = decltype(i_)::value;
                                 constexpr int kw = tap_for<K, false>(q, i);
-                                if constexpr (kw >= 0) VO::fma(acc[j][i], v, wr[kh][kw]);
+                                if constexpr (kw >= 0) {
+#pragma unroll
+                                    for (int m = 0; m < K::MT; ++m)
+                                        VO::fma(acc[j][i][m], v[m], wr[kh][kw][m]);
+                                }
                             });
                         }
                     });
@@ -537,10 +575,11 @@ dw_status_t launch(const Problem& p, Op op, const void* in, const void* w, const
     CUtensorMap map;
     constexpr cuuint64_t E = K::ESZ;
     constexpr CUtensorMapDataType dt = ActIO<typename K::TA>::kTma;
-    const cuuint64_t dims[4] = {cuuint64_t(p.C), cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.N)};
-    const cuuint64_t strides[3] = {cuuint64_t(p.C) * E, cuuint64_t(p.C * Win) * E,
-                                   cuuint64_t(p.C * Win * Hin) * E};
-    const cuuint32_t box[4] = {K::CBI, K::IW, K::IH, 1};
+    const int64_t Cin = tr ? p.Co : p.C;  // channels of the tensor read (dy or x)
+    const cuuint64_t dims[4] = {cuuint64_t(Cin), cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.N)};
+    const cuuint64_t strides[3] = {cuuint64_t(Cin) * E, cuuint64_t(Cin * Win) * E,
+                                   cuuint64_t(Cin * Win * Hin) * E};
+    const cuuint32_t box[4] = {K::SC, K::IW, K::IH, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     if (encode_tensor_map(&map, dt, 4, const_cast<void*>(in), dims, strides, box, estr) !=
         CUDA_SUCCESS)
@@ -692,6 +731,8 @@ dw_status_t bwd_launch_bf16(const Problem& p, const void* in, const void* w, voi
                             cudaStream_t stream, int32_t* err, bool dry_run);
 dw_status_t mult_launch(const Problem& p, const void* in, const void* w, const float* b,
                         void* out, cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t mult_bwd_launch(const Problem& p, const void* in, const void* w, void* out,
+                            cudaStream_t stream, int32_t* err, bool dry_run);
 
 }  // namespace nhwc
 }  // namespace dw

@@ -144,3 +144,17 @@ def test_full_size_sampled(case):
     ref, scale = gu.reference_bwd_at(case, inp, idx)
     gu.assert_close(dx.reshape(-1)[torch.from_numpy(idx).cuda()].cpu().numpy(), ref, scale,
                     f"{case.name} bwd sampled")
+
+
+@pytest.mark.parametrize("case", [c for c in TILED if c.kH == 3 and (c.multiplier == 2 or c.stride == 1)],
+                         ids=lambda c: c.name)
+def test_tiled_multiplier_input_gradient(case):
+    inp = gu.inputs(case)
+    dy, w = inp["dy"].cuda(), inp["w"].cuda()
+    dx = torch.empty(case.in_shape(), device="cuda")
+    assert gu.chosen_algo(case, 1, dy, w, dx) == dw.DW_ALGO_TILED
+    ref, scale = gu.reference_bwd(case, inp)
+    for algo in ("tiled", "direct"):
+        got = gu.gpu_bwd(case, inp, algo)
+        torch.cuda.synchronize()
+        gu.assert_close(got.cpu().numpy(), ref, scale, f"{case.name} bwd_input [{algo}]")
