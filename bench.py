@@ -490,19 +490,24 @@ def run_profile(args, local_rank):
     dwbuild.build()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    # SHAPE:OP with OP fwd, bwd, fused or wgrad, optionally suffixed _f16 / _bf16
     name, op = args.profile.split(":")
+    op, _, atype = op.partition("_")
     cases, _ = workload_cases(args.workload)
     match = [c for c in cases if c.name == name]
-    if not match or op not in ("fwd", "bwd"):
+    if not match or op not in ("fwd", "bwd", "fused", "wgrad") or atype not in ("", "f16", "bf16"):
         raise SystemExit(f"unknown kernel {args.profile!r}; shapes: {[c.name for c in cases]}")
-    sh = Shape(match[0], dw, torch, device, 1)
+    sh = Shape(match[0], dw, torch, device, 1, atype=atype or "f32")
+    if op in ("fused", "wgrad"):
+        sh.prepare_next_rows(dw, torch, device, "silu" if args.workload == "conformer" else "relu6")
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         for _ in range(args.steps):
             sh.call(dw, op, 0, stream.cuda_stream)
     torch.cuda.synchronize()
     print(json.dumps({"profile": args.profile, "launches": args.steps,
-                      "algo": dw.dwconv2d_query_algo(sh.desc, 0 if op == "fwd" else 1,
+                      "algo": dw.dwconv2d_query_algo(sh.desc, {"fwd": 0, "fused": 0, "bwd": 1,
+                                                              "wgrad": 2}[op],
                                                      sh.sets[0]["x"].data_ptr(), sh.w.data_ptr(),
                                                      sh.sets[0]["y"].data_ptr())}), flush=True)
     return 0
@@ -517,7 +522,9 @@ def oracle_step(cases, fraction, oracle, np, torch):
     jobs = []
     total_bytes = 0
     for c in cases:
-        p = oracle.problem(c.in_shape(), c.kH, c.kW, c.stride, c.dilation, c.padding, c.layout)
+        M = c.multiplier
+        p = oracle.problem(c.in_shape(), c.kH, c.kW, c.stride, c.dilation, c.padding, c.layout,
+                           multiplier=M)
         o = oracle.out_shape(p)
         Ho, Wo = (o[1], o[2]) if c.layout == "nhwc" else (o[2], o[3])
         inp = make_inputs(c, (Ho, Wo))
@@ -526,12 +533,15 @@ def oracle_step(cases, fraction, oracle, np, torch):
         sl = [slice(None)] * 4
         sl[cax] = slice(0, keep)
         x = np.ascontiguousarray(inp["x"].numpy()[tuple(sl)], dtype=np.float64)
+        sl[cax] = slice(0, keep * M)  # the kept input channels' output channels
         dy = np.ascontiguousarray(inp["dy"].numpy()[tuple(sl)], dtype=np.float64)
-        w = np.ascontiguousarray(inp["w32"].numpy()[:keep], dtype=np.float64)
-        b = None if inp["b"] is None else np.ascontiguousarray(inp["b"].numpy()[:keep], dtype=np.float64)
+        w = np.ascontiguousarray(inp["w32"].numpy()[:keep * M], dtype=np.float64)
+        b = None if inp["b"] is None else np.ascontiguousarray(inp["b"].numpy()[:keep * M],
+                                                               dtype=np.float64)
         shape = list(c.in_shape())
         shape[cax] = keep
-        ps = oracle.problem(tuple(shape), c.kH, c.kW, c.stride, c.dilation, c.padding, c.layout)
+        ps = oracle.problem(tuple(shape), c.kH, c.kW, c.stride, c.dilation, c.padding, c.layout,
+                            multiplier=M)
         sub = c.with_(C=keep)
         total_bytes += algorithmic_bytes(sub, Ho, Wo, "fwd") + algorithmic_bytes(sub, Ho, Wo, "bwd")
         jobs.append((ps, x, w, b, dy))
