@@ -24,21 +24,28 @@
  * dy onto the forward's sampled positions followed by that correlation
  * (sections "Stride-2 SAME depthwise input-VJP" and "Stride-2 XLA-SAME
  * depthwise input-VJP"); both are computed without materialising anything.
+ * The weight and bias gradients are the sums of the sections "Depthwise
+ * weight-VJP" and "Depthwise bias gradient - closed-form formula".  With a
+ * channel multiplier M (desc->multiplier) output channel o = c*M + j reads
+ * input channel c through filter o; M = 1 is the formula above.
  *
  * Conventions for every entry point:
- *   - Activations (x, y, dy, dx) are float32, dense, in the layout of
+ *   - Activations (x, y, dy, dx) are dense, of the element type desc->atype
+ *     (float32 by default, or float16 / bfloat16), in the layout of
  *     desc->layout: DW_NHWC = [N][H][W][C] (C innermost), DW_NCHW =
- *     [N][C][H][W] (W innermost).
- *   - Weights are [C][kH][kW] row-major (the PyTorch [C,1,kH,kW] depthwise
+ *     [N][C][H][W] (W innermost).  y and dy have C*M channels.
+ *   - Weights are [C*M][kH][kW] row-major (the PyTorch [C*M,1,kH,kW] grouped
  *     weight, contiguous), float32 or float16 per desc->wtype.  float16 weights
  *     are widened exactly to float32; accumulation is always float32, taps in
  *     kh-major / kw-minor order, then the bias is added.  With weights that are
  *     exactly representable in float16, the float16 and float32 weight paths
  *     return bit-identical results.
- *   - Bias is float32 [C] or NULL (NULL means zero).
+ *   - Bias is float32 [C*M] or NULL (NULL means zero).
  *   - All data pointers are DEVICE pointers owned by the caller.  The library
- *     never allocates, frees or retains them.  Unaligned pointers are accepted
- *     (a slower kernel is chosen).
+ *     never allocates, frees or retains them (the weight gradient takes a
+ *     caller workspace; its no-allocation variant uses a fixed array inside
+ *     the library).  Unaligned pointers are accepted (a slower kernel is
+ *     chosen).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous: they enqueue kernels and return without synchronising.
  *     They make no device allocation and may be captured in a CUDA graph once
