@@ -11,5 +11,5 @@ from .dwconv2d import (  # noqa: F401
     bwd_weight_noalloc_raw, bwd_weight_raw, dwconv2d_bwd_input, dwconv2d_bwd_weight, dwconv2d_bwd_weight_workspace_size,
     dwconv2d_fwd, dwconv2d_fwd_bn_act, dwconv2d_out_shape, fwd_bn_act_raw, dwconv2d_query_algo,
     dwconv2d_resolved_pads, dwconv2d_take_device_error, dwconv2d_version, fwd_raw, lib,
-    library_path, make_desc, status_string,
+    library_path, make_desc, selftest_wait_timeout_raw, status_string,
 )

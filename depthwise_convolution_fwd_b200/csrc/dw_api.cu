@@ -244,6 +244,33 @@ static dw_status_t run(const dw_desc_t* desc, Op op, const Buffers& bf, cudaStre
     return direct_launch(p, op, bf.in, bf.w, bf.b, bf.out, stream);
 }
 
+// One CTA of two warps and a barrier that nothing completes (see
+// dwconv2d_selftest_wait_timeout).  Every wait is bounded, so the kernel
+// always ends: mode 0 by its own limit, mode 1 by the abort flag (and, were
+// the flag not seen, by the 2 s limit).
+__global__ void __launch_bounds__(64) selftest_wait_kernel(int32_t* err, int mode,
+                                                          uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ volatile int abort_flag;
+    grid_dependency_wait();
+    allow_dependents();
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane != 0) return;
+    if (mode == 0) {
+        if (warp == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicExch(err, DW_ERR_DEVICE_TIMEOUT);
+    } else if (warp == 1) {
+        abort_flag = 1;  // a failing warp raises the CTA's abort flag
+    } else if (!mbar_wait_or_abort(&bar, 0, &abort_flag)) {
+        atomicExch(err, DW_ERR_DEVICE_TIMEOUT);
+    }
+}
+
 }  // namespace dw
 
 using namespace dw;
@@ -393,6 +420,16 @@ dw_status_t dwconv2d_take_device_error(int32_t* code) {
         return DW_ERR_CUDA;
     *code = v;
     return DW_OK;
+}
+
+dw_status_t dwconv2d_selftest_wait_timeout(int32_t mode, uint32_t limit_us, void* stream) {
+    if ((mode != 0 && mode != 1) || limit_us < 1 || limit_us > 1000000u) return DW_ERR_INVALID_ARG;
+    int32_t* err = device_error_ptr(current_device());
+    if (!err) return DW_ERR_CUDA;
+    if (launch_pdl(selftest_wait_kernel, dim3(1), dim3(64), 0, static_cast<cudaStream_t>(stream),
+                   err, mode, uint64_t(limit_us) * 1000u) != cudaSuccess)
+        return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
 const char* dwconv2d_status_string(dw_status_t status) {

@@ -19,7 +19,6 @@ dw_status_t tiled_nchw_launch(const Problem& p, Op op, const void* in, const voi
     using namespace nchw;
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
     if (p.M != 1) return DW_ERR_UNSUPPORTED;  // channel multiplier: direct kernels
-    if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
     const int64_t Win = op == OP_FWD ? p.W : p.Wo;
     // TMA row stride: a multiple of 16 bytes
     if ((Win * act_bytes(p.atype)) % 16 != 0) return DW_ERR_UNSUPPORTED;

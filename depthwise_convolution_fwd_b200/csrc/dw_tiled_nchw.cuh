@@ -48,9 +48,10 @@ struct Args {
 };
 
 template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
-          int MINB_ = 1, class TA_ = float>
+          int MINB_ = 1, class TA_ = float, int S_ = 1>
 struct Cfg {
     using TA = TA_;
+    static constexpr int S = S_;  // stride (forward only: output (ho, wo) reads row ho*S.., col wo*S..)
     static constexpr int ESZ = sizeof(TA);
     static constexpr int ALIGN = 16 / ESZ;  // elements per 16 bytes
     static constexpr int MINB = MINB_;  // CTAs per SM the register budget is sized for
@@ -62,21 +63,23 @@ struct Cfg {
     static constexpr int NT = WX * WY + 32;   // + one producer warp
     static constexpr int TW = 4 * WX;
     static constexpr int TH = ROWS ? 1 : THT * WY;
-    static constexpr int IH = ROWS ? 1 : TH + (KH - 1) * D;
-    static constexpr int IWB = (REM + (ALIGN - 4) + TW + (KW - 1) * D + ALIGN - 1) / ALIGN * ALIGN;
+    static constexpr int IH = ROWS ? 1 : (TH - 1) * S + (KH - 1) * D + 1;
+    static constexpr int IWB =
+        (REM + (ALIGN - 4) + (TW - 1) * S + (KW - 1) * D + 1 + ALIGN - 1) / ALIGN * ALIGN;
     static constexpr int BOXH = IH;
     static constexpr int BOXC = ROWS ? WY : 1;
     // bytes one TMA box delivers, and the stage pitch: every stage must start
     // on a 128-byte boundary (shared-memory destination rule of tensor copies)
     static constexpr int STAGE_BYTES = IWB * IH * BOXC * ESZ;
     static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
-    static constexpr int RH = THT + (KH - 1) * D;           // window rows
-    static constexpr int NV = (REM + 3 + (KW - 1) * D) / 4 + 1;  // float4 per window row
+    static constexpr int RH = (THT - 1) * S + (KH - 1) * D + 1;       // window rows
+    static constexpr int NV = (REM + 3 * S + (KW - 1) * D) / 4 + 1;  // 4-vectors per window row
     static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NS) * 8 + 16;
     static_assert((WX * WY) % 32 == 0, "whole consumer warps");
     static_assert(IWB <= 256 && IH <= 256 && BOXC <= 256, "TMA box dimension limit");
     static_assert(STAGE_PITCH % 128 == 0 && (IWB * ESZ) % 16 == 0, "TMA alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+    static_assert(S == 1 || (!REV && !ROWS), "strided tiles: 2-D forward only");
 };
 
 
@@ -139,13 +142,13 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 }
                 int tx, ty, c, n;
                 decode_tile<K>(t, a, tx, ty, c, n);
-                const int ix0 = tx * K::TW - a.pl - K::REM - a.sh4;
+                const int ix0 = tx * K::TW * K::S - a.pl - K::REM - a.sh4;
                 unsigned char* dst = smem + size_t(s) * K::STAGE_PITCH;
                 mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
                 if constexpr (K::ROWS)
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
                 else
-                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH - a.pt, c, n);
+                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt, c, n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -218,9 +221,9 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
 
-        const int row0 = K::ROWS ? yi : yi * K::THT;
+        const int row0 = K::ROWS ? yi : yi * K::THT;  // first output row of this thread
         const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
-                        size_t(row0) * K::IWB + 4 * xi + a.sh4;
+                        size_t(row0 * K::S) * K::IWB + 4 * xi * K::S + a.sh4;
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             float v[4 * K::NV];
@@ -234,14 +237,14 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
             }
             static_for<0, K::THT>([&](auto j_) {
                 constexpr int j = decltype(j_)::value;
-                constexpr int khn = r - j;
+                constexpr int khn = r - j * K::S;
                 if constexpr (khn >= 0 && khn % K::D == 0 && khn / K::D < K::KH) {
                     constexpr int kh = khn / K::D;
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
 #pragma unroll
                         for (int kw = 0; kw < K::KW; ++kw)
-                            acc[j][i] = fmaf(v[K::REM + i + kw * K::D], wr[kh][kw], acc[j][i]);
+                            acc[j][i] = fmaf(v[K::REM + i * K::S + kw * K::D], wr[kh][kw], acc[j][i]);
                 }
             });
         });
@@ -691,10 +694,37 @@ dw_status_t launch_op(const Problem& p, Op op, const void* in, const void* w, co
                                                                (KW - 1) - p.pl);
 }
 
+// Stride-2 forward (2-D kernel with S = 2): a tile is TH x 4*WX outputs, its
+// box the (TH-1)*2 + kH rows and (TW-1)*2 + kW columns they read.
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA>
+dw_status_t launch_s2_fwd(const Problem& p, const void* in, const void* w, const float* b,
+                          void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    int rem, sh4;
+    box_shift<TA>(p.pl, rem, sh4);
+#define DW_S2(R) \
+    return launch<Cfg<KH, KW, 1, false, R, THT, WX, WY, NS, 1, TA, 2>>(p, in, w, b, out, stream, \
+                                                                       err, dry_run, p.pt, p.pl, sh4);
+    switch (rem) {
+        case 0: DW_S2(0)
+        case 1: DW_S2(1)
+        case 2: DW_S2(2)
+        default: DW_S2(3)
+    }
+#undef DW_S2
+}
+
 // The configurations of one activation type.
 template <class TA>
 dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w, const float* b,
                           void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
+    if (p.sh == 2 && p.sw == 2) {
+        // strided: the forward of 3x3 filters (input gradients on the direct kernel)
+        if (op == OP_FWD && p.kH == 3 && p.kW == 3)
+            return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA>(p, in, w, b, out, stream, err, dry_run);
+        return DW_ERR_UNSUPPORTED;
+    }
+    if (p.sh != 1 || p.sw != 1) return DW_ERR_UNSUPPORTED;
     //                                                       KH  KW THT WX  WY NS
     if (p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 32, 8, 4, TA>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 32, 8, 4, TA>(p, op, in, w, b, out, stream, err, dry_run);

@@ -34,6 +34,7 @@ EXPORTS = ("dwconv2d_out_shape", "dwconv2d_resolved_pads", "dwconv2d_fwd", "dwco
            "dwconv2d_bwd_input", "dwconv2d_bwd_weight", "dwconv2d_bwd_weight_workspace_size",
            "dwconv2d_bwd_weight_noalloc",
            "dwconv2d_query_algo", "dwconv2d_take_device_error", "dwconv2d_status_string",
+           "dwconv2d_selftest_wait_timeout",
            "dwconv2d_version")
 
 
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
     L.dwconv2d_query_algo.argtypes = [P(DwDesc), i32, vp, vp, vp]
     L.dwconv2d_take_device_error.restype = i32
     L.dwconv2d_take_device_error.argtypes = [P(i32)]
+    L.dwconv2d_selftest_wait_timeout.restype = i32
+    L.dwconv2d_selftest_wait_timeout.argtypes = [i32, ctypes.c_uint32, vp]
     L.dwconv2d_status_string.restype = ctypes.c_char_p
     L.dwconv2d_status_string.argtypes = [i32]
     L.dwconv2d_version.restype = i32
@@ -171,6 +174,13 @@ def dwconv2d_take_device_error() -> int:
     if st != DW_OK:
         raise DwError(st, "dwconv2d_take_device_error")
     return int(code.value)
+
+
+def selftest_wait_timeout_raw(mode: int, limit_us: int, stream: int) -> int:
+    """dwconv2d_selftest_wait_timeout: a kernel whose bounded wait runs out
+    (mode 0) or is aborted by another warp (mode 1); returns the status.  The
+    device error word then holds DW_ERR_DEVICE_TIMEOUT."""
+    return int(lib().dwconv2d_selftest_wait_timeout(int(mode), int(limit_us), stream or None))
 
 
 def dwconv2d_version() -> int:

@@ -279,6 +279,23 @@ DW_API int32_t dwconv2d_query_algo(const dw_desc_t* desc, int32_t op, const void
  */
 DW_API dw_status_t dwconv2d_take_device_error(int32_t* code);
 
+/*
+ * Self-test of the failure path (the pages have no counterpart: it exists so
+ * that tests can check, on a GPU, what a kernel does when one of its waits
+ * on an asynchronous copy never completes).  Launches one small CTA that
+ * waits, with the same bounded wait every kernel uses, on a shared-memory
+ * barrier that nothing completes:
+ *   mode 0: one thread waits until `limit_us` microseconds have passed;
+ *   mode 1: one warp waits (limit 2 s) while another raises the CTA's abort
+ *           flag, as a failing warp does, and the waiting warp gives up.
+ * Either way the kernel records DW_ERR_DEVICE_TIMEOUT in the device error
+ * word (read it with dwconv2d_take_device_error) and returns; nothing faults,
+ * and the context stays usable.  limit_us: 1 .. 10^6; mode: 0 or 1, else
+ * DW_ERR_INVALID_ARG.  Asynchronous on `stream` like every call.
+ */
+DW_API dw_status_t dwconv2d_selftest_wait_timeout(int32_t mode, uint32_t limit_us,
+                                                  void* stream);
+
 /* Human-readable name of a status code (static string). */
 DW_API const char* dwconv2d_status_string(dw_status_t status);
 

@@ -144,7 +144,9 @@ def test_query_algo_selects_tiled_for_covered_shapes(lib):
     assert q(dw.make_desc(1, 30, 19, 128, 7, 7, layout="nchw")) == D     # W % 4 != 0
     assert q(dw.make_desc(1, 16, 16, 8, 3, 3), align=4) == D             # unaligned pointers
     assert q(dw.make_desc(1, 16, 16, 8, 2, 2)) == D                      # no 2x2 instance
-    assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2)) == D
+    assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2)) == T        # strided fwd
+    assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2), op=1) == D  # strided bwd
+    assert q(dw.make_desc(1, 16, 16, 8, 5, 5, layout="nchw", stride=2)) == D
     # forcing
     assert q(dw.make_desc(1, 13, 17, 7, 3, 3, algo="direct")) == D
     assert q(dw.make_desc(1, 512, 512, 256, 3, 3, algo="direct")) == D
@@ -273,3 +275,9 @@ def test_half_activation_host_checks(lib):
         dn4 = dw.make_desc(1, 8, 12, 8, 3, 3, layout="nchw")  # W = 12: 24-byte rows
         dn4.atype = at
         assert dw.dwconv2d_query_algo(dn4, 0, base, w, base + 4096) == dw.DW_ALGO_DIRECT
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    # validation only: nothing is launched for these
+    for mode, limit in ((2, 1000), (-1, 1000), (0, 0), (1, 2_000_000)):
+        assert dw.selftest_wait_timeout_raw(mode, limit, 0) == dw.DW_ERR_INVALID_ARG
