@@ -151,6 +151,73 @@ __global__ void __launch_bounds__(256) partial_direct_nchw(const TA* __restrict_
     }
 }
 
+// NCHW with the filter extent known at compile time: one warp per (chunk,
+// output channel) forms every tap's sum at once, so each dy value is read
+// once (not once per tap) and the x values a position's taps share come from
+// L1.  Partials in the layout of partial_direct_nchw, same finalize.
+template <class TA, int KH, int KW>
+__global__ void __launch_bounds__(256) partial_direct_nchw_taps(const TA* __restrict__ x,
+                                                                const TA* __restrict__ dy,
+                                                                double* __restrict__ part, DArgs a) {
+    grid_dependency_wait();
+    allow_dependents();
+    constexpr int T = KH * KW + 1;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    const int64_t n_items = a.chunks * a.Co;
+    for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < n_items;
+         i += warps) {
+        const int64_t o = i % a.Co;  // output channel; it reads input channel o / M
+        const int64_t c = o / a.M;
+        const int64_t j = i / a.Co;
+        const int64_t p0 = j * a.chunk;
+        const int64_t p1 = p0 + a.chunk < a.P ? p0 + a.chunk : a.P;
+        double acc64[T];
+        float acc[T];
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            acc64[t] = 0.0;
+            acc[t] = 0.f;
+        }
+        int cnt = 0;
+        const TA* xc = x + c * a.H * a.W;  // plane of (n = 0, c); n added below
+        for (int64_t pp = p0 + lane; pp < p1; pp += 32) {
+            const int64_t wo = pp % a.Wo, q = pp / a.Wo;
+            const int64_t ho = q % a.Ho, n = q / a.Ho;
+            const float g = ActIO<TA>::load1(dy + ((n * a.Co + o) * a.Ho + ho) * a.Wo + wo);
+            const TA* xp = xc + n * a.C * a.H * a.W;
+#pragma unroll
+            for (int kh = 0; kh < KH; ++kh) {
+                const int64_t hi = ho * a.sh + int64_t(kh) * a.dh - a.pt;
+                const bool hin = hi >= 0 && hi < a.H;
+#pragma unroll
+                for (int kw = 0; kw < KW; ++kw) {
+                    const int64_t wi = wo * a.sw + int64_t(kw) * a.dw - a.pl;
+                    if (hin && wi >= 0 && wi < a.W)
+                        acc[kh * KW + kw] = fmaf(g, ActIO<TA>::load1(xp + hi * a.W + wi),
+                                                 acc[kh * KW + kw]);
+                }
+            }
+            acc[T - 1] += g;
+            if (++cnt == kFold) {
+#pragma unroll
+                for (int t = 0; t < T; ++t) {
+                    acc64[t] += double(acc[t]);
+                    acc[t] = 0.f;
+                }
+                cnt = 0;
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            double v = acc64[t] + double(acc[t]);
+#pragma unroll
+            for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+            if (lane == 0) part[(j * T + t) * a.Co + o] = v;
+        }
+    }
+}
+
 // Fixed-order sum of `count` float64 terms by one warp: lane l adds terms
 // l, l+32, ... in order, then a fixed butterfly combines the lanes; lane 0's
 // value is the result (the same bits on every run).  32 independent load
@@ -458,6 +525,18 @@ cudaError_t launch_direct_partial(const Problem& p, const void* x, const void* d
                                   const DArgs& a, int64_t blocks, cudaStream_t stream) {
     const TA* xt = static_cast<const TA*>(x);
     const TA* gt = static_cast<const TA*>(dy);
+    if (p.layout == DW_NCHW && p.kH == p.kW && (p.kH == 3 || p.kH == 5)) {
+        // one warp per (chunk, output channel) with every tap in registers
+        int64_t nb = (a.chunks * a.Co * 32 + 255) / 256;
+        const int64_t cap = int64_t(sm_count(current_device())) * 8;
+        if (nb > cap) nb = cap;
+        if (nb < 1) nb = 1;
+        if (p.kH == 3)
+            return launch_pdl(partial_direct_nchw_taps<TA, 3, 3>, dim3(unsigned(nb)), dim3(256), 0,
+                              stream, xt, gt, part, a);
+        return launch_pdl(partial_direct_nchw_taps<TA, 5, 5>, dim3(unsigned(nb)), dim3(256), 0,
+                          stream, xt, gt, part, a);
+    }
     return p.layout == DW_NHWC ? launch_pdl(partial_direct_nhwc<TA>, dim3(unsigned(blocks)),
                                             dim3(256), 0, stream, xt, gt, part, a)
                                : launch_pdl(partial_direct_nchw<TA>, dim3(unsigned(blocks)),

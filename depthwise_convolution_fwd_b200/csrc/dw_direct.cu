@@ -119,6 +119,99 @@ __global__ void __launch_bounds__(256) direct_bwd_kernel(const TA* __restrict__ 
     }
 }
 
+// Input gradient of a strided forward with the filter extent and the stride
+// known at compile time (dilation 1, no multiplier): the same gather and the
+// same tap order as direct_bwd_kernel, with 32-bit multiply-shift index
+// decoding and the divisibility tests resolved to masks.  Serves the strided
+// input gradients the tiled families leave to the direct path (NCHW).
+struct StridedArgs {
+    int C, H, W, Ho, Wo, pt, pl, wtype, total;
+    FastDiv fC, fH, fW;
+};
+
+template <int LAYOUT, class TA, int KH, int KW, int S>
+__global__ void __launch_bounds__(256) strided_bwd_kernel(const TA* __restrict__ dy,
+                                                          const void* __restrict__ w,
+                                                          TA* __restrict__ dx, StridedArgs a) {
+    grid_dependency_wait();
+    allow_dependents();
+    const int stride = gridDim.x * blockDim.x;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.total; i += stride) {
+        int n, c, hi, wi;
+        if (LAYOUT == DW_NHWC) {
+            const int q = fast_div(i, a.fC);
+            c = i - q * a.C;
+            const int r = fast_div(q, a.fW);
+            wi = q - r * a.W;
+            n = fast_div(r, a.fH);
+            hi = r - n * a.H;
+        } else {
+            const int q = fast_div(i, a.fW);
+            wi = i - q * a.W;
+            const int r = fast_div(q, a.fH);
+            hi = q - r * a.H;
+            n = fast_div(r, a.fC);
+            c = r - n * a.C;
+        }
+        const int th0 = hi + a.pt, tw0 = wi + a.pl;
+        const int wbase = c * (KH * KW);
+        float acc = 0.f;
+#pragma unroll
+        for (int kh = 0; kh < KH; ++kh) {
+            const int th = th0 - kh;  // = ho * S
+            if (th < 0 || th % S != 0) continue;
+            const int ho = th / S;
+            if (ho >= a.Ho) continue;
+#pragma unroll
+            for (int kw = 0; kw < KW; ++kw) {
+                const int tw = tw0 - kw;  // = wo * S
+                if (tw < 0 || tw % S != 0) continue;
+                const int wo = tw / S;
+                if (wo >= a.Wo) continue;
+                const int off = LAYOUT == DW_NHWC ? ((n * a.Ho + ho) * a.Wo + wo) * a.C + c
+                                                  : ((n * a.C + c) * a.Ho + ho) * a.Wo + wo;
+                acc = fmaf(load_weight(w, a.wtype, wbase + kh * KW + kw), ActIO<TA>::load1(dy + off),
+                           acc);
+            }
+        }
+        ActIO<TA>::store1(dx + i, acc);
+    }
+}
+
+template <class TA, int KH, int KW, int S>
+cudaError_t launch_strided_bwd(const Problem& p, const void* in, const void* w, void* out,
+                               cudaStream_t stream, dim3 grid, dim3 block) {
+    StridedArgs a;
+    a.C = int(p.C); a.H = int(p.H); a.W = int(p.W); a.Ho = int(p.Ho); a.Wo = int(p.Wo);
+    a.pt = p.pt; a.pl = p.pl; a.wtype = p.wtype;
+    a.total = int(p.N * p.C * p.H * p.W);
+    a.fC = make_fastdiv(a.C);
+    a.fH = make_fastdiv(a.H);
+    a.fW = make_fastdiv(a.W);
+    const TA* src = static_cast<const TA*>(in);
+    TA* dst = static_cast<TA*>(out);
+    return p.layout == DW_NHWC
+               ? launch_pdl(strided_bwd_kernel<DW_NHWC, TA, KH, KW, S>, grid, block, 0, stream, src,
+                            w, dst, a)
+               : launch_pdl(strided_bwd_kernel<DW_NCHW, TA, KH, KW, S>, grid, block, 0, stream, src,
+                            w, dst, a);
+}
+
+// The strided input gradients with a compile-time kernel: 3x3, 5x5, 7x7 at
+// stride 2, dilation 1, no multiplier, every index inside int32.
+template <class TA>
+bool try_strided_bwd(const Problem& p, const void* in, const void* w, void* out,
+                     cudaStream_t stream, dim3 grid, dim3 block, cudaError_t* e) {
+    if (p.M != 1 || p.dh != 1 || p.dw != 1 || p.sh != 2 || p.sw != 2 || p.kH != p.kW) return false;
+    const int64_t big = p.N * p.C * (p.H > p.Ho ? p.H : p.Ho) * (p.W > p.Wo ? p.W : p.Wo);
+    if (big >= (int64_t(1) << 30) || p.pt + p.H >= (1 << 29) || p.pl + p.W >= (1 << 29)) return false;
+    if (p.kH == 3) *e = launch_strided_bwd<TA, 3, 3, 2>(p, in, w, out, stream, grid, block);
+    else if (p.kH == 5) *e = launch_strided_bwd<TA, 5, 5, 2>(p, in, w, out, stream, grid, block);
+    else if (p.kH == 7) *e = launch_strided_bwd<TA, 7, 7, 2>(p, in, w, out, stream, grid, block);
+    else return false;
+    return true;
+}
+
 template <class TA, class I>
 cudaError_t launch_typed(const Problem& p, Op op, const void* in, const void* w, const float* b,
                          void* out, cudaStream_t stream, dim3 grid, dim3 block,
@@ -142,6 +235,8 @@ template <class TA>
 cudaError_t launch_index(const Problem& p, Op op, const void* in, const void* w, const float* b,
                          void* out, cudaStream_t stream, dim3 grid, dim3 block,
                          const DirectArgs& a) {
+    cudaError_t e;
+    if (op == OP_BWD_INPUT && try_strided_bwd<TA>(p, in, w, out, stream, grid, block, &e)) return e;
     // every flat index and intermediate (with pads and taps) inside int32?
     const int64_t big = p.N * (p.Co > p.C ? p.Co : p.C) * (p.H > p.Ho ? p.H : p.Ho) *
                         (p.W > p.Wo ? p.W : p.Wo);
