@@ -364,3 +364,62 @@ def test_tiled_forward_with_ragged_output_width(case):
     got = gu.gpu_fwd(case, inp, algo="tiled")
     torch.cuda.synchronize()
     gu.assert_close(got.cpu().numpy(), ref, sc, case.name)
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+@pytest.mark.parametrize("graph", [False, True])
+def test_dependent_calls_with_epilogue_and_gradients(layout, graph):
+    """Stream order across the other calls: the fused forward's output is the
+    next call's dy, whose weight gradient (two kernels and a workspace) and
+    input gradient follow, then a forward of that input gradient; eager and
+    in a CUDA graph, checked against the oracle's composition."""
+    import oracle
+    from depthwise_convolution_fwd_b200.workloads import make_bn
+    N, H, W, C = 2, 36, 64, 32
+    shape = (N, H, W, C) if layout == "nhwc" else (N, C, H, W)
+    g = torch.Generator().manual_seed(123)
+    x = torch.rand(shape, generator=g) * 2 - 1
+    w = torch.randn(C, 3, 3, generator=g) / 3
+    b = torch.rand(C, generator=g) * 0.2 - 0.1
+    bn = make_bn(C, 124)
+    xd, wd, bd = x.cuda(), w.cuda(), b.cuda()
+    bnd = tuple(t.cuda() for t in bn[:4]) + (bn[4],)
+    need = dw.dwconv2d_bwd_weight_workspace_size(dw.make_desc(N, H, W, C, 3, 3, layout=layout))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    gw = torch.empty(C, 3, 3, device="cuda")
+    gb = torch.empty(C, device="cuda")
+
+    def chain(src):
+        y = dw.dwconv2d_fwd_bn_act(src, wd, bd, bnd, "silu", layout=layout)
+        dw.dwconv2d_bwd_weight(src, y, (3, 3), layout=layout, dw=gw, db=gb, workspace=ws)
+        dx = dw.dwconv2d_bwd_input(y, wd, (H, W), layout=layout)
+        return dw.dwconv2d_fwd(dx, wd, bd, layout=layout), y
+
+    if graph:
+        chain(xd)
+        torch.cuda.synchronize()
+        static_in = xd.clone()
+        gr = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        with torch.cuda.graph(gr, stream=s):
+            out, y = chain(static_in)
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+    else:
+        for _ in range(3):
+            out, y = chain(xd)
+        torch.cuda.synchronize()
+
+    p = oracle.problem(shape, 3, 3, 1, 1, "same", layout)
+    xn, wn, bn_ = x.double().numpy(), w.double().numpy(), b.double().numpy()
+    bn64 = tuple(t.double().numpy() for t in bn[:4]) + (bn[4],)
+    y_ref = oracle.fwd_bn_act(p, xn, wn, bn_, bn64, "silu")
+    assert np.abs(y.cpu().double().numpy() - y_ref).max() <= 1e-4 * np.abs(y_ref).max()
+    # the gradients of what the GPU actually produced as y
+    yn = y.cpu().double().numpy()
+    dw_ref, db_ref = oracle.bwd_weight(p, xn, yn)
+    assert np.abs(gw.cpu().double().numpy() - dw_ref).max() <= 1e-4 * np.abs(dw_ref).max()
+    assert np.abs(gb.cpu().double().numpy() - db_ref).max() <= 1e-4 * np.abs(db_ref).max()
+    out_ref = oracle.fwd(p, oracle.bwd_input(p, yn, wn), wn, bn_)
+    assert np.abs(out.cpu().double().numpy() - out_ref).max() <= 1e-4 * np.abs(out_ref).max()
