@@ -48,9 +48,12 @@ struct Args {
 };
 
 template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
-          int MINB_ = 1, class TA_ = float, int S_ = 1>
+          int MINB_ = 1, class TA_ = float, int S_ = 1, int PL_ = 1>
 struct Cfg {
     using TA = TA_;
+    // planes per tile: small planes share a CTA tile, the WY thread rows
+    // split into PL groups of YP rows, one (n, c) plane each
+    static constexpr int PL = PL_;
     static constexpr int S = S_;  // stride (forward only: output (ho, wo) reads row ho*S.., col wo*S..)
     static constexpr int ESZ = sizeof(TA);
     static constexpr int ALIGN = 16 / ESZ;  // elements per 16 bytes
@@ -62,12 +65,13 @@ struct Cfg {
     static constexpr int NCW = WX * WY / 32;  // consumer warps
     static constexpr int NT = WX * WY + 32;   // + one producer warp
     static constexpr int TW = 4 * WX;
-    static constexpr int TH = ROWS ? 1 : THT * WY;
+    static constexpr int YP = WY / PL;  // thread rows per plane
+    static constexpr int TH = ROWS ? 1 : THT * YP;
     static constexpr int IH = ROWS ? 1 : (TH - 1) * S + (KH - 1) * D + 1;
     static constexpr int IWB =
         (REM + (ALIGN - 4) + (TW - 1) * S + (KW - 1) * D + 1 + ALIGN - 1) / ALIGN * ALIGN;
     static constexpr int BOXH = IH;
-    static constexpr int BOXC = ROWS ? WY : 1;
+    static constexpr int BOXC = ROWS ? WY : PL;
     // bytes one TMA box delivers, and the stage pitch: every stage must start
     // on a 128-byte boundary (shared-memory destination rule of tensor copies)
     static constexpr int STAGE_BYTES = IWB * IH * BOXC * ESZ;
@@ -80,6 +84,7 @@ struct Cfg {
     static_assert(STAGE_PITCH % 128 == 0 && (IWB * ESZ) % 16 == 0, "TMA alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
     static_assert(S == 1 || (!REV && !ROWS), "strided tiles: 2-D forward only");
+    static_assert(WY % PL == 0 && (PL == 1 || !ROWS), "whole thread rows per plane");
 };
 
 
@@ -148,7 +153,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 if constexpr (K::ROWS)
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
                 else
-                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt, c, n);
+                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt, c * K::PL, n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -178,7 +183,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
         const int s = k % K::NS;
         int tx, ty, cg, n;
         decode_tile<K>(t, a, tx, ty, cg, n);
-        const int c = K::ROWS ? cg * K::WY + yi : cg;
+        const int c = K::ROWS ? cg * K::WY + yi : cg * K::PL + yi / K::YP;
         const int key = cg + n * a.tiles_c.d;
         if (key != cur_key) {
             cur_key = key;
@@ -221,9 +226,10 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
 
-        const int row0 = K::ROWS ? yi : yi * K::THT;  // first output row of this thread
+        const int row0 = K::ROWS ? yi : (yi % K::YP) * K::THT;  // first output row of this thread
+        const int plane = K::ROWS ? 0 : yi / K::YP;            // the thread's plane in the box
         const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
-                        size_t(row0 * K::S) * K::IWB + 4 * xi * K::S + a.sh4;
+                        size_t(plane * K::IH + row0 * K::S) * K::IWB + 4 * xi * K::S + a.sh4;
         static_for<0, K::RH>([&](auto r_) {
             constexpr int r = decltype(r_)::value;
             float v[4 * K::NV];
@@ -295,7 +301,7 @@ dw_status_t launch(const Problem& p, const void* in, const void* w, const float*
     a.sh4 = sh4;
     const int64_t tx = (a.Wout + K::TW - 1) / K::TW;
     const int64_t ty = K::ROWS ? a.Hout : (a.Hout + K::TH - 1) / K::TH;
-    const int64_t tc = K::ROWS ? (p.C + K::WY - 1) / K::WY : p.C;
+    const int64_t tc = K::ROWS ? (p.C + K::WY - 1) / K::WY : (p.C + K::PL - 1) / K::PL;
     const int64_t nt = tx * ty * tc * p.N;
     if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
     a.tiles_x = make_fastdiv(static_cast<int>(tx));
@@ -665,15 +671,15 @@ dw_status_t launch_chl_op(const Problem& p, Op op, const void* in, const void* w
                                                       -p.pt, (KW - 1) - p.pl);
 }
 
-template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB, class TA>
+template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB, class TA, int PL = 1>
 dw_status_t launch_rem(const Problem& p, const void* in, const void* w, const float* b,
                        void* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
                        int pl_eff) {
     int rem, sh4;
     box_shift<TA>(pl_eff, rem, sh4);
 #define DW_2D(R) \
-    return launch<Cfg<KH, KW, 1, REV, R, THT, WX, WY, NS, MINB, TA>>(p, in, w, b, out, stream, \
-                                                                    err, dry_run, pt_eff, pl_eff, sh4);
+    return launch<Cfg<KH, KW, 1, REV, R, THT, WX, WY, NS, MINB, TA, 1, PL>>(         \
+        p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff, sh4);
     switch (rem) {
         case 0: DW_2D(0)
         case 1: DW_2D(1)
@@ -683,27 +689,27 @@ dw_status_t launch_rem(const Problem& p, const void* in, const void* w, const fl
 #undef DW_2D
 }
 
-template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int MINB = 1>
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int MINB = 1, int PL = 1>
 dw_status_t launch_op(const Problem& p, Op op, const void* in, const void* w, const float* b,
                       void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     if (op == OP_FWD)
-        return launch_rem<KH, KW, false, THT, WX, WY, NS, MINB, TA>(p, in, w, b, out, stream, err,
-                                                                    dry_run, p.pt, p.pl);
-    return launch_rem<KH, KW, true, THT, WX, WY, NS, MINB, TA>(p, in, w, b, out, stream, err,
-                                                               dry_run, (KH - 1) - p.pt,
-                                                               (KW - 1) - p.pl);
+        return launch_rem<KH, KW, false, THT, WX, WY, NS, MINB, TA, PL>(p, in, w, b, out, stream,
+                                                                        err, dry_run, p.pt, p.pl);
+    return launch_rem<KH, KW, true, THT, WX, WY, NS, MINB, TA, PL>(p, in, w, b, out, stream, err,
+                                                                   dry_run, (KH - 1) - p.pt,
+                                                                   (KW - 1) - p.pl);
 }
 
 // Stride-2 forward (2-D kernel with S = 2): a tile is TH x 4*WX outputs, its
 // box the (TH-1)*2 + kH rows and (TW-1)*2 + kW columns they read.
-template <int KH, int KW, int THT, int WX, int WY, int NS, class TA>
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int PL = 1>
 dw_status_t launch_s2_fwd(const Problem& p, const void* in, const void* w, const float* b,
                           void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     int rem, sh4;
     box_shift<TA>(p.pl, rem, sh4);
 #define DW_S2(R) \
-    return launch<Cfg<KH, KW, 1, false, R, THT, WX, WY, NS, 1, TA, 2>>(p, in, w, b, out, stream, \
-                                                                       err, dry_run, p.pt, p.pl, sh4);
+    return launch<Cfg<KH, KW, 1, false, R, THT, WX, WY, NS, 1, TA, 2, PL>>(            \
+        p, in, w, b, out, stream, err, dry_run, p.pt, p.pl, sh4);
     switch (rem) {
         case 0: DW_S2(0)
         case 1: DW_S2(1)
@@ -720,11 +726,21 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
     if (p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
     if (p.sh == 2 && p.sw == 2) {
         // strided: the forward of 3x3 filters (input gradients on the direct kernel)
-        if (op == OP_FWD && p.kH == 3 && p.kW == 3)
+        if (op == OP_FWD && p.kH == 3 && p.kW == 3) {
+            // small planes (at most 32 output columns): 4 planes of 32 x 32 outputs per tile
+            if (p.Wo <= 32)
+                return launch_s2_fwd<3, 3, 4, 8, 32, 3, TA, 4>(p, in, w, b, out, stream, err, dry_run);
             return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA>(p, in, w, b, out, stream, err, dry_run);
+        }
         return DW_ERR_UNSUPPORTED;
     }
     if (p.sh != 1 || p.sw != 1) return DW_ERR_UNSUPPORTED;
+    // small planes (at most 64 columns, the 3x3 and 5x5 filters): 2 planes of
+    // 32 x 64 per tile instead of one plane in a 32 x 128 tile
+    const int64_t wmax = p.W > p.Wo ? p.W : p.Wo;
+    //                                                                    KH KW THT WX WY NS     MINB PL
+    if (wmax <= 64 && p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 16, 16, 4, TA, 1, 2>(p, op, in, w, b, out, stream, err, dry_run);
+    if (wmax <= 64 && p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 16, 16, 4, TA, 1, 2>(p, op, in, w, b, out, stream, err, dry_run);
     //                                                       KH  KW THT WX  WY NS
     if (p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 32, 8, 4, TA>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 32, 8, 4, TA>(p, op, in, w, b, out, stream, err, dry_run);
