@@ -646,17 +646,21 @@ struct NArgs {
     int units;             // N * C * bands
 };
 
-template <int KH_, int KW_, int REM_, int THT_, int WY_, int NS_>
+template <int KH_, int KW_, int REM_, int THT_, int WY_, int NS_, int S_ = 1>
 struct NWCfg {
     static constexpr int KH = KH_, KW = KW_, REM = REM_, THT = THT_, WY = WY_, NS = NS_;
+    // stride S (1 or 2): a lane owns OPL = 4 / S consecutive outputs, whose
+    // input window starts 4 columns after its neighbour's in both cases
+    static constexpr int S = S_, OPL = 4 / S_;
     static constexpr int T = KH * KW + 1;
-    static constexpr int NCW = WY;  // consumer warps, one 128-column row strip each
+    static constexpr int NCW = WY;  // consumer warps, one row strip of 32 * OPL outputs each
     static constexpr int NCT = NCW * 32;
     static constexpr int NT = NCT + 32;
-    static constexpr int TW = 128, TH = THT * WY;
-    static constexpr int IH = TH + KH - 1;
-    static constexpr int IWB = (REM + TW + KW - 1 + 3) / 4 * 4;
-    static constexpr int NV = (REM + 3 + KW - 1) / 4 + 1;  // float4 per window row
+    static constexpr int TW = 32 * OPL, TH = THT * WY;
+    static constexpr int IH = (TH - 1) * S + KH;
+    static constexpr int IWB = (REM + (TW - 1) * S + KW + 3) / 4 * 4;
+    static constexpr int NV = (REM + (OPL - 1) * S + KW - 1) / 4 + 1;  // float4 per window row
+    static_assert(S == 1 || S == 2, "stride 1 or 2");
     static constexpr int XBYTES = IWB * IH * 4;
     static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;
     static constexpr int GBYTES = TW * TH * 4;
@@ -723,8 +727,8 @@ __global__ void __launch_bounds__(K::NT, 1)
                         const int ty = ty0 + r;
                         unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
                         mbar_arrive_expect_tx(&full[s], K::XBYTES + K::GBYTES);
-                        tma_load_4d(st, &xmap, &full[s], tx * K::TW - a.pl - K::REM,
-                                    ty * K::TH - a.pt, c, n);
+                        tma_load_4d(st, &xmap, &full[s], tx * K::TW * K::S - a.pl - K::REM,
+                                    ty * K::TH * K::S - a.pt, c, n);
                         tma_load_4d(st + K::XPITCH, &gmap, &full[s], tx * K::TW, ty * K::TH, c, n);
                     }
             }
@@ -759,20 +763,27 @@ __global__ void __launch_bounds__(K::NT, 1)
                 break;
             }
             const unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
-            const float4* xw = reinterpret_cast<const float4*>(st) + row0 * (K::IWB / 4) + lane;
-            const float4* gw = reinterpret_cast<const float4*>(st + K::XPITCH) + row0 * (K::TW / 4) + lane;
-            float g[K::THT][4];
+            const float4* xw =
+                reinterpret_cast<const float4*>(st) + row0 * K::S * (K::IWB / 4) + lane;
+            const float* gw = reinterpret_cast<const float*>(st + K::XPITCH) + row0 * K::TW +
+                              lane * K::OPL;
+            float g[K::THT][K::OPL];
 #pragma unroll
             for (int j = 0; j < K::THT; ++j) {
-                const float4 f = gw[j * (K::TW / 4)];
-                g[j][0] = f.x; g[j][1] = f.y; g[j][2] = f.z; g[j][3] = f.w;
+                if constexpr (K::OPL == 4) {
+                    const float4 f = *reinterpret_cast<const float4*>(gw + j * K::TW);
+                    g[j][0] = f.x; g[j][1] = f.y; g[j][2] = f.z; g[j][3] = f.w;
+                } else {
+                    const float2 f = *reinterpret_cast<const float2*>(gw + j * K::TW);
+                    g[j][0] = f.x; g[j][1] = f.y;
+                }
             }
             float acc[K::KH][K::KW];
 #pragma unroll
             for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
                 for (int kw = 0; kw < K::KW; ++kw) acc[kh][kw] = 0.f;
-            static_for<0, K::THT + K::KH - 1>([&](auto r_) {
+            static_for<0, (K::THT - 1) * K::S + K::KH>([&](auto r_) {
                 constexpr int r = decltype(r_)::value;
                 float v[4 * K::NV];
 #pragma unroll
@@ -782,13 +793,13 @@ __global__ void __launch_bounds__(K::NT, 1)
                 }
                 static_for<0, K::THT>([&](auto j_) {
                     constexpr int j = decltype(j_)::value;
-                    constexpr int kh = r - j;
+                    constexpr int kh = r - j * K::S;
                     if constexpr (kh >= 0 && kh < K::KH) {
 #pragma unroll
-                        for (int ii = 0; ii < 4; ++ii)
+                        for (int ii = 0; ii < K::OPL; ++ii)
 #pragma unroll
                             for (int kw = 0; kw < K::KW; ++kw)
-                                acc[kh][kw] = fmaf(g[j][ii], v[K::REM + ii + kw], acc[kh][kw]);
+                                acc[kh][kw] = fmaf(g[j][ii], v[K::REM + ii * K::S + kw], acc[kh][kw]);
                     }
                 });
             });
@@ -796,7 +807,10 @@ __global__ void __launch_bounds__(K::NT, 1)
             if (lane == 0) mbar_arrive(&empty[s]);
             float gs = 0.f;
 #pragma unroll
-            for (int j = 0; j < K::THT; ++j) gs += (g[j][0] + g[j][1]) + (g[j][2] + g[j][3]);
+            for (int j = 0; j < K::THT; ++j) {
+                if constexpr (K::OPL == 4) gs += (g[j][0] + g[j][1]) + (g[j][2] + g[j][3]);
+                else gs += g[j][0] + g[j][1];
+            }
 #pragma unroll
             for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
@@ -1166,14 +1180,14 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
-template <int KH, int KW, int THT, int WY, int NS>
+template <int KH, int KW, int THT, int WY, int NS, int S = 1>
 dw_status_t launch_nchw_rem(const Problem& p, const float* x, const float* dy, float* dw,
                             float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
     switch (((-p.pl) % 4 + 4) % 4) {
-        case 0: return launch_tiled_nchw<NWCfg<KH, KW, 0, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        case 1: return launch_tiled_nchw<NWCfg<KH, KW, 1, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        case 2: return launch_tiled_nchw<NWCfg<KH, KW, 2, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        default: return launch_tiled_nchw<NWCfg<KH, KW, 3, THT, WY, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 0: return launch_tiled_nchw<NWCfg<KH, KW, 0, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 1: return launch_tiled_nchw<NWCfg<KH, KW, 1, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 2: return launch_tiled_nchw<NWCfg<KH, KW, 2, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        default: return launch_tiled_nchw<NWCfg<KH, KW, 3, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
     }
 }
 
@@ -1181,11 +1195,16 @@ dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, f
                             float* db, void* ws, cudaStream_t stream, int32_t* err,
                             bool dry_run) {
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
-    if (p.sh != 1 || p.sw != 1 || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
+    if (p.dh != 1 || p.dw != 1 || p.sh != p.sw || p.sh > 2) return DW_ERR_UNSUPPORTED;
     if (p.W % 4 != 0 || p.Wo % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row pitches
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
         return DW_ERR_UNSUPPORTED;
     if (p.N >= INT_MAX || p.C >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    if (p.sh == 2) {
+        //                                                        KH KW THT WY NS S
+        if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3, 2>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        return DW_ERR_UNSUPPORTED;
+    }
     if (p.kH == 1) {
         if (p.kW == 3) return launch_rows_rem<3, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
         if (p.kW == 5) return launch_rows_rem<5, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);

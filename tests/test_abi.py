@@ -188,7 +188,9 @@ def test_weight_gradient_host_checks(lib):
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 7, 7, layout="nchw"), 2, x, dy, dwp) == T
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 18, 32, 3, 3, layout="nchw"), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(
-        dw.make_desc(2, 16, 16, 32, 3, 3, stride=2, layout="nchw"), 2, x, dy, dwp) == D
+        dw.make_desc(2, 16, 16, 32, 3, 3, stride=2, layout="nchw"), 2, x, dy, dwp) == T
+    assert dw.dwconv2d_query_algo(
+        dw.make_desc(2, 16, 16, 32, 5, 5, stride=2, layout="nchw"), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 1, 31, layout="nchw"), 2, x, dy, dwp) == T
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 18, 32, 1, 31, layout="nchw"), 2, x, dy, dwp) == D
     assert dw.dwconv2d_query_algo(dw.make_desc(2, 16, 16, 32, 1, 9, layout="nchw"), 2, x, dy, dwp) == D

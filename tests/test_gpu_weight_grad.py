@@ -86,6 +86,11 @@ TILED = [
          layout="nchw", seed=90),
     Case("w_nchw_1x3", 2, 5, 40, 9, 1, 3, padding=(0, 0, 0, 2), layout="nchw", seed=91),
     Case("w_nchw_1x7", 5, 1, 44, 16, 1, 7, padding=(0, 0, 5, 1), layout="nchw", seed=92),
+    # NCHW, stride 2 (3x3): two outputs per lane, the box start's column phases
+    Case("w_nchw_s2_pad1", 2, 29, 40, 12, 3, 3, stride=2, padding=1, layout="nchw", seed=93),
+    Case("w_nchw_s2_same", 2, 30, 48, 6, 3, 3, stride=2, layout="nchw", seed=94),
+    Case("w_nchw_s2_pl3", 1, 26, 44, 5, 3, 3, stride=2, padding=(1, 1, 3, 2), layout="nchw", seed=95),
+    Case("w_nchw_s2_pl2", 1, 33, 44, 7, 3, 3, stride=2, padding=(2, 0, 2, 4), layout="nchw", seed=96),
 ]
 
 
@@ -111,6 +116,12 @@ def test_repeatable_bit_for_bit():
 @pytest.mark.parametrize("layout", ["nhwc", "nchw"])
 def test_large_full_size(layout):
     case = [c for c in wl.large() if c.H == 512 and c.layout == layout][0]
+    check(case, algos=("auto",))
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+def test_mobilenet_stride2_full_size(layout):
+    case = wl.mobilenet()[2].with_(layout=layout)
     check(case, algos=("auto",))
 
 
