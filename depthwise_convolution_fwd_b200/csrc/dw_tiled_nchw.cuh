@@ -633,6 +633,258 @@ dw_status_t launch_chl(const Problem& p, const void* in, const void* w, const fl
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Input gradient at stride 2 (stride-2 input-VJP sections): dx(hi, wi) gathers
+// W[kh][kw] * dy((hi + pt - kh) / 2, (wi + pl - kw) / 2) over the taps for
+// which both divisions are exact.  A tile is TH x TW dx values at the aligned
+// origin (ty*TH, tx*TW); with PH = pt mod 2 and PW = pl mod 2 as template
+// parameters, every (dx row, tap) and (dx column, tap) pairing is known at
+// compile time.  A lane owns 8 consecutive dx columns, which read 6
+// consecutive dy columns (2 or 3 aligned 4-vectors), and THT rows; results
+// leave as two 4-vectors per row.  The dy box starts at the row
+// ty*TH/2 + floor(pt/2) - AH and at the column tx*TW/2 + floor(pl/2) - AW,
+// moved left by REM (compile time) + sh4 (run time) to a 16-byte boundary.
+template <int KH_, int KW_, int PH_, int PW_, int REM_, int THT_, int WX_, int WY_, int NS_,
+          class TA_>
+struct T2Cfg {
+    using TA = TA_;
+    static constexpr int ESZ = sizeof(TA), ALIGN = 16 / ESZ;
+    static constexpr int KH = KH_, KW = KW_, PH = PH_, PW = PW_, REM = REM_;
+    static constexpr int THT = THT_, WX = WX_, WY = WY_, NS = NS_;
+    static constexpr int NCW = WX * WY / 32, NT = WX * WY + 32;
+    static constexpr int TW = 8 * WX, TH = THT * WY;     // dx tile
+    static constexpr int AH = KH / 2, AW = KW / 2;      // dy rows / columns before the tile's
+    static constexpr int DMAX = (7 + PW) / 2;           // largest (e + PW - kw) / 2
+    static constexpr int NV = (DMAX + AW + REM) / 4 + 1;  // 4-vectors per lane and dy row
+    static constexpr int IH = AH + (TH - 1 + PH) / 2 + 1;
+    static constexpr int IWB =
+        ((TW / 2 - 4 + 4 * NV + (ALIGN - 4)) + ALIGN - 1) / ALIGN * ALIGN;
+    static constexpr int RH = AH + (THT - 1 + PH) / 2 + 1;  // dy rows one thread reads
+    static constexpr int STAGE_BYTES = IWB * IH * ESZ;
+    static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
+    static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NS) * 8 + 16;
+    static_assert(THT % 2 == 0 && (TW / 2) % ALIGN == 0, "even rows, aligned dy columns");
+    static_assert((WX * WY) % 32 == 0, "whole consumer warps");
+    static_assert(IWB <= 256 && IH <= 256, "TMA box dimension limit");
+    static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <class K>
+__global__ void __launch_bounds__(K::NT, 1)
+    t2_kernel(const __grid_constant__ CUtensorMap tmap, const Args a) {
+    using TA = typename K::TA;
+    using IO = ActIO<TA>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(K::NS) * K::STAGE_PITCH);
+    uint64_t* empty = full + K::NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + K::NS);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int t_begin = int((int64_t(blockIdx.x) * a.ntiles) / gridDim.x);
+    const int t_end = int((int64_t(blockIdx.x + 1) * a.ntiles) / gridDim.x);
+
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < K::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], K::NCW);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    grid_dependency_wait();
+    allow_dependents();
+
+    // a.pt, a.pl hold floor(pt/2) and floor(pl/2)
+    if (warp == K::NCW) {
+        if (lane == 0) {
+            prefetch_tensor_map(&tmap);
+            int k = 0;
+            bool ok = true;
+            for (int t = t_begin; t < t_end; ++t, ++k) {
+                const int s = k % K::NS;
+                if (k >= K::NS && !mbar_wait_or_abort(&empty[s], ((k / K::NS) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                int tx, ty, c, n;
+                decode_tile<K>(t, a, tx, ty, c, n);
+                mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
+                tma_load_4d(smem + size_t(s) * K::STAGE_PITCH, &tmap, &full[s],
+                            tx * (K::TW / 2) + a.pl - K::AW - K::REM - a.sh4,
+                            ty * (K::TH / 2) + a.pt - K::AH, c, n);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+                for (int j = (k > K::NS ? k - K::NS : 0); j < k; ++j)
+                    mbar_wait_bounded(&full[j % K::NS], (j / K::NS) & 1);
+            }
+        }
+        return;
+    }
+
+    const int xi = tid % K::WX;
+    const int yi = tid / K::WX;
+    const int row0 = yi * K::THT;  // first dx row of this thread in the tile (even)
+    float wr[K::KH][K::KW];
+    int cur_key = -1;
+    bool live = false;
+    int k = 0;
+    for (int t = t_begin; t < t_end; ++t, ++k) {
+        const int s = k % K::NS;
+        int tx, ty, c, n;
+        decode_tile<K>(t, a, tx, ty, c, n);
+        const int key = c + n * a.tiles_c.d;
+        if (key != cur_key) {
+            cur_key = key;
+            live = c < a.C;
+            const int64_t base = int64_t(live ? c : 0) * (K::KH * K::KW);
+#pragma unroll
+            for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                for (int kw = 0; kw < K::KW; ++kw)
+                    wr[kh][kw] = live ? load_weight(a.w, a.wtype, base + kh * K::KW + kw) : 0.f;
+        }
+        if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
+            }
+            break;
+        }
+        float acc[K::THT][8];
+#pragma unroll
+        for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+        // dy row (row0/2 + rr) of the box and the lane's dy columns from 4*xi
+        const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
+                        size_t(row0 / 2) * K::IWB + 4 * xi + a.sh4;
+        static_for<0, K::RH>([&](auto rr_) {
+            constexpr int rr = decltype(rr_)::value;
+            float v[4 * K::NV];
+#pragma unroll
+            for (int u = 0; u < K::NV; ++u) {
+                const float4 f = IO::load4(win + rr * K::IWB + 4 * u);
+                v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
+            }
+            static_for<0, K::THT>([&](auto j_) {
+                constexpr int j = decltype(j_)::value;
+                static_for<0, K::KH>([&](auto kh_) {
+                    constexpr int kh = decltype(kh_)::value;
+                    // dx row row0 + j reads dy box row row0/2 + (j + PH - kh)/2 + AH
+                    constexpr int num = j + K::PH - kh;
+                    if constexpr (num % 2 == 0 && num / 2 + K::AH == rr) {
+                        static_for<0, 8>([&](auto e_) {
+                            constexpr int e = decltype(e_)::value;
+                            static_for<0, K::KW>([&](auto kw_) {
+                                constexpr int kw = decltype(kw_)::value;
+                                constexpr int numw = e + K::PW - kw;
+                                if constexpr (((numw % 2) + 2) % 2 == 0)
+                                    acc[j][e] = fmaf(wr[kh][kw], v[numw / 2 + K::AW + K::REM], acc[j][e]);
+                            });
+                        });
+                    }
+                });
+            });
+        });
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
+        if (live) {
+            const int wi0 = tx * K::TW + 8 * xi;
+#pragma unroll
+            for (int j = 0; j < K::THT; ++j) {
+                const int hi = ty * K::TH + row0 + j;
+                if (hi >= a.Hout) continue;
+                TA* dst = static_cast<TA*>(a.out) + ((int64_t(n) * a.C + c) * a.Hout + hi) * a.Wout + wi0;
+                const float4 lo = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+                const float4 hi4 = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+                if ((a.Wout & 3) == 0 && wi0 + 7 < a.Wout) {
+                    IO::store4(dst, lo);
+                    IO::store4(dst + 4, hi4);
+                } else {
+                    const float vals[8] = {lo.x, lo.y, lo.z, lo.w, hi4.x, hi4.y, hi4.z, hi4.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (wi0 + e < a.Wout) IO::store1(dst + e, vals[e]);
+                }
+            }
+        }
+    }
+}
+
+template <class K>
+dw_status_t launch_t2(const Problem& p, const void* in, const void* w, void* out,
+                      cudaStream_t stream, int32_t* err, bool dry_run, int sh4) {
+    Args a;
+    a.w = w;
+    a.b = nullptr;
+    a.out = out;
+    a.err = err;
+    a.wtype = p.wtype;
+    a.N = int(p.N);
+    a.C = int(p.C);
+    a.Hout = int(p.H);
+    a.Wout = int(p.W);
+    a.pt = p.pt / 2;  // floor(pt/2), floor(pl/2): the parities are template parameters
+    a.pl = p.pl / 2;
+    a.sh4 = sh4;
+    const int64_t tx = (p.W + K::TW - 1) / K::TW, ty = (p.H + K::TH - 1) / K::TH;
+    const int64_t nt = tx * ty * p.C * p.N;
+    if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
+    a.tiles_x = make_fastdiv(int(tx));
+    a.tiles_y = make_fastdiv(int(ty));
+    a.tiles_c = make_fastdiv(int(p.C));
+    a.ntiles = int(nt);
+    if (dry_run) return DW_OK;
+    static LaunchCache cache;
+    const int dev = current_device();
+    const int occ = prepare_kernel(reinterpret_cast<const void*>(&t2_kernel<K>), K::NT, K::SMEM,
+                                   cache, dev);
+    if (occ < 1) return DW_ERR_CUDA;
+    CUtensorMap map;
+    constexpr cuuint64_t E = K::ESZ;
+    const cuuint64_t dims[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t strides[3] = {cuuint64_t(p.Wo) * E, cuuint64_t(p.Wo * p.Ho) * E,
+                                   cuuint64_t(p.Wo * p.Ho * p.C) * E};
+    const cuuint32_t box[4] = {K::IWB, K::IH, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (encode_tensor_map(&map, ActIO<typename K::TA>::kTma, 4, const_cast<void*>(in), dims,
+                          strides, box, estr) != CUDA_SUCCESS)
+        return DW_ERR_CUDA;
+    int64_t grid = int64_t(sm_count(dev)) * occ;
+    if (grid > a.ntiles) grid = a.ntiles;
+    if (launch_pdl(t2_kernel<K>, dim3(unsigned(grid)), dim3(K::NT), K::SMEM, stream, map, a) !=
+        cudaSuccess)
+        return DW_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
+}
+
+// dispatch on the pad parities and the box remainder
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA>
+dw_status_t launch_t2_any(const Problem& p, const void* in, const void* w, void* out,
+                          cudaStream_t stream, int32_t* err, bool dry_run) {
+    constexpr int align = 16 / int(sizeof(TA));
+    const int full = ((p.pl / 2 - KW / 2) % align + align) % align;  // box start mod 16 bytes
+    const int rem = full % 4, sh4 = full - rem;
+    const int par = (p.pt & 1) * 2 + (p.pl & 1);
+#define DW_T2(PH, PW, R) \
+    return launch_t2<T2Cfg<KH, KW, PH, PW, R, THT, WX, WY, NS, TA>>(p, in, w, out, stream, err, dry_run, sh4);
+#define DW_T2R(PH, PW) \
+    switch (rem) { case 0: DW_T2(PH, PW, 0) case 1: DW_T2(PH, PW, 1) case 2: DW_T2(PH, PW, 2) default: DW_T2(PH, PW, 3) }
+    switch (par) {
+        case 0: DW_T2R(0, 0)
+        case 1: DW_T2R(0, 1)
+        case 2: DW_T2R(1, 0)
+        default: DW_T2R(1, 1)
+    }
+#undef DW_T2R
+#undef DW_T2
+}
+
 // Box shift (-pl) mod (16 bytes / element size): its part mod 4 is the
 // configuration's REM, the rest (0 or 4) the run-time sh4.
 template <class TA>
@@ -731,6 +983,11 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
             if (p.Wo <= 32)
                 return launch_s2_fwd<3, 3, 4, 8, 32, 3, TA, 4>(p, in, w, b, out, stream, err, dry_run);
             return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA>(p, in, w, b, out, stream, err, dry_run);
+        }
+        if (op == OP_BWD_INPUT && p.kH == 3 && p.kW == 3) {
+            //                            KH KW THT WX WY NS
+            if (p.W <= 64) return launch_t2_any<3, 3, 4, 8, 16, 4, TA>(p, in, w, out, stream, err, dry_run);
+            return launch_t2_any<3, 3, 4, 16, 16, 4, TA>(p, in, w, out, stream, err, dry_run);
         }
         return DW_ERR_UNSUPPORTED;
     }

@@ -145,7 +145,8 @@ def test_query_algo_selects_tiled_for_covered_shapes(lib):
     assert q(dw.make_desc(1, 16, 16, 8, 3, 3), align=4) == D             # unaligned pointers
     assert q(dw.make_desc(1, 16, 16, 8, 2, 2)) == D                      # no 2x2 instance
     assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2)) == T        # strided fwd
-    assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2), op=1) == D  # strided bwd
+    assert q(dw.make_desc(1, 16, 16, 8, 3, 3, layout="nchw", stride=2), op=1) == T  # strided bwd
+    assert q(dw.make_desc(1, 16, 12, 8, 3, 3, layout="nchw", stride=2), op=1) == D  # Wo = 6
     assert q(dw.make_desc(1, 16, 16, 8, 5, 5, layout="nchw", stride=2)) == D
     # forcing
     assert q(dw.make_desc(1, 13, 17, 7, 3, 3, algo="direct")) == D

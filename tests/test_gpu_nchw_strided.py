@@ -52,6 +52,31 @@ def test_nchw_stride2_forward(case):
     gu.assert_close(dx.cpu().numpy(), dxr, dxs, f"{case.name} bwd")
 
 
+# input gradient tiles: both pad parities in each direction, ragged dx widths
+BWD = [
+    Case("b2_pad1", 2, 29, 40, 12, 3, 3, stride=2, padding=1, layout="nchw", seed=511),
+    Case("b2_p00", 1, 30, 40, 5, 3, 3, stride=2, padding=(0, 1, 0, 1), layout="nchw", seed=512),
+    Case("b2_p10", 1, 27, 40, 5, 3, 3, stride=2, padding=(1, 0, 0, 1), layout="nchw", seed=513),
+    Case("b2_p01", 2, 22, 40, 3, 3, 3, stride=2, padding=(0, 1, 1, 0), layout="nchw", seed=514),
+    Case("b2_pl3", 1, 25, 36, 7, 3, 3, stride=2, padding=(2, 1, 3, 2), layout="nchw", seed=515),
+    Case("b2_w39", 1, 17, 39, 4, 3, 3, stride=2, padding=1, layout="nchw", seed=516),
+    Case("b2_wide", 1, 12, 296, 3, 3, 3, stride=2, padding=(1, 1, 1, 0), layout="nchw", seed=517),
+]
+
+
+@pytest.mark.parametrize("case", BWD, ids=lambda c: c.name)
+def test_nchw_stride2_input_gradient_tiles(case):
+    inp = gu.inputs(case)
+    dy, w = inp["dy"].cuda(), inp["w"].cuda()
+    dx = torch.empty(case.in_shape(), device="cuda")
+    assert gu.chosen_algo(case, 1, dy, w, dx) == dw.DW_ALGO_TILED
+    ref, scale = gu.reference_bwd(case, inp)
+    for algo in ("tiled", "direct"):
+        got = gu.gpu_bwd(case, inp, algo)
+        torch.cuda.synchronize()
+        gu.assert_close(got.cpu().numpy(), ref, scale, f"{case.name} bwd [{algo}]")
+
+
 @pytest.mark.parametrize("case", CASES[:3], ids=lambda c: c.name)
 def test_nchw_stride2_fused(case):
     inp = gu.inputs(case)
@@ -78,3 +103,9 @@ def test_nchw_stride2_full_size_sampled():
     ref, scale = gu.reference_fwd_at(case, inp, idx)
     gu.assert_close(y.reshape(-1)[torch.from_numpy(idx).cuda()].cpu().numpy(), ref, scale,
                     "mobilenet nchw stride 2 sampled")
+    dx = gu.gpu_bwd(case, inp)
+    torch.cuda.synchronize()
+    idx = gu.structured_sample(tuple(dx.shape), case.layout, rng, count=4000)
+    ref, scale = gu.reference_bwd_at(case, inp, idx)
+    gu.assert_close(dx.reshape(-1)[torch.from_numpy(idx).cuda()].cpu().numpy(), ref, scale,
+                    "mobilenet nchw stride 2 input gradient sampled")
