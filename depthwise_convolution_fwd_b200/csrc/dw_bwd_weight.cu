@@ -640,7 +640,8 @@ dw_status_t launch_tiled(const Problem& p, const void* x, const void* dy, float*
 struct NArgs {
     double* part;
     int32_t* err;
-    int C, pt, pl;
+    int C, pt, pl;         // C: output channels (planes of dy); x plane of o is o / M
+    int M;
     int tiles_x, tiles_y;  // tiles per plane
     int bands, band_rows;  // row bands per plane, tile rows per band
     int units;             // N * C * bands
@@ -715,7 +716,7 @@ __global__ void __launch_bounds__(K::NT, 1)
             for (int u = blockIdx.x; u < a.units && ok; u += G) {
                 int plane, ty0, rows;
                 unit_tiles(u, plane, ty0, rows);
-                const int c = plane % a.C, n = plane / a.C;
+                const int c = plane % a.C, n = plane / a.C;  // c: output channel
                 for (int r = 0; r < rows && ok; ++r)
                     for (int tx = 0; tx < a.tiles_x; ++tx, ++k) {
                         const int s = k % K::NS;
@@ -728,7 +729,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                         unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
                         mbar_arrive_expect_tx(&full[s], K::XBYTES + K::GBYTES);
                         tma_load_4d(st, &xmap, &full[s], tx * K::TW * K::S - a.pl - K::REM,
-                                    ty * K::TH * K::S - a.pt, c, n);
+                                    ty * K::TH * K::S - a.pt, c / a.M, n);
                         tma_load_4d(st + K::XPITCH, &gmap, &full[s], tx * K::TW, ty * K::TH, c, n);
                     }
             }
@@ -1109,14 +1110,14 @@ dw_status_t launch_rows_rem(const Problem& p, const float* x, const float* dy, f
 constexpr int kNchwUnitsCap = 2048;  // bands are added until N*C*bands reaches this
 
 int nchw_bands_cap(const Problem& p) {
-    const int64_t planes = p.N * p.C;
+    const int64_t planes = p.N * p.Co;
     int64_t r = (kNchwUnitsCap + planes - 1) / planes;
     return int(r < 1 ? 1 : r);
 }
 
 size_t tiled_nchw_workspace(const Problem& p) {
-    if (p.layout != DW_NCHW || p.M != 1) return 0;
-    return size_t(p.N) * size_t(p.C) * size_t(nchw_bands_cap(p)) * size_t(p.kH * p.kW + 1) *
+    if (p.layout != DW_NCHW) return 0;
+    return size_t(p.N) * size_t(p.Co) * size_t(nchw_bands_cap(p)) * size_t(p.kH * p.kW + 1) *
            sizeof(double);
 }
 
@@ -1127,14 +1128,15 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     NArgs a;
     a.part = static_cast<double*>(ws);
     a.err = err;
-    a.C = int(p.C);
+    a.C = int(p.Co);
+    a.M = int(p.M);
     a.pt = p.pt;
     a.pl = p.pl;
     const int64_t ty = (p.Ho + K::TH - 1) / K::TH, tx = (p.Wo + K::TW - 1) / K::TW;
     if (ty >= INT_MAX || tx >= INT_MAX) return DW_ERR_UNSUPPORTED;
     a.tiles_x = int(tx);
     a.tiles_y = int(ty);
-    const int64_t planes = p.N * p.C;
+    const int64_t planes = p.N * p.Co;
     // enough units to spread over every SM, never more bands than tile rows
     int64_t bands = (2 * 148 + planes - 1) / planes;
     if (bands > nchw_bands_cap(p)) bands = nchw_bands_cap(p);
@@ -1160,9 +1162,9 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     const cuuint64_t xs[3] = {cuuint64_t(p.W) * 4, cuuint64_t(p.W * p.H) * 4,
                               cuuint64_t(p.W * p.H * p.C) * 4};
     const cuuint32_t xbox[4] = {K::IWB, K::IH, 1, 1};
-    const cuuint64_t gd[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const cuuint64_t gd[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.Co), cuuint64_t(p.N)};
     const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * 4, cuuint64_t(p.Wo * p.Ho) * 4,
-                              cuuint64_t(p.Wo * p.Ho * p.C) * 4};
+                              cuuint64_t(p.Wo * p.Ho * p.Co) * 4};
     const cuuint32_t gbox[4] = {K::TW, K::TH, 1, 1};
     if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
                           xbox, estr) != CUDA_SUCCESS ||
@@ -1172,9 +1174,9 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     if (launch_pdl(partial_tiled_nchw<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap,
                    gmap, a) != cudaSuccess)
         return DW_ERR_CUDA;
-    const int64_t fb = finalize_blocks(p.C * K::T, sm_count(dev));
+    const int64_t fb = finalize_blocks(p.Co * K::T, sm_count(dev));
     if (launch_pdl(finalize_tiled_nchw, dim3(unsigned(fb)), dim3(kFinalizeThreads), 0, stream,
-                   static_cast<const double*>(a.part), dw, db, int(p.N), int(p.C), K::T,
+                   static_cast<const double*>(a.part), dw, db, int(p.N), int(p.Co), K::T,
                    a.bands) != cudaSuccess)
         return DW_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
@@ -1263,6 +1265,12 @@ dw_status_t tiled_pick_mult(const Problem& p, const void* x, const void* dy, flo
 
 dw_status_t tiled_pick(const Problem& p, const void* x, const void* dy, float* dw, float* db,
                        void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.M != 1 && p.layout == DW_NCHW) {
+        // channel multiplier, NCHW: the plane-per-unit tiles (2-D filters, float32)
+        if (p.atype != DW_F32 || p.kH == 1) return DW_ERR_UNSUPPORTED;
+        return tiled_pick_nchw(p, static_cast<const float*>(x), static_cast<const float*>(dy), dw,
+                               db, ws, stream, err, dry_run);
+    }
     if (p.M != 1) {
         // channel multiplier: float32 NHWC tiles for M = 2, 4; else the direct kernels
         if (p.layout != DW_NHWC || p.atype != DW_F32 || (p.M != 2 && p.M != 4)) return DW_ERR_UNSUPPORTED;

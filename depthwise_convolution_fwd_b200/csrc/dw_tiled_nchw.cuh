@@ -39,7 +39,8 @@ struct Args {
     void* out;   // elements of the configuration's activation type
     int32_t* err;
     int wtype;
-    int N, C, Hout, Wout;
+    int N, C, Hout, Wout;  // C: channels of the tensor written (C*M for a forward)
+    int M;                 // channel multiplier of the 2-D forward (1 elsewhere)
     int pt, pl;  // effective low pads of the correlation this kernel runs
     int sh4;     // extra box shift beyond REM (0, or 4 for 16-bit elements)
     FastDiv tiles_x, tiles_y, tiles_c;
@@ -153,7 +154,9 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 if constexpr (K::ROWS)
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
                 else
-                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt, c * K::PL, n);
+                    // output plane c reads input plane c / M (one plane per tile when M > 1)
+                    tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt,
+                                K::PL == 1 ? c / a.M : c * K::PL, n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -293,7 +296,10 @@ dw_status_t launch(const Problem& p, const void* in, const void* w, const float*
     a.err = err;
     a.wtype = p.wtype;
     a.N = static_cast<int>(p.N);
-    a.C = static_cast<int>(p.C);
+    // channel multiplier: the 2-D forward with one plane per tile
+    if (p.M != 1 && (K::REV || K::ROWS || K::PL != 1)) return DW_ERR_UNSUPPORTED;
+    a.M = static_cast<int>(p.M);
+    a.C = static_cast<int>(K::REV ? p.C : p.Co);
     a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
     a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
     a.pt = pt_eff;
@@ -301,7 +307,7 @@ dw_status_t launch(const Problem& p, const void* in, const void* w, const float*
     a.sh4 = sh4;
     const int64_t tx = (a.Wout + K::TW - 1) / K::TW;
     const int64_t ty = K::ROWS ? a.Hout : (a.Hout + K::TH - 1) / K::TH;
-    const int64_t tc = K::ROWS ? (p.C + K::WY - 1) / K::WY : (p.C + K::PL - 1) / K::PL;
+    const int64_t tc = K::ROWS ? (a.C + K::WY - 1) / K::WY : (a.C + K::PL - 1) / K::PL;
     const int64_t nt = tx * ty * tc * p.N;
     if (nt >= INT_MAX) return DW_ERR_UNSUPPORTED;
     a.tiles_x = make_fastdiv(static_cast<int>(tx));
@@ -569,6 +575,8 @@ dw_status_t launch_chl(const Problem& p, const void* in, const void* w, const fl
     a.err = err;
     a.wtype = p.wtype;
     a.N = static_cast<int>(p.N);
+    if (p.M != 1) return DW_ERR_UNSUPPORTED;  // boxes of 32 consecutive channels
+    a.M = 1;
     a.C = static_cast<int>(p.C);
     a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
     a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
@@ -825,6 +833,8 @@ dw_status_t launch_t2(const Problem& p, const void* in, const void* w, void* out
     a.out = out;
     a.err = err;
     a.wtype = p.wtype;
+    if (p.M != 1) return DW_ERR_UNSUPPORTED;
+    a.M = 1;
     a.N = int(p.N);
     a.C = int(p.C);
     a.Hout = int(p.H);
@@ -980,7 +990,7 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
         // strided: the forward of 3x3 filters (input gradients on the direct kernel)
         if (op == OP_FWD && p.kH == 3 && p.kW == 3) {
             // small planes (at most 32 output columns): 4 planes of 32 x 32 outputs per tile
-            if (p.Wo <= 32)
+            if (p.Wo <= 32 && p.M == 1)
                 return launch_s2_fwd<3, 3, 4, 8, 32, 3, TA, 4>(p, in, w, b, out, stream, err, dry_run);
             return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA>(p, in, w, b, out, stream, err, dry_run);
         }
@@ -996,8 +1006,9 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
     // 32 x 64 per tile instead of one plane in a 32 x 128 tile
     const int64_t wmax = p.W > p.Wo ? p.W : p.Wo;
     //                                                                    KH KW THT WX WY NS     MINB PL
-    if (wmax <= 64 && p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 16, 16, 4, TA, 1, 2>(p, op, in, w, b, out, stream, err, dry_run);
-    if (wmax <= 64 && p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 16, 16, 4, TA, 1, 2>(p, op, in, w, b, out, stream, err, dry_run);
+    const bool small = wmax <= 64 && p.M == 1;  // several planes per tile need M = 1
+    if (small && p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 16, 16, 4, TA, 1, 2>(p, op, in, w, b, out, stream, err, dry_run);
+    if (small && p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 16, 16, 4, TA, 1, 2>(p, op, in, w, b, out, stream, err, dry_run);
     //                                                       KH  KW THT WX  WY NS
     if (p.kH == 3 && p.kW == 3) return launch_op<3, 3, 4, 32, 8, 4, TA>(p, op, in, w, b, out, stream, err, dry_run);
     if (p.kH == 5 && p.kW == 5) return launch_op<5, 5, 4, 32, 8, 4, TA>(p, op, in, w, b, out, stream, err, dry_run);

@@ -158,3 +158,21 @@ def test_tiled_multiplier_input_gradient(case):
         got = gu.gpu_bwd(case, inp, algo)
         torch.cuda.synchronize()
         gu.assert_close(got.cpu().numpy(), ref, scale, f"{case.name} bwd_input [{algo}]")
+
+
+NCHW_TILED = [
+    Case("mn2_3x3", 2, 21, 40, 6, 3, 3, multiplier=2, layout="nchw", seed=331),
+    Case("mn4_5x5", 1, 19, 96, 3, 5, 5, multiplier=4, layout="nchw", seed=332),
+    Case("mn3_7x7", 1, 17, 36, 2, 7, 7, multiplier=3, layout="nchw", seed=333),
+    Case("mn2_s2", 2, 29, 80, 4, 3, 3, stride=2, padding=1, multiplier=2, layout="nchw", seed=334),
+]
+
+
+@pytest.mark.parametrize("case", NCHW_TILED, ids=lambda c: c.name)
+def test_nchw_multiplier_tiles(case):
+    inp = gu.inputs(case)
+    x, w = inp["x"].cuda(), inp["w"].cuda()
+    y = torch.empty(case.out_shape(*gu.out_hw(case)), device="cuda")
+    assert gu.chosen_algo(case, 0, x, w, y) == dw.DW_ALGO_TILED
+    assert gu.chosen_algo(case, 2, x, y, w) == dw.DW_ALGO_TILED
+    check_all(case, fwd_algos=("tiled", "direct"))
