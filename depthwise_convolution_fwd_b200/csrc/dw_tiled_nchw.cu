@@ -18,8 +18,6 @@ dw_status_t tiled_nchw_launch(const Problem& p, Op op, const void* in, const voi
                               bool dry_run) {
     using namespace nchw;
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
-    // channel multiplier: the forward's one-plane tiles; gradients on the direct kernels
-    if (p.M != 1 && op != OP_FWD) return DW_ERR_UNSUPPORTED;
     const int64_t Win = op == OP_FWD ? p.W : p.Wo;
     // TMA row stride: a multiple of 16 bytes
     if ((Win * act_bytes(p.atype)) % 16 != 0) return DW_ERR_UNSUPPORTED;

@@ -49,12 +49,15 @@ struct Args {
 };
 
 template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
-          int MINB_ = 1, class TA_ = float, int S_ = 1, int PL_ = 1>
+          int MINB_ = 1, class TA_ = float, int S_ = 1, int PL_ = 1, int MB_ = 1>
 struct Cfg {
     using TA = TA_;
     // planes per tile: small planes share a CTA tile, the WY thread rows
     // split into PL groups of YP rows, one (n, c) plane each
     static constexpr int PL = PL_;
+    // input gradient with a channel multiplier: dx plane c is the sum of the
+    // reversed correlations of the MB dy planes c*MB .. c*MB+MB-1 (one box)
+    static constexpr int MB = MB_;
     static constexpr int S = S_;  // stride (forward only: output (ho, wo) reads row ho*S.., col wo*S..)
     static constexpr int ESZ = sizeof(TA);
     static constexpr int ALIGN = 16 / ESZ;  // elements per 16 bytes
@@ -72,7 +75,7 @@ struct Cfg {
     static constexpr int IWB =
         (REM + (ALIGN - 4) + (TW - 1) * S + (KW - 1) * D + 1 + ALIGN - 1) / ALIGN * ALIGN;
     static constexpr int BOXH = IH;
-    static constexpr int BOXC = ROWS ? WY : PL;
+    static constexpr int BOXC = ROWS ? WY : PL * MB;
     // bytes one TMA box delivers, and the stage pitch: every stage must start
     // on a 128-byte boundary (shared-memory destination rule of tensor copies)
     static constexpr int STAGE_BYTES = IWB * IH * BOXC * ESZ;
@@ -86,6 +89,7 @@ struct Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
     static_assert(S == 1 || (!REV && !ROWS), "strided tiles: 2-D forward only");
     static_assert(WY % PL == 0 && (PL == 1 || !ROWS), "whole thread rows per plane");
+    static_assert(MB == 1 || (REV && !ROWS && PL == 1), "summed dy planes: 2-D input gradient");
 };
 
 
@@ -154,9 +158,10 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 if constexpr (K::ROWS)
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
                 else
-                    // output plane c reads input plane c / M (one plane per tile when M > 1)
+                    // forward: output plane c reads input plane c / M (one plane per
+                    // tile when M > 1); multiplier input gradient: dy planes c*MB..
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt,
-                                K::PL == 1 ? c / a.M : c * K::PL, n);
+                                K::MB > 1 ? c * K::MB : (K::PL == 1 ? c / a.M : c * K::PL), n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     // -------------------------- consumer warps --------------------------------
     const int xi = tid % K::WX;
     const int yi = tid / K::WX;
-    float wr[K::KH][K::KW];
+    float wr[K::MB][K::KH][K::KW];
     float bias = 0.f;
     int cur_key = -1;
     bool live = false;
@@ -191,15 +196,19 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
         if (key != cur_key) {
             cur_key = key;
             live = c < a.C;
-            const int64_t base = int64_t(live ? c : 0) * (K::KH * K::KW);
 #pragma unroll
-            for (int kh = 0; kh < K::KH; ++kh)
+            for (int m = 0; m < K::MB; ++m) {
+                // filter of output channel c*MB + m (MB = 1: channel c)
+                const int64_t base = (int64_t(live ? c : 0) * K::MB + m) * (K::KH * K::KW);
 #pragma unroll
-                for (int kw = 0; kw < K::KW; ++kw) {
-                    const int src = K::REV ? (K::KH - 1 - kh) * K::KW + (K::KW - 1 - kw)
-                                           : kh * K::KW + kw;
-                    wr[kh][kw] = live ? load_weight(a.w, a.wtype, base + src) : 0.f;
-                }
+                for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                    for (int kw = 0; kw < K::KW; ++kw) {
+                        const int src = K::REV ? (K::KH - 1 - kh) * K::KW + (K::KW - 1 - kw)
+                                               : kh * K::KW + kw;
+                        wr[m][kh][kw] = live ? load_weight(a.w, a.wtype, base + src) : 0.f;
+                    }
+            }
             bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
             if constexpr (EPI != kNoEpilogue) {
                 // fold the normalisation into the filter and the bias
@@ -209,7 +218,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 #pragma unroll
                     for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw] *= sc;
+                        for (int kw = 0; kw < K::KW; ++kw) wr[0][kh][kw] *= sc;
                     bias = fmaf(bias, sc, sh);
                 }
             }
@@ -231,30 +240,35 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 
         const int row0 = K::ROWS ? yi : (yi % K::YP) * K::THT;  // first output row of this thread
         const int plane = K::ROWS ? 0 : yi / K::YP;            // the thread's plane in the box
-        const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
-                        size_t(plane * K::IH + row0 * K::S) * K::IWB + 4 * xi * K::S + a.sh4;
-        static_for<0, K::RH>([&](auto r_) {
-            constexpr int r = decltype(r_)::value;
-            float v[4 * K::NV];
+        const TA* win0 = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
+                         size_t(plane * K::IH + row0 * K::S) * K::IWB + 4 * xi * K::S + a.sh4;
+        static_for<0, K::MB>([&](auto m_) {
+            constexpr int m = decltype(m_)::value;
+            const TA* win = win0 + size_t(m) * K::IH * K::IWB;  // dy plane c*MB + m
+            static_for<0, K::RH>([&](auto r_) {
+                constexpr int r = decltype(r_)::value;
+                float v[4 * K::NV];
 #pragma unroll
-            for (int u = 0; u < K::NV; ++u) {
-                const float4 f = IO::load4(win + r * K::IWB + 4 * u);
-                v[4 * u] = f.x;
-                v[4 * u + 1] = f.y;
-                v[4 * u + 2] = f.z;
-                v[4 * u + 3] = f.w;
-            }
-            static_for<0, K::THT>([&](auto j_) {
-                constexpr int j = decltype(j_)::value;
-                constexpr int khn = r - j * K::S;
-                if constexpr (khn >= 0 && khn % K::D == 0 && khn / K::D < K::KH) {
-                    constexpr int kh = khn / K::D;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw)
-                            acc[j][i] = fmaf(v[K::REM + i * K::S + kw * K::D], wr[kh][kw], acc[j][i]);
+                for (int u = 0; u < K::NV; ++u) {
+                    const float4 f = IO::load4(win + r * K::IWB + 4 * u);
+                    v[4 * u] = f.x;
+                    v[4 * u + 1] = f.y;
+                    v[4 * u + 2] = f.z;
+                    v[4 * u + 3] = f.w;
                 }
+                static_for<0, K::THT>([&](auto j_) {
+                    constexpr int j = decltype(j_)::value;
+                    constexpr int khn = r - j * K::S;
+                    if constexpr (khn >= 0 && khn % K::D == 0 && khn / K::D < K::KH) {
+                        constexpr int kh = khn / K::D;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int kw = 0; kw < K::KW; ++kw)
+                                acc[j][i] = fmaf(v[K::REM + i * K::S + kw * K::D], wr[m][kh][kw],
+                                                 acc[j][i]);
+                    }
+                });
             });
         });
 
@@ -296,9 +310,10 @@ dw_status_t launch(const Problem& p, const void* in, const void* w, const float*
     a.err = err;
     a.wtype = p.wtype;
     a.N = static_cast<int>(p.N);
-    // channel multiplier: the 2-D forward with one plane per tile
-    if (p.M != 1 && (K::REV || K::ROWS || K::PL != 1)) return DW_ERR_UNSUPPORTED;
-    a.M = static_cast<int>(p.M);
+    // channel multiplier: the 2-D forward with one plane per tile, or the
+    // 2-D input gradient summing MB = M dy planes
+    if (K::REV ? p.M != K::MB : (p.M != 1 && (K::ROWS || K::PL != 1))) return DW_ERR_UNSUPPORTED;
+    a.M = K::REV ? 1 : static_cast<int>(p.M);
     a.C = static_cast<int>(K::REV ? p.C : p.Co);
     a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
     a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
@@ -332,10 +347,11 @@ dw_status_t launch(const Problem& p, const void* in, const void* w, const float*
     if (occ < 1) return DW_ERR_CUDA;
 
     CUtensorMap map;
-    const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(p.C), cuuint64_t(p.N)};
+    const int64_t Cin = K::REV ? p.Co : p.C;  // planes of the tensor read (dy: C*M)
+    const cuuint64_t dims[4] = {cuuint64_t(Win), cuuint64_t(Hin), cuuint64_t(Cin), cuuint64_t(p.N)};
     constexpr cuuint64_t E = K::ESZ;
     const cuuint64_t strides[3] = {cuuint64_t(Win) * E, cuuint64_t(Win * Hin) * E,
-                                   cuuint64_t(Win * Hin * p.C) * E};
+                                   cuuint64_t(Win * Hin * Cin) * E};
     const cuuint32_t box[4] = {K::IWB, K::BOXH, K::BOXC, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     if (encode_tensor_map(&map, ActIO<typename K::TA>::kTma, 4, const_cast<void*>(in), dims,
@@ -933,14 +949,15 @@ dw_status_t launch_chl_op(const Problem& p, Op op, const void* in, const void* w
                                                       -p.pt, (KW - 1) - p.pl);
 }
 
-template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB, class TA, int PL = 1>
+template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB, class TA, int PL = 1,
+          int MB = 1>
 dw_status_t launch_rem(const Problem& p, const void* in, const void* w, const float* b,
                        void* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
                        int pl_eff) {
     int rem, sh4;
     box_shift<TA>(pl_eff, rem, sh4);
 #define DW_2D(R) \
-    return launch<Cfg<KH, KW, 1, REV, R, THT, WX, WY, NS, MINB, TA, 1, PL>>(         \
+    return launch<Cfg<KH, KW, 1, REV, R, THT, WX, WY, NS, MINB, TA, 1, PL, MB>>(     \
         p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff, sh4);
     switch (rem) {
         case 0: DW_2D(0)
@@ -960,6 +977,15 @@ dw_status_t launch_op(const Problem& p, Op op, const void* in, const void* w, co
     return launch_rem<KH, KW, true, THT, WX, WY, NS, MINB, TA, PL>(p, in, w, b, out, stream, err,
                                                                    dry_run, (KH - 1) - p.pt,
                                                                    (KW - 1) - p.pl);
+}
+
+// Input gradient with channel multiplier MB (stride 1): one box holds the MB
+// dy planes of a dx plane, summed in the window loop.
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int MB>
+dw_status_t launch_mult_bwd(const Problem& p, const void* in, const void* w, void* out,
+                            cudaStream_t stream, int32_t* err, bool dry_run) {
+    return launch_rem<KH, KW, true, THT, WX, WY, NS, 1, TA, 1, MB>(
+        p, in, w, nullptr, out, stream, err, dry_run, (KH - 1) - p.pt, (KW - 1) - p.pl);
 }
 
 // Stride-2 forward (2-D kernel with S = 2): a tile is TH x 4*WX outputs, its
@@ -1002,6 +1028,14 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
         return DW_ERR_UNSUPPORTED;
     }
     if (p.sh != 1 || p.sw != 1) return DW_ERR_UNSUPPORTED;
+    if (p.M != 1 && op == OP_BWD_INPUT) {
+        //                                                            KH KW THT WX WY NS     MB
+        if (p.kH == 3 && p.kW == 3 && p.M == 2) return launch_mult_bwd<3, 3, 4, 32, 8, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
+        if (p.kH == 3 && p.kW == 3 && p.M == 4) return launch_mult_bwd<3, 3, 2, 32, 8, 4, TA, 4>(p, in, w, out, stream, err, dry_run);
+        if (p.kH == 5 && p.kW == 5 && p.M == 2) return launch_mult_bwd<5, 5, 4, 32, 8, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
+        if (p.kH == 7 && p.kW == 7 && p.M == 2) return launch_mult_bwd<7, 7, 4, 32, 4, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
+        return DW_ERR_UNSUPPORTED;
+    }
     // small planes (at most 64 columns, the 3x3 and 5x5 filters): 2 planes of
     // 32 x 64 per tile instead of one plane in a 32 x 128 tile
     const int64_t wmax = p.W > p.Wo ? p.W : p.Wo;

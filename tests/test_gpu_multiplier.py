@@ -176,3 +176,47 @@ def test_nchw_multiplier_tiles(case):
     assert gu.chosen_algo(case, 0, x, w, y) == dw.DW_ALGO_TILED
     assert gu.chosen_algo(case, 2, x, y, w) == dw.DW_ALGO_TILED
     check_all(case, fwd_algos=("tiled", "direct"))
+
+
+# NCHW input gradient with a multiplier: one box of M dy planes per dx tile
+# (stride 1; 3x3 with M = 2, 4, 5x5 and 7x7 with M = 2; dy rows a multiple of
+# 16 bytes)
+NCHW_BWD = [
+    Case("mnb2_3x3", 2, 21, 40, 6, 3, 3, multiplier=2, layout="nchw", seed=341),
+    Case("mnb4_3x3_pad", 1, 19, 36, 5, 3, 3, padding=(0, 2, 3, 3), multiplier=4,
+         layout="nchw", seed=342),
+    Case("mnb2_5x5", 2, 35, 48, 3, 5, 5, multiplier=2, layout="nchw", seed=343),
+    Case("mnb2_7x7_wide", 1, 17, 260, 2, 7, 7, multiplier=2, layout="nchw", seed=344),
+    Case("mnb2_3x3_many", 4, 64, 64, 8, 3, 3, multiplier=2, layout="nchw", seed=345),
+]
+
+
+@pytest.mark.parametrize("case", NCHW_BWD, ids=lambda c: c.name)
+def test_nchw_multiplier_input_gradient_tiles(case):
+    inp = gu.inputs(case)
+    dy, w = inp["dy"].cuda(), inp["w"].cuda()
+    dx = torch.empty(case.in_shape(), device="cuda")
+    assert gu.chosen_algo(case, 1, dy, w, dx) == dw.DW_ALGO_TILED
+    ref, scale = gu.reference_bwd(case, inp)
+    for algo in ("tiled", "direct"):
+        got = gu.gpu_bwd(case, inp, algo)
+        torch.cuda.synchronize()
+        gu.assert_close(got.cpu().numpy(), ref, scale, f"{case.name} bwd_input [{algo}]")
+
+
+@pytest.mark.parametrize("name", ["f16", "bf16"])
+@pytest.mark.parametrize("case", [NCHW_BWD[0], NCHW_TILED[1]], ids=lambda c: c.name)
+def test_nchw_multiplier_half(case, name):
+    from tests import test_gpu_half_activations as ha
+    dt, _ = ha.DTYPES[name]
+    inp = ha.inputs16(case, dt)
+    x = inp["x"].cuda()
+    Ho, Wo = gu.out_hw(case)
+    y = torch.empty(case.out_shape(Ho, Wo), device="cuda", dtype=dt)
+    desc = gu.desc_of(case)
+    desc.atype = {"f16": dw.DW_F16, "bf16": dw.DW_BF16}[name]
+    wp = inp["w"].cuda().data_ptr()
+    assert dw.dwconv2d_query_algo(desc, 0, x.data_ptr(), wp, y.data_ptr()) == dw.DW_ALGO_TILED
+    if case in NCHW_BWD:
+        assert dw.dwconv2d_query_algo(desc, 1, y.data_ptr(), wp, x.data_ptr()) == dw.DW_ALGO_TILED
+    ha.run_case(case, name, "auto")
