@@ -39,8 +39,9 @@ struct Args {
     void* out;   // elements of the configuration's activation type
     int32_t* err;
     int wtype;
-    int N, C, Hout, Wout;  // C: channels of the tensor written (C*M for a forward)
-    int M;                 // channel multiplier of the 2-D forward (1 elsewhere)
+    int N, C, Hout, Wout;  // C: channels the tiles run over
+    int Cout;              // channels of the tensor written
+    int M;                 // forward, one output plane per tile: it reads input plane c / M
     int pt, pl;  // effective low pads of the correlation this kernel runs
     int sh4;     // extra box shift beyond REM (0, or 4 for 16-bit elements)
     FastDiv tiles_x, tiles_y, tiles_c;
@@ -49,15 +50,19 @@ struct Args {
 };
 
 template <int KH_, int KW_, int D_, bool REV_, int REM_, int THT_, int WX_, int WY_, int NS_,
-          int MINB_ = 1, class TA_ = float, int S_ = 1, int PL_ = 1, int MB_ = 1>
+          int MINB_ = 1, class TA_ = float, int S_ = 1, int PL_ = 1, int MP_ = 1>
 struct Cfg {
     using TA = TA_;
     // planes per tile: small planes share a CTA tile, the WY thread rows
     // split into PL groups of YP rows, one (n, c) plane each
     static constexpr int PL = PL_;
-    // input gradient with a channel multiplier: dx plane c is the sum of the
-    // reversed correlations of the MB dy planes c*MB .. c*MB+MB-1 (one box)
-    static constexpr int MB = MB_;
+    // channel multiplier inside a tile: in the forward one input plane c feeds
+    // the MP output planes c*MP .. c*MP+MP-1 (NA accumulator sets per thread);
+    // in the input gradient one box holds the MP dy planes c*MP .. whose
+    // reversed correlations sum into dx plane c (NB planes per box)
+    static constexpr int MP = MP_;
+    static constexpr int NA = REV_ ? 1 : MP;
+    static constexpr int NB = REV_ ? MP : 1;
     static constexpr int S = S_;  // stride (forward only: output (ho, wo) reads row ho*S.., col wo*S..)
     static constexpr int ESZ = sizeof(TA);
     static constexpr int ALIGN = 16 / ESZ;  // elements per 16 bytes
@@ -75,7 +80,7 @@ struct Cfg {
     static constexpr int IWB =
         (REM + (ALIGN - 4) + (TW - 1) * S + (KW - 1) * D + 1 + ALIGN - 1) / ALIGN * ALIGN;
     static constexpr int BOXH = IH;
-    static constexpr int BOXC = ROWS ? WY : PL * MB;
+    static constexpr int BOXC = ROWS ? WY : PL * NB;
     // bytes one TMA box delivers, and the stage pitch: every stage must start
     // on a 128-byte boundary (shared-memory destination rule of tensor copies)
     static constexpr int STAGE_BYTES = IWB * IH * BOXC * ESZ;
@@ -89,7 +94,7 @@ struct Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
     static_assert(S == 1 || (!REV && !ROWS), "strided tiles: 2-D forward only");
     static_assert(WY % PL == 0 && (PL == 1 || !ROWS), "whole thread rows per plane");
-    static_assert(MB == 1 || (REV && !ROWS && PL == 1), "summed dy planes: 2-D input gradient");
+    static_assert(MP == 1 || (!ROWS && PL == 1), "multiplier planes: 2-D tiles of one plane");
 };
 
 
@@ -158,10 +163,11 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                 if constexpr (K::ROWS)
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty - a.pt, c * K::WY, n);
                 else
-                    // forward: output plane c reads input plane c / M (one plane per
-                    // tile when M > 1); multiplier input gradient: dy planes c*MB..
+                    // input gradient: dy planes c*PL*MP..; forward: PL input planes
+                    // c*PL.., or input plane c / M for one output plane c per tile
                     tma_load_4d(dst, &tmap, &full[s], ix0, ty * K::TH * K::S - a.pt,
-                                K::MB > 1 ? c * K::MB : (K::PL == 1 ? c / a.M : c * K::PL), n);
+                                K::REV ? c * K::PL * K::MP : (K::PL > 1 ? c * K::PL : c / a.M),
+                                n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -176,14 +182,14 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     // -------------------------- consumer warps --------------------------------
     const int xi = tid % K::WX;
     const int yi = tid / K::WX;
-    float wr[K::MB][K::KH][K::KW];
-    float bias = 0.f;
+    float wr[K::MP][K::KH][K::KW];
+    float bias[K::NA];
     int cur_key = -1;
     bool live = false;
-    // the value stored for one output: acc + bias (-> epilogue)
-    auto finish = [&](float v) -> float {
-        if constexpr (EPI != kNoEpilogue) return activate<EPI>(v + bias);
-        else return v + bias;
+    // the value stored for output set q: acc + bias (-> epilogue)
+    auto finish = [&](float v, int q) -> float {
+        if constexpr (EPI != kNoEpilogue) return activate<EPI>(v + bias[q]);
+        else return v + bias[q];
     };
 
     int k = 0;
@@ -197,9 +203,9 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
             cur_key = key;
             live = c < a.C;
 #pragma unroll
-            for (int m = 0; m < K::MB; ++m) {
-                // filter of output channel c*MB + m (MB = 1: channel c)
-                const int64_t base = (int64_t(live ? c : 0) * K::MB + m) * (K::KH * K::KW);
+            for (int m = 0; m < K::MP; ++m) {
+                // filter of channel c*MP + m (MP = 1: channel c)
+                const int64_t base = (int64_t(live ? c : 0) * K::MP + m) * (K::KH * K::KW);
 #pragma unroll
                 for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
@@ -209,17 +215,21 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                         wr[m][kh][kw] = live ? load_weight(a.w, a.wtype, base + src) : 0.f;
                     }
             }
-            bias = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + c) : 0.f;
-            if constexpr (EPI != kNoEpilogue) {
-                // fold the normalisation into the filter and the bias
-                if (live) {
-                    float sc, sh;
-                    bn_scale_shift(a.epi, c, sc, sh);
 #pragma unroll
-                    for (int kh = 0; kh < K::KH; ++kh)
+            for (int q = 0; q < K::NA; ++q) {
+                const int oc = c * K::NA + q;  // output channel of set q
+                bias[q] = (!K::REV && a.b != nullptr && live) ? __ldg(a.b + oc) : 0.f;
+                if constexpr (EPI != kNoEpilogue) {
+                    // fold the normalisation into the filter and the bias
+                    if (live) {
+                        float sc, sh;
+                        bn_scale_shift(a.epi, oc, sc, sh);
 #pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw) wr[0][kh][kw] *= sc;
-                    bias = fmaf(bias, sc, sh);
+                        for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                            for (int kw = 0; kw < K::KW; ++kw) wr[q][kh][kw] *= sc;
+                        bias[q] = fmaf(bias[q], sc, sh);
+                    }
                 }
             }
         }
@@ -232,19 +242,21 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
             break;
         }
 
-        float acc[K::THT][4];
+        float acc[K::NA][K::THT][4];
 #pragma unroll
-        for (int j = 0; j < K::THT; ++j)
+        for (int q = 0; q < K::NA; ++q)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+            for (int j = 0; j < K::THT; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[q][j][i] = 0.f;
 
         const int row0 = K::ROWS ? yi : (yi % K::YP) * K::THT;  // first output row of this thread
         const int plane = K::ROWS ? 0 : yi / K::YP;            // the thread's plane in the box
         const TA* win0 = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
                          size_t(plane * K::IH + row0 * K::S) * K::IWB + 4 * xi * K::S + a.sh4;
-        static_for<0, K::MB>([&](auto m_) {
-            constexpr int m = decltype(m_)::value;
-            const TA* win = win0 + size_t(m) * K::IH * K::IWB;  // dy plane c*MB + m
+        static_for<0, K::NB>([&](auto b_) {
+            constexpr int pb = decltype(b_)::value;
+            const TA* win = win0 + size_t(pb) * K::IH * K::IWB;  // dy plane c*MP + pb
             static_for<0, K::RH>([&](auto r_) {
                 constexpr int r = decltype(r_)::value;
                 float v[4 * K::NV];
@@ -262,11 +274,13 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     if constexpr (khn >= 0 && khn % K::D == 0 && khn / K::D < K::KH) {
                         constexpr int kh = khn / K::D;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
+                        for (int q = 0; q < K::NA; ++q)
 #pragma unroll
-                            for (int kw = 0; kw < K::KW; ++kw)
-                                acc[j][i] = fmaf(v[K::REM + i * K::S + kw * K::D], wr[m][kh][kw],
-                                                 acc[j][i]);
+                            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                                for (int kw = 0; kw < K::KW; ++kw)
+                                    acc[q][j][i] = fmaf(v[K::REM + i * K::S + kw * K::D],
+                                                        wr[K::REV ? pb : q][kh][kw], acc[q][j][i]);
                     }
                 });
             });
@@ -278,20 +292,24 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
         if (live) {
             const int wo0 = tx * K::TW + 4 * xi;
 #pragma unroll
-            for (int j = 0; j < K::THT; ++j) {
-                const int ho = K::ROWS ? ty : ty * K::TH + row0 + j;
-                if (ho >= a.Hout) continue;
-                TA* dst = static_cast<TA*>(a.out) + ((int64_t(n) * a.C + c) * a.Hout + ho) * a.Wout +
-                          wo0;
-                const float4 v = make_float4(finish(acc[j][0]), finish(acc[j][1]),
-                                             finish(acc[j][2]), finish(acc[j][3]));
-                if ((a.Wout & 3) == 0 && wo0 + 3 < a.Wout) {
-                    IO::store4(dst, v);
-                } else {
-                    if (wo0 < a.Wout) IO::store1(dst, v.x);
-                    if (wo0 + 1 < a.Wout) IO::store1(dst + 1, v.y);
-                    if (wo0 + 2 < a.Wout) IO::store1(dst + 2, v.z);
-                    if (wo0 + 3 < a.Wout) IO::store1(dst + 3, v.w);
+            for (int q = 0; q < K::NA; ++q) {
+                const int oc = c * K::NA + q;
+#pragma unroll
+                for (int j = 0; j < K::THT; ++j) {
+                    const int ho = K::ROWS ? ty : ty * K::TH + row0 + j;
+                    if (ho >= a.Hout) continue;
+                    TA* dst = static_cast<TA*>(a.out) +
+                              ((int64_t(n) * a.Cout + oc) * a.Hout + ho) * a.Wout + wo0;
+                    const float4 v = make_float4(finish(acc[q][j][0], q), finish(acc[q][j][1], q),
+                                                 finish(acc[q][j][2], q), finish(acc[q][j][3], q));
+                    if ((a.Wout & 3) == 0 && wo0 + 3 < a.Wout) {
+                        IO::store4(dst, v);
+                    } else {
+                        if (wo0 < a.Wout) IO::store1(dst, v.x);
+                        if (wo0 + 1 < a.Wout) IO::store1(dst + 1, v.y);
+                        if (wo0 + 2 < a.Wout) IO::store1(dst + 2, v.z);
+                        if (wo0 + 3 < a.Wout) IO::store1(dst + 3, v.w);
+                    }
                 }
             }
         }
@@ -310,11 +328,14 @@ dw_status_t launch(const Problem& p, const void* in, const void* w, const float*
     a.err = err;
     a.wtype = p.wtype;
     a.N = static_cast<int>(p.N);
-    // channel multiplier: the 2-D forward with one plane per tile, or the
-    // 2-D input gradient summing MB = M dy planes
-    if (K::REV ? p.M != K::MB : (p.M != 1 && (K::ROWS || K::PL != 1))) return DW_ERR_UNSUPPORTED;
-    a.M = K::REV ? 1 : static_cast<int>(p.M);
-    a.C = static_cast<int>(K::REV ? p.C : p.Co);
+    // channel multiplier: MP = M planes inside a tile (forward fan-out, or
+    // the input gradient's summed dy planes), or a forward with one output
+    // plane per tile (MP = 1, PL = 1)
+    if (K::MP > 1 ? p.M != K::MP : (p.M != 1 && (K::REV || K::ROWS || K::PL != 1)))
+        return DW_ERR_UNSUPPORTED;
+    a.M = K::MP > 1 ? 1 : static_cast<int>(p.M);
+    a.C = static_cast<int>((K::REV || K::MP > 1) ? p.C : p.Co);
+    a.Cout = static_cast<int>(K::REV ? p.C : p.Co);
     a.Hout = static_cast<int>(K::REV ? p.H : p.Ho);
     a.Wout = static_cast<int>(K::REV ? p.W : p.Wo);
     a.pt = pt_eff;
@@ -950,14 +971,14 @@ dw_status_t launch_chl_op(const Problem& p, Op op, const void* in, const void* w
 }
 
 template <int KH, int KW, bool REV, int THT, int WX, int WY, int NS, int MINB, class TA, int PL = 1,
-          int MB = 1>
+          int MP = 1>
 dw_status_t launch_rem(const Problem& p, const void* in, const void* w, const float* b,
                        void* out, cudaStream_t stream, int32_t* err, bool dry_run, int pt_eff,
                        int pl_eff) {
     int rem, sh4;
     box_shift<TA>(pl_eff, rem, sh4);
 #define DW_2D(R) \
-    return launch<Cfg<KH, KW, 1, REV, R, THT, WX, WY, NS, MINB, TA, 1, PL, MB>>(     \
+    return launch<Cfg<KH, KW, 1, REV, R, THT, WX, WY, NS, MINB, TA, 1, PL, MP>>(     \
         p, in, w, b, out, stream, err, dry_run, pt_eff, pl_eff, sh4);
     switch (rem) {
         case 0: DW_2D(0)
@@ -979,24 +1000,34 @@ dw_status_t launch_op(const Problem& p, Op op, const void* in, const void* w, co
                                                                    (KW - 1) - p.pl);
 }
 
-// Input gradient with channel multiplier MB (stride 1): one box holds the MB
-// dy planes of a dx plane, summed in the window loop.
-template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int MB>
-dw_status_t launch_mult_bwd(const Problem& p, const void* in, const void* w, void* out,
-                            cudaStream_t stream, int32_t* err, bool dry_run) {
-    return launch_rem<KH, KW, true, THT, WX, WY, NS, 1, TA, 1, MB>(
-        p, in, w, nullptr, out, stream, err, dry_run, (KH - 1) - p.pt, (KW - 1) - p.pl);
+// Channel multiplier MP inside a tile (stride 1): the forward computes the MP
+// output planes of one input plane, the input gradient sums the MP dy planes
+// of one dx plane (one box).  OPS: 1 = forward only, 2 = input gradient only,
+// 3 = both.
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int MP, int OPS = 3>
+dw_status_t launch_mult(const Problem& p, Op op, const void* in, const void* w, const float* b,
+                        void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (op == OP_FWD) {
+        if constexpr ((OPS & 1) != 0)
+            return launch_rem<KH, KW, false, THT, WX, WY, NS, 1, TA, 1, MP>(
+                p, in, w, b, out, stream, err, dry_run, p.pt, p.pl);
+        return DW_ERR_UNSUPPORTED;
+    }
+    if constexpr ((OPS & 2) != 0)
+        return launch_rem<KH, KW, true, THT, WX, WY, NS, 1, TA, 1, MP>(
+            p, in, w, nullptr, out, stream, err, dry_run, (KH - 1) - p.pt, (KW - 1) - p.pl);
+    return DW_ERR_UNSUPPORTED;
 }
 
 // Stride-2 forward (2-D kernel with S = 2): a tile is TH x 4*WX outputs, its
 // box the (TH-1)*2 + kH rows and (TW-1)*2 + kW columns they read.
-template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int PL = 1>
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int PL = 1, int MP = 1>
 dw_status_t launch_s2_fwd(const Problem& p, const void* in, const void* w, const float* b,
                           void* out, cudaStream_t stream, int32_t* err, bool dry_run) {
     int rem, sh4;
     box_shift<TA>(p.pl, rem, sh4);
 #define DW_S2(R) \
-    return launch<Cfg<KH, KW, 1, false, R, THT, WX, WY, NS, 1, TA, 2, PL>>(            \
+    return launch<Cfg<KH, KW, 1, false, R, THT, WX, WY, NS, 1, TA, 2, PL, MP>>(        \
         p, in, w, b, out, stream, err, dry_run, p.pt, p.pl, sh4);
     switch (rem) {
         case 0: DW_S2(0)
@@ -1018,6 +1049,8 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
             // small planes (at most 32 output columns): 4 planes of 32 x 32 outputs per tile
             if (p.Wo <= 32 && p.M == 1)
                 return launch_s2_fwd<3, 3, 4, 8, 32, 3, TA, 4>(p, in, w, b, out, stream, err, dry_run);
+            if (p.M == 2)  // both output planes of an input plane per tile
+                return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA, 1, 2>(p, in, w, b, out, stream, err, dry_run);
             return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA>(p, in, w, b, out, stream, err, dry_run);
         }
         if (op == OP_BWD_INPUT && p.kH == 3 && p.kW == 3) {
@@ -1028,13 +1061,17 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
         return DW_ERR_UNSUPPORTED;
     }
     if (p.sh != 1 || p.sw != 1) return DW_ERR_UNSUPPORTED;
-    if (p.M != 1 && op == OP_BWD_INPUT) {
-        //                                                            KH KW THT WX WY NS     MB
-        if (p.kH == 3 && p.kW == 3 && p.M == 2) return launch_mult_bwd<3, 3, 4, 32, 8, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
-        if (p.kH == 3 && p.kW == 3 && p.M == 4) return launch_mult_bwd<3, 3, 2, 32, 8, 4, TA, 4>(p, in, w, out, stream, err, dry_run);
-        if (p.kH == 5 && p.kW == 5 && p.M == 2) return launch_mult_bwd<5, 5, 4, 32, 8, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
-        if (p.kH == 7 && p.kW == 7 && p.M == 2) return launch_mult_bwd<7, 7, 4, 32, 4, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
-        return DW_ERR_UNSUPPORTED;
+    if (p.M != 1) {
+        // the input gradient's box of M dy planes (M = 4: half the rows per tile)
+        const bool fw = op == OP_FWD;
+        //                                                          KH KW THT WX WY NS     MP OPS
+        if (p.kH == 3 && p.kW == 3 && p.M == 2) return launch_mult<3, 3, 4, 32, 8, 4, TA, 2>(p, op, in, w, b, out, stream, err, dry_run);
+        if (p.kH == 3 && p.kW == 3 && p.M == 4 && fw) return launch_mult<3, 3, 4, 32, 8, 4, TA, 4, 1>(p, op, in, w, b, out, stream, err, dry_run);
+        if (p.kH == 3 && p.kW == 3 && p.M == 4) return launch_mult<3, 3, 2, 32, 8, 4, TA, 4, 2>(p, op, in, w, b, out, stream, err, dry_run);
+        if (p.kH == 5 && p.kW == 5 && p.M == 2) return launch_mult<5, 5, 4, 32, 8, 4, TA, 2>(p, op, in, w, b, out, stream, err, dry_run);
+        if (p.kH == 7 && p.kW == 7 && p.M == 2 && !fw) return launch_mult<7, 7, 4, 32, 4, 4, TA, 2, 2>(p, op, in, w, b, out, stream, err, dry_run);
+        if (op == OP_BWD_INPUT) return DW_ERR_UNSUPPORTED;
+        // other multipliers: one output plane per tile (below)
     }
     // small planes (at most 64 columns, the 3x3 and 5x5 filters): 2 planes of
     // 32 x 64 per tile instead of one plane in a 32 x 128 tile

@@ -1,7 +1,9 @@
 """GPU parity of the channel multiplier (C input channels, C*M outputs,
-output o reads input o // M) against the float64 oracle: forward (tiled NHWC
-kernels for M = 2 and 4 with 3x3 and 5x5 filters, the direct kernel
-otherwise), input gradient, weight and bias gradients and the fused epilogue.
+output o reads input o // M) against the float64 oracle: forward, input
+gradient, weight and bias gradients and the fused epilogue, on the tiled NHWC
+kernels (M = 2 and 4, 3x3 and 5x5 filters), the tiled NCHW kernels (one input
+plane feeding its M output planes, M dy planes summed into one dx plane, or
+one output plane per tile) and the direct kernels.
 Error rule as for the plain calls: |gpu - ref| <= 1e-5 * sum|terms|, exact
 where there is no term."""
 import numpy as np
@@ -168,7 +170,13 @@ NCHW_TILED = [
 ]
 
 
-@pytest.mark.parametrize("case", NCHW_TILED, ids=lambda c: c.name)
+@pytest.mark.parametrize("case", NCHW_TILED + [
+    Case("mnf4_3x3", 2, 21, 36, 5, 3, 3, padding=(0, 2, 3, 3), multiplier=4, layout="nchw",
+         seed=335),
+    Case("mnf2_5x5", 2, 35, 44, 3, 5, 5, multiplier=2, layout="nchw", seed=336),
+    Case("mnf2_3x3_many", 4, 64, 64, 8, 3, 3, multiplier=2, layout="nchw", seed=337),
+    Case("mnf2_s2_same", 2, 30, 72, 3, 3, 3, stride=2, multiplier=2, layout="nchw", seed=338),
+], ids=lambda c: c.name)
 def test_nchw_multiplier_tiles(case):
     inp = gu.inputs(case)
     x, w = inp["x"].cuda(), inp["w"].cuda()
