@@ -1224,9 +1224,9 @@ dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, f
 
 //                         KH KW  S  D THT TWT WX WY NS
 template <class TA> using W33s1 = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4, TA>;
-template <int M> using W33s1m = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4, float, M>;
-template <int M> using W33s2m = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4, float, M>;
-template <int M> using W55s1m = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3, float, M>;
+template <int M, class TA> using W33s1m = WCfg<3, 3, 1, 1, 2, 4, 4, 2, 4, TA, M>;
+template <int M, class TA> using W33s2m = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4, TA, M>;
+template <int M, class TA> using W55s1m = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3, TA, M>;
 template <class TA> using W33s2 = WCfg<3, 3, 2, 1, 2, 4, 4, 2, 4, TA>;
 template <class TA> using W55s1 = WCfg<5, 5, 1, 1, 2, 4, 4, 2, 3, TA>;
 template <class TA> using W77s1 = WCfg<7, 7, 1, 1, 1, 4, 4, 2, 3, TA>;
@@ -1250,12 +1250,12 @@ dw_status_t tiled_pick_nhwc(const Problem& p, const void* x, const void* dy, flo
     return DW_ERR_UNSUPPORTED;
 }
 
-// Channel multiplier (float32 NHWC, M = 2 or 4): 3x3, 3x3 stride 2, 5x5.
-template <int M>
+// Channel multiplier (NHWC, M = 2 or 4): 3x3, 3x3 stride 2, 5x5.
+template <int M, class TA>
 dw_status_t tiled_pick_mult(const Problem& p, const void* x, const void* dy, float* dw,
                             float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
     const int S = p.sh;
-#define DW_W(CFG) return launch_tiled<CFG<M>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+#define DW_W(CFG) return launch_tiled<CFG<M, TA>>(p, x, dy, dw, db, ws, stream, err, dry_run);
     if (p.kH == 3 && p.kW == 3 && S == 1) DW_W(W33s1m)
     if (p.kH == 3 && p.kW == 3 && S == 2) DW_W(W33s2m)
     if (p.kH == 5 && p.kW == 5 && S == 1) DW_W(W55s1m)
@@ -1272,15 +1272,22 @@ dw_status_t tiled_pick(const Problem& p, const void* x, const void* dy, float* d
                                db, ws, stream, err, dry_run);
     }
     if (p.M != 1) {
-        // channel multiplier: float32 NHWC tiles for M = 2, 4; else the direct kernels
-        if (p.layout != DW_NHWC || p.atype != DW_F32 || (p.M != 2 && p.M != 4)) return DW_ERR_UNSUPPORTED;
-        if (p.C % 4 != 0 || ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15))
+        // channel multiplier: NHWC tiles for M = 2, 4; else the direct kernels
+        if (p.layout != DW_NHWC || (p.M != 2 && p.M != 4)) return DW_ERR_UNSUPPORTED;
+        // TMA row strides: C elements a multiple of 16 bytes
+        if ((p.C * act_bytes(p.atype)) % 16 != 0 ||
+            ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15))
             return DW_ERR_UNSUPPORTED;
         if (p.sh != p.sw || p.dh != 1 || p.dw != 1) return DW_ERR_UNSUPPORTED;
         if (p.N >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX || p.Co >= INT_MAX)
             return DW_ERR_UNSUPPORTED;
-        return p.M == 2 ? tiled_pick_mult<2>(p, x, dy, dw, db, ws, stream, err, dry_run)
-                        : tiled_pick_mult<4>(p, x, dy, dw, db, ws, stream, err, dry_run);
+#define DW_M(TA)                                                                        \
+    return p.M == 2 ? tiled_pick_mult<2, TA>(p, x, dy, dw, db, ws, stream, err, dry_run) \
+                    : tiled_pick_mult<4, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (p.atype == DW_F16) DW_M(__half)
+        if (p.atype == DW_BF16) DW_M(__nv_bfloat16)
+        DW_M(float)
+#undef DW_M
     }
     if (p.layout == DW_NCHW) {
         if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;  // 16-bit NCHW: direct kernels

@@ -29,8 +29,8 @@ dw_status_t tiled_nhwc_launch(const Problem& p, Op op, const void* in, const voi
         return DW_ERR_UNSUPPORTED;
     const bool f = op == OP_FWD;
     if (p.M != 1) {
-        // channel multiplier: float32 tiles; the rest runs on the direct kernels
-        if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;
+        // channel multiplier tiles (any activation type); the rest runs on the
+        // direct kernels
         return f ? mult_launch(p, in, w, b, out, stream, err, dry_run)
                  : mult_bwd_launch(p, in, w, out, stream, err, dry_run);
     }

@@ -733,6 +733,14 @@ dw_status_t mult_launch(const Problem& p, const void* in, const void* w, const f
                         void* out, cudaStream_t stream, int32_t* err, bool dry_run);
 dw_status_t mult_bwd_launch(const Problem& p, const void* in, const void* w, void* out,
                             cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t mult_launch_f16(const Problem& p, const void* in, const void* w, const float* b,
+                          void* out, cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t mult_bwd_launch_f16(const Problem& p, const void* in, const void* w, void* out,
+                              cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t mult_launch_bf16(const Problem& p, const void* in, const void* w, const float* b,
+                          void* out, cudaStream_t stream, int32_t* err, bool dry_run);
+dw_status_t mult_bwd_launch_bf16(const Problem& p, const void* in, const void* w, void* out,
+                              cudaStream_t stream, int32_t* err, bool dry_run);
 
 }  // namespace nhwc
 }  // namespace dw

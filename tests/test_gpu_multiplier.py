@@ -228,3 +228,33 @@ def test_nchw_multiplier_half(case, name):
     if case in NCHW_BWD:
         assert dw.dwconv2d_query_algo(desc, 1, y.data_ptr(), wp, x.data_ptr()) == dw.DW_ALGO_TILED
     ha.run_case(case, name, "auto")
+
+
+# NHWC multiplier tiles with 16-bit activations (C a multiple of 8: rows of
+# 16 bytes): forward, input gradient, weight gradient
+HALF_TILED = [
+    Case("hm2_3x3", 2, 19, 37, 24, 3, 3, multiplier=2, seed=351),
+    Case("hm4_3x3", 2, 17, 40, 16, 3, 3, multiplier=4, seed=352),
+    Case("hm2_3x3_s2", 3, 29, 31, 40, 3, 3, stride=2, padding=1, multiplier=2, seed=353),
+    Case("hm4_3x3_s2_same", 2, 30, 33, 8, 3, 3, stride=2, multiplier=4, seed=354),
+    Case("hm2_5x5", 2, 23, 21, 32, 5, 5, multiplier=2, seed=355),
+]
+
+
+@pytest.mark.parametrize("name", ["f16", "bf16"])
+@pytest.mark.parametrize("case", HALF_TILED, ids=lambda c: c.name)
+def test_nhwc_multiplier_half_tiles(case, name):
+    from tests import test_gpu_half_activations as ha
+    dt, _ = ha.DTYPES[name]
+    inp = ha.inputs16(case, dt)
+    x, g = inp["x"].cuda(), inp["dy"].cuda()
+    y = torch.empty(case.out_shape(*gu.out_hw(case)), device="cuda", dtype=dt)
+    desc = gu.desc_of(case)
+    desc.atype = {"f16": dw.DW_F16, "bf16": dw.DW_BF16}[name]
+    wp = inp["w"].cuda().data_ptr()
+    assert dw.dwconv2d_query_algo(desc, 0, x.data_ptr(), wp, y.data_ptr()) == dw.DW_ALGO_TILED
+    if case.kH == 3 and (case.multiplier == 2 or case.stride == 1):
+        assert dw.dwconv2d_query_algo(desc, 1, y.data_ptr(), wp, x.data_ptr()) == dw.DW_ALGO_TILED
+    gw = torch.empty(case.multiplier * case.C, case.kH, case.kW, device="cuda")
+    assert dw.dwconv2d_query_algo(desc, 2, x.data_ptr(), g.data_ptr(), gw.data_ptr()) == dw.DW_ALGO_TILED
+    ha.run_case(case, name, "auto")
