@@ -361,11 +361,12 @@ def run_ours(args, rank, world, local_rank):
         for c in cases:
             for at in ("f16", "bf16"):
                 sh16 = Shape(c, dw, torch, device, 1, atype=at)
+                sh16.prepare_next_rows(dw, torch, device, act)
                 with torch.cuda.stream(stream):
-                    for op in ("fwd", "bwd"):
+                    for op in ("fwd", "bwd", "wgrad"):
                         sh16.call(dw, op, 0, sptr)
                 torch.cuda.synchronize()
-                for op in ("fwd", "bwd"):
+                for op in ("fwd", "bwd", "wgrad"):
                     k = time_kernel(torch, dw, sh16, op, l2, stream)
                     k["frac"] = k["gbs"] / peak
                     next_rows[f"{c.name}:{op}_{at}"] = k

@@ -642,13 +642,19 @@ struct NArgs {
     int32_t* err;
     int C, pt, pl;         // C: output channels (planes of dy); x plane of o is o / M
     int M;
+    int sh4;               // extra x-box shift beyond REM (0, or 4 for 16-bit elements)
     int tiles_x, tiles_y;  // tiles per plane
     int bands, band_rows;  // row bands per plane, tile rows per band
     int units;             // N * C * bands
 };
 
-template <int KH_, int KW_, int REM_, int THT_, int WY_, int NS_, int S_ = 1>
+template <int KH_, int KW_, int REM_, int THT_, int WY_, int NS_, int S_ = 1, class TA_ = float>
 struct NWCfg {
+    using TA = TA_;  // activation element type of x and dy
+    static constexpr int ESZ = sizeof(TA);
+    // x boxes start on 16-byte boundaries: REM = the start shift mod 4 (compile
+    // time), plus 0 or 4 more elements at run time for 16-bit elements
+    static constexpr int ALIGN = 16 / ESZ;
     static constexpr int KH = KH_, KW = KW_, REM = REM_, THT = THT_, WY = WY_, NS = NS_;
     // stride S (1 or 2): a lane owns OPL = 4 / S consecutive outputs, whose
     // input window starts 4 columns after its neighbour's in both cases
@@ -659,16 +665,16 @@ struct NWCfg {
     static constexpr int NT = NCT + 32;
     static constexpr int TW = 32 * OPL, TH = THT * WY;
     static constexpr int IH = (TH - 1) * S + KH;
-    static constexpr int IWB = (REM + (TW - 1) * S + KW + 3) / 4 * 4;
+    static constexpr int IWB = (REM + (ALIGN - 4) + (TW - 1) * S + KW + ALIGN - 1) / ALIGN * ALIGN;
     static constexpr int NV = (REM + (OPL - 1) * S + KW - 1) / 4 + 1;  // float4 per window row
     static_assert(S == 1 || S == 2, "stride 1 or 2");
-    static constexpr int XBYTES = IWB * IH * 4;
+    static constexpr int XBYTES = IWB * IH * ESZ;
     static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;
-    static constexpr int GBYTES = TW * TH * 4;
+    static constexpr int GBYTES = TW * TH * ESZ;
     static constexpr int STAGE_BYTES = XPITCH + GBYTES;
     static constexpr int RED_BYTES = NCW * T * 8;
     static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + RED_BYTES + size_t(2 * NS) * 8 + 16;
-    static_assert(GBYTES % 128 == 0, "TMA shared-memory alignment");
+    static_assert(GBYTES % 128 == 0 && (IWB * ESZ) % 16 == 0, "TMA shared-memory alignment");
     static_assert(IWB <= 256 && IH <= 256, "TMA box limit");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -728,7 +734,8 @@ __global__ void __launch_bounds__(K::NT, 1)
                         const int ty = ty0 + r;
                         unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
                         mbar_arrive_expect_tx(&full[s], K::XBYTES + K::GBYTES);
-                        tma_load_4d(st, &xmap, &full[s], tx * K::TW * K::S - a.pl - K::REM,
+                        tma_load_4d(st, &xmap, &full[s],
+                                    tx * K::TW * K::S - a.pl - K::REM - a.sh4,
                                     ty * K::TH * K::S - a.pt, c / a.M, n);
                         tma_load_4d(st + K::XPITCH, &gmap, &full[s], tx * K::TW, ty * K::TH, c, n);
                     }
@@ -763,19 +770,21 @@ __global__ void __launch_bounds__(K::NT, 1)
                 failed = true;
                 break;
             }
+            using TA = typename K::TA;
+            using IO = ActIO<TA>;
             const unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
-            const float4* xw =
-                reinterpret_cast<const float4*>(st) + row0 * K::S * (K::IWB / 4) + lane;
-            const float* gw = reinterpret_cast<const float*>(st + K::XPITCH) + row0 * K::TW +
-                              lane * K::OPL;
+            // lane window: 4-element vectors from column 4*lane (+ the run-time shift)
+            const TA* xw = reinterpret_cast<const TA*>(st) + row0 * K::S * K::IWB + 4 * lane + a.sh4;
+            const TA* gw = reinterpret_cast<const TA*>(st + K::XPITCH) + row0 * K::TW +
+                           lane * K::OPL;
             float g[K::THT][K::OPL];
 #pragma unroll
             for (int j = 0; j < K::THT; ++j) {
                 if constexpr (K::OPL == 4) {
-                    const float4 f = *reinterpret_cast<const float4*>(gw + j * K::TW);
+                    const float4 f = IO::load4(gw + j * K::TW);
                     g[j][0] = f.x; g[j][1] = f.y; g[j][2] = f.z; g[j][3] = f.w;
                 } else {
-                    const float2 f = *reinterpret_cast<const float2*>(gw + j * K::TW);
+                    const float2 f = IO::load2(gw + j * K::TW);
                     g[j][0] = f.x; g[j][1] = f.y;
                 }
             }
@@ -789,7 +798,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                 float v[4 * K::NV];
 #pragma unroll
                 for (int q = 0; q < K::NV; ++q) {
-                    const float4 f = xw[r * (K::IWB / 4) + q];
+                    const float4 f = IO::load4(xw + r * K::IWB + 4 * q);
                     v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
                 }
                 static_for<0, K::THT>([&](auto j_) {
@@ -1122,7 +1131,7 @@ size_t tiled_nchw_workspace(const Problem& p) {
 }
 
 template <class K>
-dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy, float* dw,
+dw_status_t launch_tiled_nchw(const Problem& p, const void* x, const void* dy, float* dw,
                               float* db, void* ws, cudaStream_t stream, int32_t* err,
                               bool dry_run) {
     NArgs a;
@@ -1132,6 +1141,7 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     a.M = int(p.M);
     a.pt = p.pt;
     a.pl = p.pl;
+    a.sh4 = ((-p.pl) % K::ALIGN + K::ALIGN) % K::ALIGN - K::REM;  // 0 or 4
     const int64_t ty = (p.Ho + K::TH - 1) / K::TH, tx = (p.Wo + K::TW - 1) / K::TW;
     if (ty >= INT_MAX || tx >= INT_MAX) return DW_ERR_UNSUPPORTED;
     a.tiles_x = int(tx);
@@ -1158,18 +1168,18 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     if (G > units) G = units;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMap xmap, gmap;
+    constexpr cuuint64_t E = K::ESZ;
     const cuuint64_t xd[4] = {cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.C), cuuint64_t(p.N)};
-    const cuuint64_t xs[3] = {cuuint64_t(p.W) * 4, cuuint64_t(p.W * p.H) * 4,
-                              cuuint64_t(p.W * p.H * p.C) * 4};
+    const cuuint64_t xs[3] = {cuuint64_t(p.W) * E, cuuint64_t(p.W * p.H) * E,
+                              cuuint64_t(p.W * p.H * p.C) * E};
     const cuuint32_t xbox[4] = {K::IWB, K::IH, 1, 1};
     const cuuint64_t gd[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.Co), cuuint64_t(p.N)};
-    const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * 4, cuuint64_t(p.Wo * p.Ho) * 4,
-                              cuuint64_t(p.Wo * p.Ho * p.Co) * 4};
+    const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * E, cuuint64_t(p.Wo * p.Ho) * E,
+                              cuuint64_t(p.Wo * p.Ho * p.Co) * E};
     const cuuint32_t gbox[4] = {K::TW, K::TH, 1, 1};
-    if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
-                          xbox, estr) != CUDA_SUCCESS ||
-        encode_tensor_map(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(dy), gd, gs,
-                          gbox, estr) != CUDA_SUCCESS)
+    constexpr CUtensorMapDataType dt = ActIO<typename K::TA>::kTma;
+    if (encode_tensor_map(&xmap, dt, 4, const_cast<void*>(x), xd, xs, xbox, estr) != CUDA_SUCCESS ||
+        encode_tensor_map(&gmap, dt, 4, const_cast<void*>(dy), gd, gs, gbox, estr) != CUDA_SUCCESS)
         return DW_ERR_CUDA;
     if (launch_pdl(partial_tiled_nchw<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap,
                    gmap, a) != cudaSuccess)
@@ -1182,44 +1192,61 @@ dw_status_t launch_tiled_nchw(const Problem& p, const float* x, const float* dy,
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
-template <int KH, int KW, int THT, int WY, int NS, int S = 1>
-dw_status_t launch_nchw_rem(const Problem& p, const float* x, const float* dy, float* dw,
+template <int KH, int KW, int THT, int WY, int NS, int S, class TA>
+dw_status_t launch_nchw_rem(const Problem& p, const void* x, const void* dy, float* dw,
                             float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+#define DW_N(R) return launch_tiled_nchw<NWCfg<KH, KW, R, THT, WY, NS, S, TA>>(p, x, dy, dw, db, ws, stream, err, dry_run);
     switch (((-p.pl) % 4 + 4) % 4) {
-        case 0: return launch_tiled_nchw<NWCfg<KH, KW, 0, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        case 1: return launch_tiled_nchw<NWCfg<KH, KW, 1, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        case 2: return launch_tiled_nchw<NWCfg<KH, KW, 2, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        default: return launch_tiled_nchw<NWCfg<KH, KW, 3, THT, WY, NS, S>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 0: DW_N(0)
+        case 1: DW_N(1)
+        case 2: DW_N(2)
+        default: DW_N(3)
     }
+#undef DW_N
 }
 
-dw_status_t tiled_pick_nchw(const Problem& p, const float* x, const float* dy, float* dw,
+template <class TA>
+dw_status_t tiled_pick_nchw_2d(const Problem& p, const void* x, const void* dy, float* dw,
+                               float* db, void* ws, cudaStream_t stream, int32_t* err,
+                               bool dry_run) {
+    if (p.sh == 2) {
+        //                                                          KH KW THT WY NS S
+        if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3, 2, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        return DW_ERR_UNSUPPORTED;
+    }
+    //                                                          KH KW THT WY NS S
+    if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3, 1, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 5 && p.kW == 5) return launch_nchw_rem<5, 5, 4, 8, 3, 1, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kH == 7 && p.kW == 7) return launch_nchw_rem<7, 7, 2, 8, 3, 1, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
+}
+
+dw_status_t tiled_pick_nchw(const Problem& p, const void* x, const void* dy, float* dw,
                             float* db, void* ws, cudaStream_t stream, int32_t* err,
                             bool dry_run) {
     if (p.layout != DW_NCHW) return DW_ERR_UNSUPPORTED;
     if (p.dh != 1 || p.dw != 1 || p.sh != p.sw || p.sh > 2) return DW_ERR_UNSUPPORTED;
-    if (p.W % 4 != 0 || p.Wo % 4 != 0) return DW_ERR_UNSUPPORTED;  // TMA row pitches
+    const int esz = act_bytes(p.atype);
+    if ((p.W * esz) % 16 != 0 || (p.Wo * esz) % 16 != 0) return DW_ERR_UNSUPPORTED;  // TMA row pitches
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
         return DW_ERR_UNSUPPORTED;
     if (p.N >= INT_MAX || p.C >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX) return DW_ERR_UNSUPPORTED;
-    if (p.sh == 2) {
-        //                                                        KH KW THT WY NS S
-        if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3, 2>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        return DW_ERR_UNSUPPORTED;
-    }
     if (p.kH == 1) {
-        if (p.kW == 3) return launch_rows_rem<3, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 5) return launch_rows_rem<5, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 7) return launch_rows_rem<7, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 15) return launch_rows_rem<15, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 31) return launch_rows_rem<31, 8>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        // rows of 1 x kW filters: float32 activations
+        if (p.sh != 1 || p.atype != DW_F32) return DW_ERR_UNSUPPORTED;
+        const float* xf = static_cast<const float*>(x);
+        const float* gf = static_cast<const float*>(dy);
+        if (p.kW == 3) return launch_rows_rem<3, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 5) return launch_rows_rem<5, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 7) return launch_rows_rem<7, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 15) return launch_rows_rem<15, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
+        if (p.kW == 31) return launch_rows_rem<31, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
         return DW_ERR_UNSUPPORTED;
     }
-    //                                                    KH KW THT WY NS
-    if (p.kH == 3 && p.kW == 3) return launch_nchw_rem<3, 3, 4, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 5 && p.kW == 5) return launch_nchw_rem<5, 5, 4, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    if (p.kH == 7 && p.kW == 7) return launch_nchw_rem<7, 7, 2, 8, 3>(p, x, dy, dw, db, ws, stream, err, dry_run);
-    return DW_ERR_UNSUPPORTED;
+    if (p.atype == DW_F16) return tiled_pick_nchw_2d<__half>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.atype == DW_BF16)
+        return tiled_pick_nchw_2d<__nv_bfloat16>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    return tiled_pick_nchw_2d<float>(p, x, dy, dw, db, ws, stream, err, dry_run);
 }
 
 //                         KH KW  S  D THT TWT WX WY NS
@@ -1266,10 +1293,9 @@ dw_status_t tiled_pick_mult(const Problem& p, const void* x, const void* dy, flo
 dw_status_t tiled_pick(const Problem& p, const void* x, const void* dy, float* dw, float* db,
                        void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
     if (p.M != 1 && p.layout == DW_NCHW) {
-        // channel multiplier, NCHW: the plane-per-unit tiles (2-D filters, float32)
-        if (p.atype != DW_F32 || p.kH == 1) return DW_ERR_UNSUPPORTED;
-        return tiled_pick_nchw(p, static_cast<const float*>(x), static_cast<const float*>(dy), dw,
-                               db, ws, stream, err, dry_run);
+        // channel multiplier, NCHW: the plane-per-unit tiles (2-D filters)
+        if (p.kH == 1) return DW_ERR_UNSUPPORTED;
+        return tiled_pick_nchw(p, x, dy, dw, db, ws, stream, err, dry_run);
     }
     if (p.M != 1) {
         // channel multiplier: NHWC tiles for M = 2, 4; else the direct kernels
@@ -1289,11 +1315,7 @@ dw_status_t tiled_pick(const Problem& p, const void* x, const void* dy, float* d
         DW_M(float)
 #undef DW_M
     }
-    if (p.layout == DW_NCHW) {
-        if (p.atype != DW_F32) return DW_ERR_UNSUPPORTED;  // 16-bit NCHW: direct kernels
-        return tiled_pick_nchw(p, static_cast<const float*>(x), static_cast<const float*>(dy), dw,
-                               db, ws, stream, err, dry_run);
-    }
+    if (p.layout == DW_NCHW) return tiled_pick_nchw(p, x, dy, dw, db, ws, stream, err, dry_run);
     if (p.layout != DW_NHWC) return DW_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 15)
         return DW_ERR_UNSUPPORTED;

@@ -161,3 +161,51 @@ def test_no_bias_gradient_and_small_workspace_error():
     with pytest.raises(ValueError):
         dw.dwconv2d_bwd_weight(inp["x"].cuda(), inp["dy"].cuda(), (3, 3),
                                workspace=torch.empty(8, dtype=torch.uint8, device="cuda"))
+
+
+# NCHW tiled weight gradient with 16-bit activations: every column phase of
+# the 16-byte x box (REM 0..3 and the extra 4-element shift), stride 2, 5x5,
+# 7x7 and a multiplier; float32 results, the same bits as the float32 call on
+# the widened tensors (same kernel family, same summation order)
+HALF_NCHW = [
+    Case("wh_3x3_same", 2, 37, 48, 6, 3, 3, layout="nchw", seed=91),
+    Case("wh_3x3_pl0", 2, 29, 40, 5, 3, 3, padding=(0, 1, 0, 2), layout="nchw", seed=92),
+    Case("wh_3x3_pl2", 1, 31, 40, 4, 3, 3, padding=(2, 0, 2, 0), layout="nchw", seed=93),
+    Case("wh_3x3_pl3", 1, 26, 40, 6, 3, 3, padding=(1, 3, 3, 7), layout="nchw", seed=94),
+    Case("wh_3x3_pl5", 1, 21, 40, 5, 3, 3, padding=(1, 1, 5, 5), layout="nchw", seed=95),
+    Case("wh_3x3_pl4", 1, 17, 40, 3, 3, 3, padding=(1, 1, 4, 6), layout="nchw", seed=100),
+    Case("wh_3x3_pl6", 1, 17, 40, 3, 3, 3, padding=(1, 1, 6, 4), layout="nchw", seed=101),
+    Case("wh_3x3_pl7", 1, 17, 40, 3, 3, 3, padding=(1, 1, 7, 3), layout="nchw", seed=102),
+    Case("wh_3x3_s2", 3, 29, 80, 4, 3, 3, stride=2, padding=1, layout="nchw", seed=96),
+    Case("wh_5x5", 2, 35, 48, 5, 5, 5, layout="nchw", seed=97),
+    Case("wh_7x7", 2, 33, 32, 4, 7, 7, layout="nchw", seed=98),
+    Case("wh_m2_3x3", 2, 21, 40, 3, 3, 3, multiplier=2, layout="nchw", seed=99),
+]
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("case", HALF_NCHW, ids=lambda c: c.name)
+def test_nchw_tiled_half_weight_gradient(case, dt):
+    inp = gu.inputs(case)
+    x16, g16 = inp["x"].to(dt), inp["dy"].to(dt)
+    x32, g32 = x16.float(), g16.float()
+    p = gu.problem(case)
+    xd, gd = gu.f64(x32), gu.f64(g32)
+    dwr, dbr = oracle.bwd_weight(p, xd, gd)
+    dws, dbs = oracle.bwd_weight(p, np.abs(xd), np.abs(gd))
+    desc = gu.desc_of(case)
+    desc.atype = dw.DW_F16 if dt == torch.float16 else dw.DW_BF16
+    gw = torch.empty(case.multiplier * case.C, case.kH, case.kW, device="cuda")
+    xc, gc = x16.cuda(), g16.cuda()
+    assert dw.dwconv2d_query_algo(desc, 2, xc.data_ptr(), gc.data_ptr(), gw.data_ptr()) == \
+        dw.DW_ALGO_TILED
+    kw = dict(stride=case.stride, dilation=case.dilation, padding=case.padding,
+              layout=case.layout)
+    a_w, a_b = dw.dwconv2d_bwd_weight(xc, gc, (case.kH, case.kW), **kw)
+    b_w, b_b = dw.dwconv2d_bwd_weight(x32.cuda(), g32.cuda(), (case.kH, case.kW), **kw)
+    d_w, d_b = dw.dwconv2d_bwd_weight(xc, gc, (case.kH, case.kW), algo="direct", **kw)
+    torch.cuda.synchronize()
+    gu.assert_close(a_w.cpu().numpy(), dwr, dws, f"{case.name} dW")
+    gu.assert_close(a_b.cpu().numpy(), dbr, dbs, f"{case.name} db")
+    gu.assert_close(d_w.cpu().numpy(), dwr, dws, f"{case.name} dW direct")
+    assert torch.equal(a_w, b_w) and torch.equal(a_b, b_b)
