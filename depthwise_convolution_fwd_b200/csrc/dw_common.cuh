@@ -350,7 +350,7 @@ __device__ __forceinline__ void store4(float* p, const float4& v) {
 
 // Activation element types: float32, float16, bfloat16.  Loads widen to
 // float32 exactly; stores round to nearest even.  load4/store4 move 4
-// consecutive elements (16 or 8 bytes, aligned to that size).
+// consecutive elements (16 or 8 bytes, aligned to that size), load2/store2 two.
 template <class TA>
 struct ActIO;
 
@@ -365,6 +365,9 @@ struct ActIO<float> {
         return *reinterpret_cast<const float4*>(p);
     }
     static __device__ __forceinline__ void store1(float* p, float v) { *p = v; }
+    static __device__ __forceinline__ void store2(float* p, const float2& v) {
+        *reinterpret_cast<float2*>(p) = v;
+    }
     static __device__ __forceinline__ void store4(float* p, const float4& v) { dw::store4(p, v); }
 };
 
@@ -382,6 +385,9 @@ struct ActIO<__half> {
         return make_float4(a.x, a.y, b.x, b.y);
     }
     static __device__ __forceinline__ void store1(__half* p, float v) { *p = __float2half_rn(v); }
+    static __device__ __forceinline__ void store2(__half* p, const float2& v) {
+        *reinterpret_cast<__half2*>(p) = __floats2half2_rn(v.x, v.y);
+    }
     static __device__ __forceinline__ void store4(__half* p, const float4& v) {
         const __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
         uint2 raw;
@@ -408,6 +414,9 @@ struct ActIO<__nv_bfloat16> {
     }
     static __device__ __forceinline__ void store1(__nv_bfloat16* p, float v) {
         *p = __float2bfloat16_rn(v);
+    }
+    static __device__ __forceinline__ void store2(__nv_bfloat16* p, const float2& v) {
+        *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
     }
     static __device__ __forceinline__ void store4(__nv_bfloat16* p, const float4& v) {
         const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);

@@ -84,6 +84,18 @@ struct VecOps<4> {
     }
 };
 
+// two channels per lane: only the transposed multiplier-2 tiles (TR1 mode)
+template <>
+struct VecOps<2> {
+    using T = float2;
+    static __device__ __forceinline__ T zero() { return make_float2(0.f, 0.f); }
+    template <class TA>
+    static __device__ __forceinline__ void store(TA* p, const T& v) { ActIO<TA>::store2(p, v); }
+    static __device__ __forceinline__ T load_b(const float* b, int c) {
+        return make_float2(__ldg(b + c), __ldg(b + c + 1));
+    }
+};
+
 template <>
 struct VecOps<1> {
     using T = float;
@@ -144,7 +156,11 @@ struct Cfg {
     static constexpr int MULT = MULT_;
     static constexpr bool TR0 = TR_;
     static constexpr int SC = TR0 ? CB * MULT : CB / MULT;  // staged channels per pixel
-    static constexpr int MT = TR0 ? MULT : 1;
+    // transposed multiplier with VEC * MULT = 4 (one dx channel per lane for
+    // M = 4, two for M = 2): the lane's 4 dy channels are one float4, against
+    // one float4 of filters
+    static constexpr bool TR1 = TR0 && VEC_ < 4 && VEC_ * MULT == 4;
+    static constexpr int MT = TR0 && !TR1 ? MULT : 1;
     static constexpr int KH = KH_, KW = KW_, S = S_, D = D_;
     static constexpr bool TR = TR_;
     static constexpr int THT = THT_, TWT = TWT_, WX = WX_, WY = WY_, NS = NS_;
@@ -177,7 +193,7 @@ struct Cfg {
     static_assert(MULT > 1 || ESZ < 4 || STAGE_BYTES % 128 == 0, "TMA shared-memory alignment");
     static_assert(NO == 0 || OUT_BYTES % 128 == 0, "staging buffers on 128-byte boundaries");
     static_assert((SC * ESZ) % 16 == 0 && SC <= 256, "16-byte rows in the input box");
-    static_assert(MULT == 1 || (VEC == 4 && (TR || CB % MULT == 0)),
+    static_assert(MULT == 1 || TR1 || (VEC == 4 && (TR || CB % MULT == 0)),
                   "multiplier tiles: 4-channel lanes");
     static_assert(!TR || (THT % S == 0 && TWT % S == 0), "transposed blocks are phase aligned");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -322,14 +338,21 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
     const int j0 = yi * K::THT, i0 = xi * K::TWT;
     const int64_t row_pitch = int64_t(a.Wout) * a.C;
 
-    V wr[K::KH][K::KW][K::MT];
+    // filters and accumulators: float4 in the TR1 mode (4 dy channels per lane)
+    using VOA = VecOps<K::TR1 ? 4 : K::VEC>;
+    using VA = typename VOA::T;
+    VA wr[K::KH][K::KW][K::MT];
     V bias = VO::zero();
     int cur_cb = -1;
     // the value stored for one output: acc (+ bias) (-> activation); with a
     // multiplier in transposed mode, dx channel c + e sums the MULT
     // consecutive products of output channels (c + e) * MULT ..
-    auto finish = [&](const V (&acc)[K::MT]) -> V {
-        if constexpr (K::TR && K::MT == 2) {
+    auto finish = [&](const VA (&acc)[K::MT]) -> V {
+        if constexpr (K::TR1 && K::VEC == 1) {
+            return (acc[0].x + acc[0].y) + (acc[0].z + acc[0].w);
+        } else if constexpr (K::TR1) {
+            return make_float2(acc[0].x + acc[0].y, acc[0].z + acc[0].w);
+        } else if constexpr (K::TR && K::MT == 2) {
             return make_float4(acc[0].x + acc[0].y, acc[0].z + acc[0].w, acc[1].x + acc[1].y,
                                acc[1].z + acc[1].w);
         } else if constexpr (K::TR && K::MT == 4) {
@@ -358,6 +381,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
             constexpr int step = K::KH * K::KW;
             // filter rows: channel c (forward: the output channel), or in
             // transposed mode with a multiplier output channels c*MULT + 4m..
+            // (TR1: the 4 output channels c*4 .. c*4+3)
             const int64_t o = int64_t(live ? c : 0) * (K::TR ? K::MULT : 1) * step;
             // one branch on the weight type, then straight loads
             if (a.wtype == DW_F16) {
@@ -368,7 +392,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
                         for (int kw = 0; kw < K::KW; ++kw)
-                            wr[kh][kw][m] = VO::load_w(wp, o + 4 * m * step + kh * K::KW + kw, step);
+                            wr[kh][kw][m] = VOA::load_w(wp, o + 4 * m * step + kh * K::KW + kw, step);
             } else {
                 const float* wp = static_cast<const float*>(a.w);
 #pragma unroll
@@ -377,7 +401,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
                         for (int kw = 0; kw < K::KW; ++kw)
-                            wr[kh][kw][m] = VO::load_w(wp, o + 4 * m * step + kh * K::KW + kw, step);
+                            wr[kh][kw][m] = VOA::load_w(wp, o + 4 * m * step + kh * K::KW + kw, step);
             }
             if (!live) {
 #pragma unroll
@@ -385,7 +409,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
 #pragma unroll
                     for (int kh = 0; kh < K::KH; ++kh)
 #pragma unroll
-                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw][m] = VO::zero();
+                        for (int kw = 0; kw < K::KW; ++kw) wr[kh][kw][m] = VOA::zero();
             }
             if (!K::TR && a.b != nullptr && live) bias = VO::load_b(a.b, c);
             if constexpr (EPI != kNoEpilogue) {
@@ -416,13 +440,13 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
         // consumer barrier below, so every consumer leaves together; the
         // shared-memory reads in between stay inside the stage)
 
-        V acc[K::THT][K::TWT][K::MT];
+        VA acc[K::THT][K::TWT][K::MT];
 #pragma unroll
         for (int j = 0; j < K::THT; ++j)
 #pragma unroll
             for (int i = 0; i < K::TWT; ++i)
 #pragma unroll
-                for (int m = 0; m < K::MT; ++m) acc[j][i][m] = VO::zero();
+                for (int m = 0; m < K::MT; ++m) acc[j][i][m] = VOA::zero();
 
         // this thread's window: cell (r, q) holds SC staged channels.  The
         // lane's 4 channels cv*4.. read, in the forward, input channels
@@ -443,8 +467,10 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                     return false;
                 }();
                 if constexpr (used) {
-                    V v[K::MT];
-                    if constexpr (K::MT == 1) {
+                    VA v[K::MT];
+                    if constexpr (K::TR1) {
+                        v[0] = ActIO<TA>::load4(win + (r * K::IW + q) * K::SC);
+                    } else if constexpr (K::MT == 1) {
                         v[0] = load_cell<K>(win + (r * K::IW + q) * K::SC);
                     } else {
 #pragma unroll
@@ -461,7 +487,7 @@ __global__ void __launch_bounds__(K::NT, K::MINB)
                                 if constexpr (kw >= 0) {
 #pragma unroll
                                     for (int m = 0; m < K::MT; ++m)
-                                        VO::fma(acc[j][i][m], v[m], wr[kh][kw][m]);
+                                        VOA::fma(acc[j][i][m], v[m], wr[kh][kw][m]);
                                 }
                             });
                         }

@@ -4,11 +4,11 @@
 // channels they read; each lane's 4 output channels take their input values
 // from one (M >= 4) or two (M = 2) input channels of the staged window (the
 // kernel in dw_tiled_nhwc.cuh).  Input gradient (transposed mode): a tile
-// holds 32 dx channels and stages their 32*M dy channels; a lane keeps M
-// float4 accumulators per output (dy channels c*M .. c*M + 4M-1 against
-// their filters) and sums each dx channel's M products at the store.  Other
-// multipliers and shapes use the direct kernels.  Activations are float32,
-// float16 or bfloat16 (one instantiation unit per type).
+// holds 32 dx channels and stages their 32*M dy channels; a lane owns 4/M
+// dx channels, whose 4 dy channels form one float4 (conflict-free 16-byte
+// shared loads), and sums each dx channel's M products at the store.
+// Other multipliers and shapes use the direct kernels.  Activations are
+// float32, float16 or bfloat16 (one instantiation unit per type).
 #pragma once
 
 #include "dw_tiled_nhwc.cuh"
@@ -24,10 +24,12 @@ using M33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4, 4, 0, 2, 32, M, TA>;
 template <int M, class TA>
 using M55s1 = Cfg<5, 5, 1, 1, false, 2, 4, 8, 4, 2, 4, 2, 1, 32, M, TA>;
 
-// transposed mode: fewer outputs per thread (M float4 filters per tap)
-template <class TA> using MB33s1m2 = Cfg<3, 3, 1, 1, true, 2, 2, 8, 4, 4, 4, 2, 1, 32, 2, TA>;
-template <class TA> using MB33s1m4 = Cfg<3, 3, 1, 1, true, 1, 2, 8, 4, 3, 4, 2, 1, 32, 4, TA>;
-template <class TA> using MB33s2m2 = Cfg<3, 3, 2, 1, true, 2, 2, 8, 4, 4, 4, 0, 1, 32, 2, TA>;
+// transposed mode: a lane owns 4 / M dx channels (VEC = 2 for M = 2, 1 for
+// M = 4), their 4 dy channels one float4 against one float4 of filters per tap
+template <class TA> using MB33s1m2 = Cfg<3, 3, 1, 1, true, 2, 4, 4, 4, 3, 2, 2, 1, 32, 2, TA>;
+template <class TA> using MB33s2m2 = Cfg<3, 3, 2, 1, true, 2, 4, 4, 4, 4, 2, 0, 1, 32, 2, TA>;
+template <class TA> using MB33s1m4 = Cfg<3, 3, 1, 1, true, 2, 4, 2, 4, 3, 1, 2, 1, 32, 4, TA>;
+template <class TA> using MB33s2m4 = Cfg<3, 3, 2, 1, true, 2, 4, 2, 4, 4, 1, 0, 1, 32, 4, TA>;
 
 template <class TA>
 dw_status_t mult_bwd_launch_t(const Problem& p, const void* in, const void* w, void* out,
@@ -40,6 +42,8 @@ dw_status_t mult_bwd_launch_t(const Problem& p, const void* in, const void* w, v
         return launch<MB33s1m4<TA>>(p, op, in, w, nullptr, out, stream, err, dry_run);
     if (p.sh == 2 && p.M == 2)
         return launch<MB33s2m2<TA>>(p, op, in, w, nullptr, out, stream, err, dry_run);
+    if (p.sh == 2 && p.M == 4)
+        return launch<MB33s2m4<TA>>(p, op, in, w, nullptr, out, stream, err, dry_run);
     return DW_ERR_UNSUPPORTED;
 }
 

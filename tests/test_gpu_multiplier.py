@@ -148,8 +148,7 @@ def test_full_size_sampled(case):
                     f"{case.name} bwd sampled")
 
 
-@pytest.mark.parametrize("case", [c for c in TILED if c.kH == 3 and (c.multiplier == 2 or c.stride == 1)],
-                         ids=lambda c: c.name)
+@pytest.mark.parametrize("case", [c for c in TILED if c.kH == 3], ids=lambda c: c.name)
 def test_tiled_multiplier_input_gradient(case):
     inp = gu.inputs(case)
     dy, w = inp["dy"].cuda(), inp["w"].cuda()
@@ -253,7 +252,7 @@ def test_nhwc_multiplier_half_tiles(case, name):
     desc.atype = {"f16": dw.DW_F16, "bf16": dw.DW_BF16}[name]
     wp = inp["w"].cuda().data_ptr()
     assert dw.dwconv2d_query_algo(desc, 0, x.data_ptr(), wp, y.data_ptr()) == dw.DW_ALGO_TILED
-    if case.kH == 3 and (case.multiplier == 2 or case.stride == 1):
+    if case.kH == 3:
         assert dw.dwconv2d_query_algo(desc, 1, y.data_ptr(), wp, x.data_ptr()) == dw.DW_ALGO_TILED
     gw = torch.empty(case.multiplier * case.C, case.kH, case.kW, device="cuda")
     assert dw.dwconv2d_query_algo(desc, 2, x.data_ptr(), g.data_ptr(), gw.data_ptr()) == dw.DW_ALGO_TILED
