@@ -18,6 +18,7 @@ import os
 import shutil
 import subprocess
 import sys
+import time
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -61,6 +62,9 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)]
     if not force and not _stale(LIB, _deps()):
         return LIB
+    # outputs carry the time their build started, so a source edited while
+    # the build runs is still newer than them
+    started = time.time()
     os.makedirs(BUILD_DIR, exist_ok=True)
     exe = nvcc()
     flags = NVCC_FLAGS + list(extra_flags or [])
@@ -75,7 +79,10 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         cmd = [exe, "-c", src, "-o", obj] + flags
         if verbose:
             cmd += ["-Xptxas", "-v"]
+        t0 = time.time()
         r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode == 0:
+            os.utime(obj, (t0, t0))
         return src, r
 
     workers = max(1, min(len(jobs), os.cpu_count() or 1))
@@ -96,6 +103,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link of libdwconv2d.so failed")
     os.replace(tmp, LIB)
+    os.utime(LIB, (started, started))
     return LIB
 
 

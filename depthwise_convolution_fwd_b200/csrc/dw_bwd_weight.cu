@@ -883,24 +883,28 @@ struct RArgs {
     double* part;
     int32_t* err;
     int N, C, Ho, pt, pl;
+    int sh4;       // extra x-box shift beyond REM (0, or 4 for 16-bit elements)
     int tiles_x;   // 128-column strips per row
     int cgroups;   // groups of 8 channels
     int nper;      // n per block
     int units;     // n blocks * cgroups
 };
 
-template <int KW_, int REM_, int NS_>
+template <int KW_, int REM_, int NS_, class TA_ = float>
 struct RCfg {
+    using TA = TA_;  // activation element type of x and dy
+    static constexpr int ESZ = sizeof(TA);
+    static constexpr int ALIGN = 16 / ESZ;  // x boxes start on 16-byte columns
     static constexpr int KW = KW_, REM = REM_, NS = NS_;
     static constexpr int T = KW + 1;
     static constexpr int NCW = 8;  // consumer warps = channels per unit
     static constexpr int NT = NCW * 32 + 32;
     static constexpr int TW = 128;
-    static constexpr int IWB = (REM + TW + KW - 1 + 3) / 4 * 4;
-    static constexpr int NV = (REM + 3 + KW - 1) / 4 + 1;  // float4 per window
-    static constexpr int XBYTES = IWB * NCW * 4;
+    static constexpr int IWB = (REM + (ALIGN - 4) + TW + KW - 1 + ALIGN - 1) / ALIGN * ALIGN;
+    static constexpr int NV = (REM + 3 + KW - 1) / 4 + 1;  // 4-vectors per window
+    static constexpr int XBYTES = IWB * NCW * ESZ;
     static constexpr int XPITCH = (XBYTES + 127) / 128 * 128;
-    static constexpr int GBYTES = TW * NCW * 4;
+    static constexpr int GBYTES = TW * NCW * ESZ;
     static constexpr int STAGE_BYTES = XPITCH + GBYTES;
     static constexpr size_t SMEM = size_t(NS) * STAGE_BYTES + size_t(2 * NS) * 8 + 16;
     static_assert(GBYTES % 128 == 0, "TMA shared-memory alignment");
@@ -954,8 +958,8 @@ __global__ void __launch_bounds__(K::NT, 1)
                             }
                             unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
                             mbar_arrive_expect_tx(&full[s], K::XBYTES + K::GBYTES);
-                            tma_load_4d(st, &xmap, &full[s], tx * K::TW - a.pl - K::REM, h - a.pt,
-                                        cg * K::NCW, n);
+                            tma_load_4d(st, &xmap, &full[s], tx * K::TW - a.pl - K::REM - a.sh4,
+                                        h - a.pt, cg * K::NCW, n);
                             tma_load_4d(st + K::XPITCH, &gmap, &full[s], tx * K::TW, h,
                                         cg * K::NCW, n);
                         }
@@ -991,15 +995,17 @@ __global__ void __launch_bounds__(K::NT, 1)
                 failed = true;
                 break;
             }
+            using IO = ActIO<typename K::TA>;
             const unsigned char* st = smem + size_t(s) * K::STAGE_BYTES;
-            const float4* xw = reinterpret_cast<const float4*>(st) + warp * (K::IWB / 4) + lane;
-            const float4 gf =
-                reinterpret_cast<const float4*>(st + K::XPITCH)[warp * (K::TW / 4) + lane];
+            const typename K::TA* xw =
+                reinterpret_cast<const typename K::TA*>(st) + warp * K::IWB + 4 * lane + a.sh4;
+            const float4 gf = IO::load4(reinterpret_cast<const typename K::TA*>(st + K::XPITCH) +
+                                        warp * K::TW + 4 * lane);
             const float g[4] = {gf.x, gf.y, gf.z, gf.w};
             float v[4 * K::NV];
 #pragma unroll
             for (int q = 0; q < K::NV; ++q) {
-                const float4 f = xw[q];
+                const float4 f = IO::load4(xw + 4 * q);
                 v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
             }
             float acc[K::KW];
@@ -1048,7 +1054,7 @@ size_t rows_nchw_workspace(const Problem& p) {
 }
 
 template <class K>
-dw_status_t launch_rows_nchw(const Problem& p, const float* x, const float* dy, float* dw,
+dw_status_t launch_rows_nchw(const Problem& p, const void* x, const void* dy, float* dw,
                              float* db, void* ws, cudaStream_t stream, int32_t* err,
                              bool dry_run) {
     RArgs a;
@@ -1059,6 +1065,7 @@ dw_status_t launch_rows_nchw(const Problem& p, const float* x, const float* dy, 
     a.Ho = int(p.Ho);
     a.pt = p.pt;
     a.pl = p.pl;
+    a.sh4 = ((-p.pl) % K::ALIGN + K::ALIGN) % K::ALIGN - K::REM;  // 0 or 4
     const int64_t tx = (p.Wo + K::TW - 1) / K::TW;
     const int64_t cgroups = (p.C + K::NCW - 1) / K::NCW;
     int nper;
@@ -1081,18 +1088,18 @@ dw_status_t launch_rows_nchw(const Problem& p, const float* x, const float* dy, 
     if (G > units) G = units;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMap xmap, gmap;
+    constexpr cuuint64_t E = K::ESZ;
     const cuuint64_t xd[4] = {cuuint64_t(p.W), cuuint64_t(p.H), cuuint64_t(p.C), cuuint64_t(p.N)};
-    const cuuint64_t xs[3] = {cuuint64_t(p.W) * 4, cuuint64_t(p.W * p.H) * 4,
-                              cuuint64_t(p.W * p.H * p.C) * 4};
+    const cuuint64_t xs[3] = {cuuint64_t(p.W) * E, cuuint64_t(p.W * p.H) * E,
+                              cuuint64_t(p.W * p.H * p.C) * E};
     const cuuint32_t xbox[4] = {K::IWB, 1, K::NCW, 1};
     const cuuint64_t gd[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.C), cuuint64_t(p.N)};
-    const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * 4, cuuint64_t(p.Wo * p.Ho) * 4,
-                              cuuint64_t(p.Wo * p.Ho * p.C) * 4};
+    const cuuint64_t gs[3] = {cuuint64_t(p.Wo) * E, cuuint64_t(p.Wo * p.Ho) * E,
+                              cuuint64_t(p.Wo * p.Ho * p.C) * E};
     const cuuint32_t gbox[4] = {K::TW, 1, K::NCW, 1};
-    if (encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(x), xd, xs,
-                          xbox, estr) != CUDA_SUCCESS ||
-        encode_tensor_map(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(dy), gd, gs,
-                          gbox, estr) != CUDA_SUCCESS)
+    constexpr CUtensorMapDataType dt = ActIO<typename K::TA>::kTma;
+    if (encode_tensor_map(&xmap, dt, 4, const_cast<void*>(x), xd, xs, xbox, estr) != CUDA_SUCCESS ||
+        encode_tensor_map(&gmap, dt, 4, const_cast<void*>(dy), gd, gs, gbox, estr) != CUDA_SUCCESS)
         return DW_ERR_CUDA;
     if (launch_pdl(partial_rows_nchw<K>, dim3(unsigned(G)), dim3(K::NT), K::SMEM, stream, xmap,
                    gmap, a) != cudaSuccess)
@@ -1105,15 +1112,28 @@ dw_status_t launch_rows_nchw(const Problem& p, const float* x, const float* dy, 
     return cudaGetLastError() == cudaSuccess ? DW_OK : DW_ERR_CUDA;
 }
 
-template <int KW, int NS>
-dw_status_t launch_rows_rem(const Problem& p, const float* x, const float* dy, float* dw,
+template <int KW, int NS, class TA>
+dw_status_t launch_rows_rem(const Problem& p, const void* x, const void* dy, float* dw,
                             float* db, void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+#define DW_R(R) return launch_rows_nchw<RCfg<KW, R, NS, TA>>(p, x, dy, dw, db, ws, stream, err, dry_run);
     switch (((-p.pl) % 4 + 4) % 4) {
-        case 0: return launch_rows_nchw<RCfg<KW, 0, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        case 1: return launch_rows_nchw<RCfg<KW, 1, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        case 2: return launch_rows_nchw<RCfg<KW, 2, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
-        default: return launch_rows_nchw<RCfg<KW, 3, NS>>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        case 0: DW_R(0)
+        case 1: DW_R(1)
+        case 2: DW_R(2)
+        default: DW_R(3)
     }
+#undef DW_R
+}
+
+template <class TA>
+dw_status_t rows_pick(const Problem& p, const void* x, const void* dy, float* dw, float* db,
+                      void* ws, cudaStream_t stream, int32_t* err, bool dry_run) {
+    if (p.kW == 3) return launch_rows_rem<3, 8, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kW == 5) return launch_rows_rem<5, 8, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kW == 7) return launch_rows_rem<7, 8, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kW == 15) return launch_rows_rem<15, 8, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    if (p.kW == 31) return launch_rows_rem<31, 8, TA>(p, x, dy, dw, db, ws, stream, err, dry_run);
+    return DW_ERR_UNSUPPORTED;
 }
 
 constexpr int kNchwUnitsCap = 2048;  // bands are added until N*C*bands reaches this
@@ -1232,16 +1252,12 @@ dw_status_t tiled_pick_nchw(const Problem& p, const void* x, const void* dy, flo
         return DW_ERR_UNSUPPORTED;
     if (p.N >= INT_MAX || p.C >= INT_MAX || p.H >= INT_MAX || p.W >= INT_MAX) return DW_ERR_UNSUPPORTED;
     if (p.kH == 1) {
-        // rows of 1 x kW filters: float32 activations
-        if (p.sh != 1 || p.atype != DW_F32) return DW_ERR_UNSUPPORTED;
-        const float* xf = static_cast<const float*>(x);
-        const float* gf = static_cast<const float*>(dy);
-        if (p.kW == 3) return launch_rows_rem<3, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 5) return launch_rows_rem<5, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 7) return launch_rows_rem<7, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 15) return launch_rows_rem<15, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
-        if (p.kW == 31) return launch_rows_rem<31, 8>(p, xf, gf, dw, db, ws, stream, err, dry_run);
-        return DW_ERR_UNSUPPORTED;
+        // rows of 1 x kW filters
+        if (p.sh != 1) return DW_ERR_UNSUPPORTED;
+        if (p.atype == DW_F16) return rows_pick<__half>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        if (p.atype == DW_BF16)
+            return rows_pick<__nv_bfloat16>(p, x, dy, dw, db, ws, stream, err, dry_run);
+        return rows_pick<float>(p, x, dy, dw, db, ws, stream, err, dry_run);
     }
     if (p.atype == DW_F16) return tiled_pick_nchw_2d<__half>(p, x, dy, dw, db, ws, stream, err, dry_run);
     if (p.atype == DW_BF16)

@@ -165,7 +165,7 @@ def test_no_bias_gradient_and_small_workspace_error():
 
 # NCHW tiled weight gradient with 16-bit activations: every column phase of
 # the 16-byte x box (REM 0..3 and the extra 4-element shift), stride 2, 5x5,
-# 7x7 and a multiplier; float32 results, the same bits as the float32 call on
+# 7x7, a multiplier and the 1 x kW rows kernel; float32 results, the same bits as the float32 call on
 # the widened tensors (same kernel family, same summation order)
 HALF_NCHW = [
     Case("wh_3x3_same", 2, 37, 48, 6, 3, 3, layout="nchw", seed=91),
@@ -180,6 +180,12 @@ HALF_NCHW = [
     Case("wh_5x5", 2, 35, 48, 5, 5, 5, layout="nchw", seed=97),
     Case("wh_7x7", 2, 33, 32, 4, 7, 7, layout="nchw", seed=98),
     Case("wh_m2_3x3", 2, 21, 40, 3, 3, 3, multiplier=2, layout="nchw", seed=99),
+    # 1 x kW filters: the rows kernel
+    Case("wh_1x31", 3, 2, 296, 10, 1, 31, act="normal", layout="nchw", seed=103),
+    Case("wh_1x15_pad", 2, 3, 64, 11, 1, 15, padding=(0, 0, 6, 8), act="normal",
+         layout="nchw", seed=104),
+    Case("wh_1x7_pl5", 2, 2, 40, 9, 1, 7, padding=(0, 0, 5, 1), layout="nchw", seed=105),
+    Case("wh_1x3_pl4", 1, 3, 48, 12, 1, 3, padding=(0, 0, 4, 6), layout="nchw", seed=106),
 ]
 
 
