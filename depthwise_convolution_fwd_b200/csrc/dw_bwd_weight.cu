@@ -875,9 +875,37 @@ __global__ void __launch_bounds__(256) finalize_tiled_nchw(const double* __restr
 // pipeline stage holds that row of the 8 channels' planes (a 4-D TMA box of
 // one row by 8 channels, zero-filled past C).  Lanes run along W with 4
 // outputs each, the kW taps at compile-time offsets of a register window.
-// Each warp's float64 sums over its unit become one partial per
-// (n block, tap, channel), laid out as the direct partials are, so the same
-// fixed-order finalize sums the n blocks.
+// A lane accumulates float32 sums over kRowsFold strips (16 products per
+// tap), then a warp reduce-scatter (fixed butterfly order) leaves tap t's sum
+// on lane t, which adds it to its float64 total; each warp's totals over its
+// unit become one partial per (n block, tap, channel), laid out as the
+// direct partials are, so the same fixed-order finalize sums the n blocks.
+
+constexpr int kRowsFold = 4;  // strips per float32 partial sum
+
+// Warp reduce-scatter of NP (a power of two, <= 32) per-lane values: on
+// return lane l holds the sum over all 32 lanes of value l % NP.  The lane
+// bits above NP are summed first (every lane keeps all NP values), then each
+// round halves the values a lane keeps, the lane's bit choosing the half.
+template <int NP>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[NP], int lane) {
+    static_assert(NP >= 1 && NP <= 32 && (NP & (NP - 1)) == 0, "power of two up to 32");
+#pragma unroll
+    for (int o = 16; o >= NP; o >>= 1)
+#pragma unroll
+        for (int i = 0; i < NP; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+#pragma unroll
+    for (int h = NP / 2; h >= 1; h >>= 1) {
+        const bool up = (lane & h) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = up ? v[i] : v[i + h];
+            const float keep = up ? v[i + h] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, h);
+        }
+    }
+    return v[0];
+}
 
 struct RArgs {
     double* part;
@@ -897,6 +925,8 @@ struct RCfg {
     static constexpr int ALIGN = 16 / ESZ;  // x boxes start on 16-byte columns
     static constexpr int KW = KW_, REM = REM_, NS = NS_;
     static constexpr int T = KW + 1;
+    static constexpr int NP = T <= 4 ? 4 : T <= 8 ? 8 : T <= 16 ? 16 : 32;  // T rounded up to 2^k
+    static_assert(T <= 32, "taps + bias fit one warp");
     static constexpr int NCW = 8;  // consumer warps = channels per unit
     static constexpr int NT = NCW * 32 + 32;
     static constexpr int TW = 128;
@@ -981,13 +1011,16 @@ __global__ void __launch_bounds__(K::NT, 1)
         const int n0 = nb * a.nper;
         const int n1 = a.N - n0 < a.nper ? a.N : n0 + a.nper;
         const int c = cg * K::NCW + warp;
-        double acc64[K::T];
+        float acc[K::NP];  // float32 sums since the last fold (taps, then the bias)
 #pragma unroll
-        for (int t = 0; t < K::T; ++t) acc64[t] = 0.0;
+        for (int t = 0; t < K::NP; ++t) acc[t] = 0.f;
+        double total = 0.0;  // lane t: the unit's sum of tap t
         const int ntile = (n1 - n0) * a.Ho * a.tiles_x;
         for (int i = 0; i < ntile; ++i, ++k) {
             const int s = k % K::NS;
-            if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
+            // warp-uniform outcome: the fold below shuffles across the warp
+            const bool got = mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) {
                 if (lane == 0) {
                     *abort_flag = 1;
                     atomicExch(a.err, DW_ERR_DEVICE_TIMEOUT);
@@ -1008,28 +1041,25 @@ __global__ void __launch_bounds__(K::NT, 1)
                 const float4 f = IO::load4(xw + 4 * q);
                 v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
             }
-            float acc[K::KW];
 #pragma unroll
             for (int kw = 0; kw < K::KW; ++kw) {
-                float t0 = g[0] * v[K::REM + kw];
+                float t0 = fmaf(g[0], v[K::REM + kw], acc[kw]);
                 t0 = fmaf(g[1], v[K::REM + 1 + kw], t0);
                 t0 = fmaf(g[2], v[K::REM + 2 + kw], t0);
                 acc[kw] = fmaf(g[3], v[K::REM + 3 + kw], t0);
             }
+            acc[K::T - 1] += (g[0] + g[1]) + (g[2] + g[3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+            if ((i + 1) % kRowsFold == 0 || i + 1 == ntile) {
+                total += double(warp_reduce_scatter<K::NP>(acc, lane));
 #pragma unroll
-            for (int kw = 0; kw < K::KW; ++kw) acc64[kw] += double(acc[kw]);
-            acc64[K::T - 1] += double((g[0] + g[1]) + (g[2] + g[3]));
+                for (int t = 0; t < K::NP; ++t) acc[t] = 0.f;
+            }
         }
-        // the warp's sums over the unit, lanes combined in a fixed order
-#pragma unroll
-        for (int t = 0; t < K::T; ++t) {
-            double v = acc64[t];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0 && c < a.C) a.part[(int64_t(nb) * K::T + t) * a.C + c] = v;
-        }
+        if (failed) break;
+        // lane t (t < T) holds the unit's total of tap t
+        if (lane < K::T && c < a.C) a.part[(int64_t(nb) * K::T + lane) * a.C + c] = total;
     }
 }
 
