@@ -284,3 +284,43 @@ def test_selftest_rejects_bad_arguments(lib):
     # validation only: nothing is launched for these
     for mode, limit in ((2, 1000), (-1, 1000), (0, 0), (1, 2_000_000)):
         assert dw.selftest_wait_timeout_raw(mode, limit, 0) == dw.DW_ERR_INVALID_ARG
+
+
+def test_query_algo_multiplier_and_16bit_tiles(lib):
+    """Which family the multiplier and 16-bit calls run (dry-run dispatch):
+    the NHWC and NCHW multiplier tiles for every activation type, the
+    16-bit NCHW weight gradients, and the shapes that stay direct."""
+    T, D = dw.DW_ALGO_TILED, dw.DW_ALGO_DIRECT
+    base = 1 << 40
+    ins, w_, out = base, base + (1 << 34), base + (2 << 34)   # far apart: no aliasing
+
+    def qa(desc, op, atype=dw.DW_F32):
+        desc.atype = atype
+        if op == 2:   # (x, dy, dW)
+            return dw.dwconv2d_query_algo(desc, 2, ins, out, w_)
+        return dw.dwconv2d_query_algo(desc, op, ins, w_, out)
+
+    for at in (dw.DW_F32, dw.DW_F16, dw.DW_BF16):
+        # NHWC multiplier 2 and 4: forward, input gradient (stride 1 and 2), weight gradient
+        for m in (2, 4):
+            for s in (1, 2):
+                d = dw.make_desc(2, 32, 32, 16, 3, 3, stride=s, multiplier=m)
+                assert qa(d, 0, at) == T and qa(d, 1, at) == T and qa(d, 2, at) == T, (at, m, s)
+        assert qa(dw.make_desc(2, 32, 32, 16, 5, 5, multiplier=2), 0, at) == T
+        assert qa(dw.make_desc(2, 32, 32, 16, 3, 3, multiplier=3), 0, at) == D
+        # NCHW multiplier: forward fan-out / one plane per tile, summed-plane input gradient
+        for kh, m in ((3, 2), (3, 4), (5, 2), (7, 2)):
+            d = dw.make_desc(2, 32, 32, 16, kh, kh, multiplier=m, layout="nchw")
+            assert qa(d, 0, at) == T and qa(d, 1, at) == T and qa(d, 2, at) == T, (at, kh, m)
+        d = dw.make_desc(2, 32, 32, 16, 5, 5, multiplier=4, layout="nchw")
+        assert qa(d, 0, at) == T and qa(d, 1, at) == D
+        d = dw.make_desc(2, 32, 32, 16, 3, 3, stride=2, multiplier=2, layout="nchw")
+        assert qa(d, 0, at) == T and qa(d, 1, at) == D   # strided multiplier input gradient
+        # NCHW weight gradients, 2-D and 1 x kW, every activation type
+        assert qa(dw.make_desc(2, 16, 32, 32, 3, 3, layout="nchw"), 2, at) == T
+        assert qa(dw.make_desc(2, 16, 32, 32, 3, 3, stride=2, layout="nchw"), 2, at) == T
+        assert qa(dw.make_desc(2, 1, 64, 32, 1, 31, layout="nchw"), 2, at) == T
+    # 16-bit NCHW rows must be 16-byte multiples: W = 36 is for float32 only
+    assert qa(dw.make_desc(2, 16, 36, 32, 3, 3, layout="nchw"), 2, dw.DW_F32) == T
+    assert qa(dw.make_desc(2, 16, 36, 32, 3, 3, layout="nchw"), 2, dw.DW_F16) == D
+    assert qa(dw.make_desc(2, 1, 36, 32, 1, 15, layout="nchw"), 2, dw.DW_BF16) == D
