@@ -143,11 +143,11 @@ DW_API dw_status_t dwconv2d_out_shape(const dw_desc_t* desc, int64_t* Ho, int64_
 DW_API dw_status_t dwconv2d_resolved_pads(const dw_desc_t* desc, int32_t pads[4]);
 
 /*
- * Forward: y = depthwise(x; w) + b.
+ * Forward: y = depthwise(x; w) + b (Co = C*M output channels; Co = C at M = 1).
  *   x: [N,H,W,C] or [N,C,H,W] of desc->atype (float32 by default), read only.
- *   w: [C,kH,kW] float32 or float16 (desc->wtype), read only.
- *   b: [C] float32 or NULL, read only.
- *   y: [N,Ho,Wo,C] or [N,C,Ho,Wo] of desc->atype, every element written.
+ *   w: [Co,kH,kW] float32 or float16 (desc->wtype), read only.
+ *   b: [Co] float32 or NULL, read only.
+ *   y: [N,Ho,Wo,Co] or [N,Co,Ho,Wo] of desc->atype, every element written.
  * y must not overlap x, w or b (DW_ERR_ALIAS).
  * Page: LeanMlir Depthwise, "Depthwise conv2d forward"; strided forms
  * "Stride-2 SAME" / "Stride-2 XLA-SAME depthwise conv" (computed directly at
@@ -164,7 +164,7 @@ DW_API dw_status_t dwconv2d_fwd(const dw_desc_t* desc, const void* x, const void
  * to each output in registers before its single store, so y is written once
  * and never re-read.
  *   x, w, b, y: as for dwconv2d_fwd.
- *   gamma, beta, mean, var: [C] float32 each, read only; either all four are
+ *   gamma, beta, mean, var: [Co] float32 each, read only; either all four are
  *       given or all four are NULL (then BN is the identity and only the
  *       activation is applied).
  *   eps: finite, >= 0.
@@ -186,9 +186,10 @@ DW_API dw_status_t dwconv2d_fwd_bn_act(const dw_desc_t* desc, const void* x, con
                                        int32_t act, void* y, void* stream);
 
 /*
- * Input gradient: dx = J^T dy for the forward of `desc` (bias plays no part).
- *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] of desc->atype, read only.
- *   w:  [C,kH,kW] float32 or float16, read only.
+ * Input gradient: dx = J^T dy for the forward of `desc` (bias plays no part;
+ * with a multiplier, dx channel c sums its M output channels c*M ..).
+ *   dy: [N,Ho,Wo,Co] or [N,Co,Ho,Wo] of desc->atype, read only.
+ *   w:  [Co,kH,kW] float32 or float16, read only.
  *   dx: [N,H,W,C] or [N,C,H,W] of desc->atype, every element written (positions no
  *       output reads get 0; nothing is accumulated into previous contents).
  * dx must not overlap dy or w (DW_ERR_ALIAS).
@@ -200,16 +201,16 @@ DW_API dw_status_t dwconv2d_bwd_input(const dw_desc_t* desc, const void* dy, con
                                       void* dx, void* stream);
 
 /*
- * Weight and bias gradients of the forward of `desc`:
- *   dW[c,kh,kw] = sum_{n,ho,wo} dy[n,ho,wo,c] * X(n, ho*sh + kh*dh - pt,
- *                                                 wo*sw + kw*dw - pl, c)
- *   db[c]       = sum_{n,ho,wo} dy[n,ho,wo,c]
+ * Weight and bias gradients of the forward of `desc` (o < Co = C*M):
+ *   dW[o,kh,kw] = sum_{n,ho,wo} dy[n,ho,wo,o] * X(n, ho*sh + kh*dh - pt,
+ *                                                 wo*sw + kw*dw - pl, o/M)
+ *   db[o]       = sum_{n,ho,wo} dy[n,ho,wo,o]
  *   x:  [N,H,W,C] or [N,C,H,W] of desc->atype, read only.
- *   dy: [N,Ho,Wo,C] or [N,C,Ho,Wo] of desc->atype, read only.
- *   dw: [C,kH,kW] float32, every element written (also when desc->wtype is
+ *   dy: [N,Ho,Wo,Co] or [N,Co,Ho,Wo] of desc->atype, read only.
+ *   dw: [Co,kH,kW] float32, every element written (also when desc->wtype is
  *       DW_F16 or the activations are 16-bit: gradients are produced in
  *       float32).
- *   db: [C] float32 or NULL (then the bias gradient is not produced).
+ *   db: [Co] float32 or NULL (then the bias gradient is not produced).
  *   workspace: device memory of at least dwconv2d_bwd_weight_workspace_size()
  *       bytes, caller-owned; its contents on entry do not matter and are
  *       overwritten.
