@@ -17,8 +17,9 @@ namespace dw {
 namespace nhwc {
 
 // (KH KW S D TR | THT TWT WX WY NS | VEC NO MINB CB MULT TA)
+// float32: one CTA per SM (the 2-CTA register budget spills); 16-bit: two
 template <int M, class TA>
-using M33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4, 4, 0, 1, 32, M, TA>;  // one CTA per SM: no spills
+using M33s1 = Cfg<3, 3, 1, 1, false, 2, 4, 8, 4, 4, 4, 0, sizeof(TA) == 4 ? 1 : 2, 32, M, TA>;
 template <int M, class TA>
 using M33s2 = Cfg<3, 3, 2, 1, false, 1, 2, 8, 4, 4, 4, 0, 2, 32, M, TA>;
 template <int M, class TA>
