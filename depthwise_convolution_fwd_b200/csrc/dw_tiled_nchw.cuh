@@ -690,9 +690,12 @@ dw_status_t launch_chl(const Problem& p, const void* in, const void* w, const fl
 // ty*TH/2 + floor(pt/2) - AH and at the column tx*TW/2 + floor(pl/2) - AW,
 // moved left by REM (compile time) + sh4 (run time) to a 16-byte boundary.
 template <int KH_, int KW_, int PH_, int PW_, int REM_, int THT_, int WX_, int WY_, int NS_,
-          class TA_>
+          class TA_, int MP_ = 1>
 struct T2Cfg {
     using TA = TA_;
+    // channel multiplier: the box holds the MP dy planes c*MP .. of dx plane c,
+    // whose contributions are summed
+    static constexpr int MP = MP_;
     static constexpr int ESZ = sizeof(TA), ALIGN = 16 / ESZ;
     static constexpr int KH = KH_, KW = KW_, PH = PH_, PW = PW_, REM = REM_;
     static constexpr int THT = THT_, WX = WX_, WY = WY_, NS = NS_;
@@ -705,7 +708,7 @@ struct T2Cfg {
     static constexpr int IWB =
         ((TW / 2 - 4 + 4 * NV + (ALIGN - 4)) + ALIGN - 1) / ALIGN * ALIGN;
     static constexpr int RH = AH + (THT - 1 + PH) / 2 + 1;  // dy rows one thread reads
-    static constexpr int STAGE_BYTES = IWB * IH * ESZ;
+    static constexpr int STAGE_BYTES = IWB * IH * MP * ESZ;
     static constexpr int STAGE_PITCH = (STAGE_BYTES + 127) / 128 * 128;
     static constexpr size_t SMEM = size_t(NS) * STAGE_PITCH + size_t(2 * NS) * 8 + 16;
     static_assert(THT % 2 == 0 && (TW / 2) % ALIGN == 0, "even rows, aligned dy columns");
@@ -758,7 +761,7 @@ __global__ void __launch_bounds__(K::NT, 1)
                 mbar_arrive_expect_tx(&full[s], K::STAGE_BYTES);
                 tma_load_4d(smem + size_t(s) * K::STAGE_PITCH, &tmap, &full[s],
                             tx * (K::TW / 2) + a.pl - K::AW - K::REM - a.sh4,
-                            ty * (K::TH / 2) + a.pt - K::AH, c, n);
+                            ty * (K::TH / 2) + a.pt - K::AH, c * K::MP, n);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -773,7 +776,7 @@ __global__ void __launch_bounds__(K::NT, 1)
     const int xi = tid % K::WX;
     const int yi = tid / K::WX;
     const int row0 = yi * K::THT;  // first dx row of this thread in the tile (even)
-    float wr[K::KH][K::KW];
+    float wr[K::MP][K::KH][K::KW];
     int cur_key = -1;
     bool live = false;
     int k = 0;
@@ -785,12 +788,17 @@ __global__ void __launch_bounds__(K::NT, 1)
         if (key != cur_key) {
             cur_key = key;
             live = c < a.C;
-            const int64_t base = int64_t(live ? c : 0) * (K::KH * K::KW);
 #pragma unroll
-            for (int kh = 0; kh < K::KH; ++kh)
+            for (int m = 0; m < K::MP; ++m) {
+                // filter of output channel c*MP + m
+                const int64_t base = (int64_t(live ? c : 0) * K::MP + m) * (K::KH * K::KW);
 #pragma unroll
-                for (int kw = 0; kw < K::KW; ++kw)
-                    wr[kh][kw] = live ? load_weight(a.w, a.wtype, base + kh * K::KW + kw) : 0.f;
+                for (int kh = 0; kh < K::KH; ++kh)
+#pragma unroll
+                    for (int kw = 0; kw < K::KW; ++kw)
+                        wr[m][kh][kw] =
+                            live ? load_weight(a.w, a.wtype, base + kh * K::KW + kw) : 0.f;
+            }
         }
         if (!mbar_wait_or_abort(&full[s], (k / K::NS) & 1, abort_flag)) {
             if (lane == 0) {
@@ -805,33 +813,38 @@ __global__ void __launch_bounds__(K::NT, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
         // dy row (row0/2 + rr) of the box and the lane's dy columns from 4*xi
-        const TA* win = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
-                        size_t(row0 / 2) * K::IWB + 4 * xi + a.sh4;
-        static_for<0, K::RH>([&](auto rr_) {
-            constexpr int rr = decltype(rr_)::value;
-            float v[4 * K::NV];
+        const TA* win0 = reinterpret_cast<const TA*>(smem + size_t(s) * K::STAGE_PITCH) +
+                         size_t(row0 / 2) * K::IWB + 4 * xi + a.sh4;
+        static_for<0, K::MP>([&](auto m_) {
+            constexpr int m = decltype(m_)::value;
+            const TA* win = win0 + size_t(m) * K::IH * K::IWB;  // dy plane c*MP + m
+            static_for<0, K::RH>([&](auto rr_) {
+                constexpr int rr = decltype(rr_)::value;
+                float v[4 * K::NV];
 #pragma unroll
-            for (int u = 0; u < K::NV; ++u) {
-                const float4 f = IO::load4(win + rr * K::IWB + 4 * u);
-                v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
-            }
-            static_for<0, K::THT>([&](auto j_) {
-                constexpr int j = decltype(j_)::value;
-                static_for<0, K::KH>([&](auto kh_) {
-                    constexpr int kh = decltype(kh_)::value;
-                    // dx row row0 + j reads dy box row row0/2 + (j + PH - kh)/2 + AH
-                    constexpr int num = j + K::PH - kh;
-                    if constexpr (num % 2 == 0 && num / 2 + K::AH == rr) {
-                        static_for<0, 8>([&](auto e_) {
-                            constexpr int e = decltype(e_)::value;
-                            static_for<0, K::KW>([&](auto kw_) {
-                                constexpr int kw = decltype(kw_)::value;
-                                constexpr int numw = e + K::PW - kw;
-                                if constexpr (((numw % 2) + 2) % 2 == 0)
-                                    acc[j][e] = fmaf(wr[kh][kw], v[numw / 2 + K::AW + K::REM], acc[j][e]);
+                for (int u = 0; u < K::NV; ++u) {
+                    const float4 f = IO::load4(win + rr * K::IWB + 4 * u);
+                    v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
+                }
+                static_for<0, K::THT>([&](auto j_) {
+                    constexpr int j = decltype(j_)::value;
+                    static_for<0, K::KH>([&](auto kh_) {
+                        constexpr int kh = decltype(kh_)::value;
+                        // dx row row0 + j reads dy box row row0/2 + (j + PH - kh)/2 + AH
+                        constexpr int num = j + K::PH - kh;
+                        if constexpr (num % 2 == 0 && num / 2 + K::AH == rr) {
+                            static_for<0, 8>([&](auto e_) {
+                                constexpr int e = decltype(e_)::value;
+                                static_for<0, K::KW>([&](auto kw_) {
+                                    constexpr int kw = decltype(kw_)::value;
+                                    constexpr int numw = e + K::PW - kw;
+                                    if constexpr (((numw % 2) + 2) % 2 == 0)
+                                        acc[j][e] = fmaf(wr[m][kh][kw],
+                                                         v[numw / 2 + K::AW + K::REM], acc[j][e]);
+                                });
                             });
-                        });
-                    }
+                        }
+                    });
                 });
             });
         });
@@ -870,10 +883,11 @@ dw_status_t launch_t2(const Problem& p, const void* in, const void* w, void* out
     a.out = out;
     a.err = err;
     a.wtype = p.wtype;
-    if (p.M != 1) return DW_ERR_UNSUPPORTED;
+    if (p.M != K::MP) return DW_ERR_UNSUPPORTED;
     a.M = 1;
     a.N = int(p.N);
     a.C = int(p.C);
+    a.Cout = int(p.C);
     a.Hout = int(p.H);
     a.Wout = int(p.W);
     a.pt = p.pt / 2;  // floor(pt/2), floor(pl/2): the parities are template parameters
@@ -894,10 +908,11 @@ dw_status_t launch_t2(const Problem& p, const void* in, const void* w, void* out
     if (occ < 1) return DW_ERR_CUDA;
     CUtensorMap map;
     constexpr cuuint64_t E = K::ESZ;
-    const cuuint64_t dims[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.C), cuuint64_t(p.N)};
+    // dy: Co = C*MP planes
+    const cuuint64_t dims[4] = {cuuint64_t(p.Wo), cuuint64_t(p.Ho), cuuint64_t(p.Co), cuuint64_t(p.N)};
     const cuuint64_t strides[3] = {cuuint64_t(p.Wo) * E, cuuint64_t(p.Wo * p.Ho) * E,
-                                   cuuint64_t(p.Wo * p.Ho * p.C) * E};
-    const cuuint32_t box[4] = {K::IWB, K::IH, 1, 1};
+                                   cuuint64_t(p.Wo * p.Ho * p.Co) * E};
+    const cuuint32_t box[4] = {K::IWB, K::IH, K::MP, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     if (encode_tensor_map(&map, ActIO<typename K::TA>::kTma, 4, const_cast<void*>(in), dims,
                           strides, box, estr) != CUDA_SUCCESS)
@@ -911,7 +926,7 @@ dw_status_t launch_t2(const Problem& p, const void* in, const void* w, void* out
 }
 
 // dispatch on the pad parities and the box remainder
-template <int KH, int KW, int THT, int WX, int WY, int NS, class TA>
+template <int KH, int KW, int THT, int WX, int WY, int NS, class TA, int MP = 1>
 dw_status_t launch_t2_any(const Problem& p, const void* in, const void* w, void* out,
                           cudaStream_t stream, int32_t* err, bool dry_run) {
     constexpr int align = 16 / int(sizeof(TA));
@@ -919,7 +934,7 @@ dw_status_t launch_t2_any(const Problem& p, const void* in, const void* w, void*
     const int rem = full % 4, sh4 = full - rem;
     const int par = (p.pt & 1) * 2 + (p.pl & 1);
 #define DW_T2(PH, PW, R) \
-    return launch_t2<T2Cfg<KH, KW, PH, PW, R, THT, WX, WY, NS, TA>>(p, in, w, out, stream, err, dry_run, sh4);
+    return launch_t2<T2Cfg<KH, KW, PH, PW, R, THT, WX, WY, NS, TA, MP>>(p, in, w, out, stream, err, dry_run, sh4);
 #define DW_T2R(PH, PW) \
     switch (rem) { case 0: DW_T2(PH, PW, 0) case 1: DW_T2(PH, PW, 1) case 2: DW_T2(PH, PW, 2) default: DW_T2(PH, PW, 3) }
     switch (par) {
@@ -1053,8 +1068,10 @@ dw_status_t nchw_launch_t(const Problem& p, Op op, const void* in, const void* w
                 return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA, 1, 2>(p, in, w, b, out, stream, err, dry_run);
             return launch_s2_fwd<3, 3, 2, 16, 16, 4, TA>(p, in, w, b, out, stream, err, dry_run);
         }
-        if (op == OP_BWD_INPUT && p.kH == 3 && p.kW == 3) {
-            //                            KH KW THT WX WY NS
+        if (op == OP_BWD_INPUT && p.kH == 3 && p.kW == 3 && (p.M == 1 || p.M == 2)) {
+            //                                           KH KW THT WX WY NS
+            if (p.M == 2 && p.W <= 64) return launch_t2_any<3, 3, 4, 8, 16, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
+            if (p.M == 2) return launch_t2_any<3, 3, 4, 16, 16, 4, TA, 2>(p, in, w, out, stream, err, dry_run);
             if (p.W <= 64) return launch_t2_any<3, 3, 4, 8, 16, 4, TA>(p, in, w, out, stream, err, dry_run);
             return launch_t2_any<3, 3, 4, 16, 16, 4, TA>(p, in, w, out, stream, err, dry_run);
         }

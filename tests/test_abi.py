@@ -315,7 +315,9 @@ def test_query_algo_multiplier_and_16bit_tiles(lib):
         d = dw.make_desc(2, 32, 32, 16, 5, 5, multiplier=4, layout="nchw")
         assert qa(d, 0, at) == T and qa(d, 1, at) == D
         d = dw.make_desc(2, 32, 32, 16, 3, 3, stride=2, multiplier=2, layout="nchw")
-        assert qa(d, 0, at) == T and qa(d, 1, at) == D   # strided multiplier input gradient
+        assert qa(d, 0, at) == T and qa(d, 1, at) == T   # strided: M dy planes per box
+        d = dw.make_desc(2, 32, 32, 16, 3, 3, stride=2, multiplier=4, layout="nchw")
+        assert qa(d, 1, at) == D
         # NCHW weight gradients, 2-D and 1 x kW, every activation type
         assert qa(dw.make_desc(2, 16, 32, 32, 3, 3, layout="nchw"), 2, at) == T
         assert qa(dw.make_desc(2, 16, 32, 32, 3, 3, stride=2, layout="nchw"), 2, at) == T

@@ -212,7 +212,7 @@ def test_nchw_multiplier_input_gradient_tiles(case):
 
 
 @pytest.mark.parametrize("name", ["f16", "bf16"])
-@pytest.mark.parametrize("case", [NCHW_BWD[0], NCHW_TILED[1]], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", [NCHW_BWD[0], NCHW_TILED[1], NCHW_TILED[3]], ids=lambda c: c.name)
 def test_nchw_multiplier_half(case, name):
     from tests import test_gpu_half_activations as ha
     dt, _ = ha.DTYPES[name]
@@ -224,7 +224,7 @@ def test_nchw_multiplier_half(case, name):
     desc.atype = {"f16": dw.DW_F16, "bf16": dw.DW_BF16}[name]
     wp = inp["w"].cuda().data_ptr()
     assert dw.dwconv2d_query_algo(desc, 0, x.data_ptr(), wp, y.data_ptr()) == dw.DW_ALGO_TILED
-    if case in NCHW_BWD:
+    if case in NCHW_BWD or case.stride == 2:
         assert dw.dwconv2d_query_algo(desc, 1, y.data_ptr(), wp, x.data_ptr()) == dw.DW_ALGO_TILED
     ha.run_case(case, name, "auto")
 
