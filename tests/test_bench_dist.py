@@ -85,3 +85,24 @@ def test_reference_arm_prints_contract_line():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_algorithmic_bytes_hand_values():
+    """The roofline numerator: input read once, output written once, filters
+    and bias read once (hand arithmetic for the headline shapes)."""
+    import bench
+    from depthwise_convolution_fwd_b200.workloads import Case
+    # MobileNet stride-2 layer: 32x56x56x144 -> 28x28, float32
+    c = Case("m3", 32, 56, 56, 144, 3, 3, stride=2, padding=1)
+    x, y = 32 * 56 * 56 * 144 * 4, 32 * 28 * 28 * 144 * 4
+    assert bench.algorithmic_bytes(c, 28, 28, "fwd") == x + y + 144 * 9 * 4 + 144 * 4
+    assert bench.algorithmic_bytes(c, 28, 28, "bwd") == x + y + 144 * 9 * 4
+    assert bench.algorithmic_bytes(c, 28, 28, "wgrad") == x + y + 144 * 9 * 4 + 144 * 4
+    assert bench.algorithmic_bytes(c, 28, 28, "fused") == x + y + 144 * 9 * 4 + 144 * 4 + 16 * 144
+    # 512x512x256 3x3 with float16 weights and bfloat16 activations
+    c = Case("l", 1, 512, 512, 256, 3, 3, wtype="f16")
+    a = 512 * 512 * 256
+    assert bench.algorithmic_bytes(c, 512, 512, "fwd", esz=2) == 2 * (2 * a) + 256 * 9 * 2 + 256 * 4
+    # channel multiplier 2: 128 input channels, 256 outputs and filters
+    c = Case("m", 1, 512, 512, 128, 3, 3, multiplier=2)
+    assert bench.algorithmic_bytes(c, 512, 512, "bwd") == 4 * (512 * 512 * (128 + 256)) + 256 * 9 * 4
